@@ -1,0 +1,233 @@
+"""fp64 CPU oracle of the hybrid attention chunk step.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import or call this
+module: only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` use it. It shares no code with the CUDA path and imports nothing
+from the package.
+
+Every function is a plain, literal statement of the definition it cites, in
+float64 numpy, on inputs that the caller widens exactly from bf16. A library
+matmul is used as a step where the definition is a matrix product; there is no
+blocking, fusion or reordering beyond what the definitions state.
+
+Sources (page title, then the section used):
+  [HF-de]  "Long-Horizon Streaming Video Generation via Hybrid Attention with
+           Decoupled Distillation", German technical summary (gist.science),
+           §2 Methodik, A. Hybride Aufmerksamkeitsmechanismen.
+  [HF-abs] the same title, English abstract (arxivdaily.com).
+  [HF-pt]  the same title, Portuguese technical summary (gist.science),
+           §2 Metodologia, A. Mecanismo de Atenção Híbrida.
+  [LF]     "Light Forcing: Accelerating Autoregressive Video Diffusion via
+           Sparse Attention", German technical summary (gist.science),
+           §2.2 Hierarchische Spärliche Attention (token compression by mean
+           pooling; per-query-block selection).
+
+The pages give the structure (a compact KV state absorbing evicted tokens
+through a linear attention function; Top-K block-sparse attention inside the
+window; output = sum of both) but no formulas. The step's specification fixes
+the open parts, and this oracle follows them:
+  * phi(x) = elu(x) + 1, i.e. x + 1 for x > 0 and exp(x) otherwise;
+  * flat key/query blocks of ``block`` tokens over the flattened sequence, the
+    last block possibly partial;
+  * pooled block score s_IJ = mean(q in I) . mean(k in J), unscaled;
+  * each query block keeps its top-r key blocks, ties to the lower index,
+    emitted in ascending order;
+  * sparse softmax attention over the valid tokens of the kept blocks with
+    scale 1/sqrt(d), no causal mask inside the window;
+  * linear readout phi(q) S / (phi(q) . z + 1e-6);
+  * state update S += phi(K)^T V, z += sum_t phi(k_t).
+
+Parity pins: each function is checked in ``tests/test_oracle_pins.py`` against
+closed forms, brute force, library routines and hand-derived fixtures; none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+READOUT_EPS = 1e-6
+
+__all__ = [
+    "READOUT_EPS", "phi", "block_ranges", "pool_blocks", "block_scores",
+    "select_blocks", "sparse_attention_tile", "sparse_attention", "linear_readout",
+    "hybrid_attention", "hybrid_attention_tile", "absorb", "absorb_batch",
+    "dense_swa", "default_scale",
+]
+
+
+def _f64(x) -> np.ndarray:
+    a = np.asarray(x, dtype=np.float64)
+    return a
+
+
+def default_scale(d: int) -> float:
+    """Softmax scale 1/sqrt(d) (textbook attention; the pages give none)."""
+    return 1.0 / math.sqrt(d)
+
+
+def phi(x) -> np.ndarray:
+    """Feature map of the linear temporal attention: elu(x) + 1.
+
+    elu(x) = x for x > 0 and exp(x) - 1 otherwise, so phi(x) = x + 1 (x > 0),
+    exp(x) (x <= 0); phi > 0 everywhere. [HF-de] §2A (linear attention function);
+    the map itself is the specification's choice.
+    """
+    x = _f64(x)
+    return np.where(x > 0.0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def block_ranges(n: int, block: int) -> list[tuple[int, int]]:
+    """Token ranges [t*block, min((t+1)*block, n)) of the ceil(n/block) blocks."""
+    return [(t * block, min((t + 1) * block, n)) for t in range(-(-n // block))]
+
+
+def pool_blocks(X, block: int) -> np.ndarray:
+    """Mean of the valid tokens of every block: [B,H,N,d] -> [B,H,ceil(N/block),d].
+
+    [LF] §2.2: query and key tokens are compressed by mean pooling at block level.
+    """
+    X = _f64(X)
+    B, H, N, d = X.shape
+    out = np.empty((B, H, -(-N // block), d), dtype=np.float64)
+    for t, (lo, hi) in enumerate(block_ranges(N, block)):
+        out[:, :, t, :] = X[:, :, lo:hi, :].mean(axis=2)
+    return out
+
+
+def block_scores(Q, K, block: int) -> np.ndarray:
+    """s[b,h,I,J] = pooled(Q)[I] . pooled(K)[J] (unscaled), [B,H,nQB,nKB]."""
+    Qp = pool_blocks(Q, block)
+    Kp = pool_blocks(K, block)
+    return Qp @ np.swapaxes(Kp, -1, -2)
+
+
+def select_blocks(Q, K, block: int, r: int):
+    """Top-r key blocks of every query block.
+
+    For each (b, h, I), the key blocks J are ordered by decreasing s_IJ, equal
+    scores by increasing J; the first r are kept and returned in ascending J.
+    [HF-de] §2A (only the most important, Top-K, blocks are computed);
+    [LF] §2.2 (selection per query block from pooled scores).
+
+    Returns (idx int32 [B,H,nQB,r], scores float64 [B,H,nQB,nKB]).
+    """
+    s = block_scores(Q, K, block)
+    B, H, nQB, nKB = s.shape
+    if not 1 <= r <= nKB:
+        raise ValueError(f"r={r} outside [1, {nKB}]")
+    idx = np.empty((B, H, nQB, r), dtype=np.int32)
+    order_key = np.arange(nKB)
+    for b in range(B):
+        for h in range(H):
+            for I in range(nQB):
+                # lexsort sorts by the last key first: -s descending score, then J.
+                order = np.lexsort((order_key, -s[b, h, I]))
+                idx[b, h, I] = np.sort(order[:r])
+    return idx, s
+
+
+def _selected_tokens(kept_blocks, Nk: int, block: int) -> np.ndarray:
+    ranges = block_ranges(Nk, block)
+    return np.concatenate([np.arange(*ranges[int(J)]) for J in kept_blocks])
+
+
+def sparse_attention_tile(Q, K, V, idx, block: int, b: int, h: int, I: int,
+                          scale: float | None = None) -> np.ndarray:
+    """Softmax attention of query block I over the valid tokens of its kept blocks.
+
+    O_i = sum_j softmax_j(scale * q_i . k_j) v_j, j over the tokens of the key
+    blocks idx[b,h,I]; exact softmax (max-subtracted), not an online one.
+    [HF-de] §2A (block-sparse attention inside the local window);
+    [HF-pt] §2A.2.
+    Returns [L_I, d] float64.
+    """
+    Q = np.asarray(Q)
+    K = np.asarray(K)
+    V = np.asarray(V)
+    d = Q.shape[-1]
+    scale = default_scale(d) if scale is None else float(scale)
+    lo, hi = block_ranges(Q.shape[2], block)[I]
+    q = _f64(Q[b, h, lo:hi])
+    toks = _selected_tokens(idx[b, h, I], K.shape[2], block)
+    k = _f64(K[b, h, toks])
+    v = _f64(V[b, h, toks])
+    a = scale * (q @ k.T)
+    m = a.max(axis=1, keepdims=True)
+    p = np.exp(a - m)
+    return (p @ v) / p.sum(axis=1, keepdims=True)
+
+
+def sparse_attention(Q, K, V, idx, block: int, scale: float | None = None) -> np.ndarray:
+    """Sparse term O_s for all query blocks, [B,H,Nq,d] float64."""
+    B, H, Nq, d = np.shape(Q)
+    out = np.empty((B, H, Nq, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(H):
+            for I, (lo, hi) in enumerate(block_ranges(Nq, block)):
+                out[b, h, lo:hi] = sparse_attention_tile(Q, K, V, idx, block, b, h, I, scale)
+    return out
+
+
+def linear_readout(Q, S, z) -> np.ndarray:
+    """Linear term O_lin = phi(q)^T S / (phi(q) . z + 1e-6).
+
+    Q [..., N, d], S [..., d, d] (S[k, n] = sum_t phi(k_t)[k] v_t[n]), z [..., d].
+    [HF-de] §2A and [HF-abs] (compact key-value state read by linear attention);
+    the normalised form with 1e-6 is the specification's.
+    """
+    ph = phi(Q)
+    S = _f64(S)
+    z = _f64(z)
+    num = ph @ S
+    den = (ph @ z[..., :, None]) + READOUT_EPS
+    return num / den
+
+
+def hybrid_attention_tile(Q, K, V, idx, S, z, block: int, b: int, h: int, I: int,
+                          scale: float | None = None) -> np.ndarray:
+    """Output rows of query block I: O = O_s + O_lin ([HF-de] §2A Kombination; [HF-pt] §2A)."""
+    lo, hi = block_ranges(np.shape(Q)[2], block)[I]
+    o_s = sparse_attention_tile(Q, K, V, idx, block, b, h, I, scale)
+    o_l = linear_readout(np.asarray(Q)[b, h, lo:hi], np.asarray(S)[b, h], np.asarray(z)[b, h])
+    return o_s + o_l
+
+
+def hybrid_attention(Q, K, V, idx, S, z, block: int, scale: float | None = None) -> np.ndarray:
+    """O = sparse term + linear term for every query, [B,H,Nq,d] float64."""
+    return sparse_attention(Q, K, V, idx, block, scale) + linear_readout(Q, S, z)
+
+
+def absorb(S, z, K_ev, V_ev):
+    """State after absorbing evicted tokens: S + phi(K)^T V, z + sum_t phi(k_t).
+
+    S [B,H,d,d], z [B,H,d], K_ev/V_ev [B,H,Ne,d]. [HF-de] §2A (evicted frames are
+    aggregated into the compact state by a linear attention function);
+    [HF-abs] (incremental absorption of evicted tokens); [HF-pt] §2A.1.
+    Returns new (S, z); the inputs are not modified.
+    """
+    pk = phi(K_ev)
+    v = _f64(V_ev)
+    return _f64(S) + np.swapaxes(pk, -1, -2) @ v, _f64(z) + pk.sum(axis=-2)
+
+
+def absorb_batch(K_ev, V_ev):
+    """State built in one go from an empty state (S = 0, z = 0)."""
+    B, H, _, d = np.shape(K_ev)
+    return absorb(np.zeros((B, H, d, d)), np.zeros((B, H, d)), K_ev, V_ev)
+
+
+def dense_swa(Q, K, V, scale: float | None = None) -> np.ndarray:
+    """Dense sliding-window attention: softmax(scale * Q K^T) V over all window keys.
+
+    [HF-de] §1 (SWA with KV caching), the dense case the block-sparse form replaces.
+    """
+    Q = _f64(Q)
+    K = _f64(K)
+    V = _f64(V)
+    scale = default_scale(Q.shape[-1]) if scale is None else float(scale)
+    a = scale * (Q @ np.swapaxes(K, -1, -2))
+    a = a - a.max(axis=-1, keepdims=True)
+    p = np.exp(a)
+    return (p @ V) / p.sum(axis=-1, keepdims=True)

@@ -1,0 +1,272 @@
+"""Pins of the fp64 oracle against things other than itself.
+
+Each ``check_*`` takes an oracle namespace (the real module, or a copy with a
+planted mistake) and raises AssertionError when the oracle disagrees with:
+hand-derived worked examples (tests/golden/hand_examples.json), brute-force
+enumeration, closed forms, invariants, or a library routine (torch float64).
+``tests/test_oracle_pins.py`` runs them on the real oracle and checks that every
+planted mistake is caught by at least one of them.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hand_examples.json")
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _as4(x):
+    """[N, d] -> [1, 1, N, d] float64."""
+    return np.asarray(x, dtype=np.float64)[None, None]
+
+
+# ---------------------------------------------------------------------------
+# phi
+# ---------------------------------------------------------------------------
+def check_phi_library(o):
+    """phi = torch's elu + 1 (float64) on a grid spanning both branches and 0."""
+    x = np.concatenate([np.linspace(-20, 20, 4001), [0.0, -0.0, 1e-300, -1e-300, 88.0, -700.0]])
+    ref = torch.nn.functional.elu(torch.from_numpy(x)).numpy() + 1.0
+    got = o.phi(x)
+    # elu(x) + 1 = (exp(x) - 1) + 1 carries ~1e-16 absolute cancellation error for x < 0
+    assert np.allclose(got, ref, rtol=1e-15, atol=4e-16), "phi != elu + 1"
+    neg = x < -1.0
+    assert np.allclose(got[neg], np.exp(x[neg]), rtol=1e-15, atol=0.0), "phi(x<=0) != exp(x)"
+    assert np.all(got > 0.0), "phi must be positive"
+
+
+# ---------------------------------------------------------------------------
+# pooling and selection
+# ---------------------------------------------------------------------------
+def check_pool_by_hand(o):
+    """Block means over valid rows, written out with python loops on a ragged case."""
+    rng = np.random.default_rng(5)
+    X = rng.integers(-4, 5, size=(1, 2, 7, 3)).astype(np.float64)
+    block = 3
+    got = o.pool_blocks(X, block)
+    assert got.shape == (1, 2, 3, 3)
+    for h in range(2):
+        for t, (lo, hi) in enumerate([(0, 3), (3, 6), (6, 7)]):
+            for c in range(3):
+                s = 0.0
+                for i in range(lo, hi):
+                    s += X[0, h, i, c]
+                assert abs(got[0, h, t, c] - s / (hi - lo)) < 1e-14
+
+
+def check_selection_golden(o):
+    g = _golden()["selection"]
+    Q, K, block = _as4(g["Q"]), _as4(g["K"]), g["block"]
+    s = o.block_scores(Q, K, block)[0, 0, 0]
+    assert np.allclose(s, g["scores"], atol=1e-15, rtol=0), f"scores {s}"
+    for r, want in g["idx_by_r"].items():
+        idx, _ = o.select_blocks(Q, K, block, int(r))
+        assert idx[0, 0, 0].tolist() == want, f"r={r}: {idx[0, 0, 0].tolist()} != {want}"
+
+
+def _brute_force_topr(s, r):
+    """The unique size-r set M with: for j in M, j' not in M, s_j > s_j' or (s_j == s_j' and j < j')."""
+    n = len(s)
+    found = []
+    for M in itertools.combinations(range(n), r):
+        Ms = set(M)
+        ok = all((s[j] > s[jj]) or (s[j] == s[jj] and j < jj)
+                 for j in M for jj in range(n) if jj not in Ms)
+        if ok:
+            found.append(list(M))
+    assert len(found) == 1, f"expected exactly one dominant subset, got {found}"
+    return found[0]
+
+
+def check_selection_bruteforce(o):
+    """Brute force over all C(nKB, r) subsets, integer scores so that ties are common."""
+    rng = np.random.default_rng(11)
+    nKB, d = 8, 4
+    for trial in range(12):
+        # one 1-token query block q = e0 and 1-token key blocks with k[0] = score:
+        # pooled score s_J = k_J[0] exactly.
+        sc = rng.integers(-3, 4, size=nKB).astype(np.float64)
+        Q = np.zeros((1, 1, 1, d))
+        Q[0, 0, 0, 0] = 1.0
+        K = rng.normal(size=(1, 1, nKB, d))
+        K[0, 0, :, 0] = sc
+        for r in range(1, nKB + 1):
+            idx, s = o.select_blocks(Q, K, 1, r)
+            assert np.array_equal(s[0, 0, 0], sc)
+            assert idx[0, 0, 0].tolist() == _brute_force_topr(sc.tolist(), r), (trial, r)
+
+
+def check_selection_ties_constructed(o):
+    """Duplicated key blocks give exactly equal pooled scores: the lower index wins."""
+    rng = np.random.default_rng(3)
+    block, d = 4, 8
+    base = rng.normal(size=(6, block, d))
+    # key blocks 0..11 where block 6+i duplicates block i
+    Kb = np.concatenate([base, base], axis=0)
+    K = Kb.reshape(1, 1, 12 * block, d)
+    Q = rng.normal(size=(1, 1, 2 * block, d))
+    _, s = o.select_blocks(Q, K, block, 1)
+    for I in range(2):
+        for r in range(1, 13):
+            idx, _ = o.select_blocks(Q, K, block, r)
+            got = idx[0, 0, I].tolist()
+            assert got == _brute_force_topr(s[0, 0, I].tolist(), r)
+            # with duplicates, a kept upper copy implies its lower twin is kept
+            for J in got:
+                if J >= 6:
+                    assert J - 6 in got
+
+
+def check_selection_output_form(o):
+    rng = np.random.default_rng(9)
+    Q = rng.normal(size=(2, 3, 70, 16))
+    K = rng.normal(size=(2, 3, 150, 16))
+    idx, s = o.select_blocks(Q, K, 32, 3)
+    assert idx.shape == (2, 3, 3, 3) and idx.dtype == np.int32
+    assert s.shape == (2, 3, 3, 5)
+    assert np.all(np.diff(idx, axis=-1) > 0), "kept blocks must be ascending and distinct"
+    assert idx.min() >= 0 and idx.max() < 5
+
+
+# ---------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------
+def check_attention_golden(o):
+    g = _golden()["attention"]
+    Q, K, V = _as4(g["Q"]), _as4(g["K"]), _as4(g["V"])
+    idx = np.asarray(g["idx"], dtype=np.int32)[None, None, None, :]
+    got = o.sparse_attention(Q, K, V, idx, g["block"])[0, 0, 0]
+    assert np.allclose(got, g["O"], atol=1e-12, rtol=0), f"{got} != {g['O']}"
+
+
+def check_attention_dense_equivalence(o):
+    """With every block kept the sparse term equals dense attention: the oracle's own
+    dense form and torch's float64 scaled_dot_product_attention."""
+    rng = np.random.default_rng(21)
+    B, H, Nq, Nk, d, block = 1, 2, 45, 100, 16, 16  # ragged query and key tails
+    Q, K, V = (rng.normal(size=(B, H, n, d)) for n in (Nq, Nk, Nk))
+    nKB = -(-Nk // block)
+    idx, _ = o.select_blocks(Q, K, block, nKB)
+    assert idx[0, 0, 0].tolist() == list(range(nKB))
+    sp = o.sparse_attention(Q, K, V, idx, block)
+    dn = o.dense_swa(Q, K, V)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q), torch.from_numpy(K), torch.from_numpy(V)).numpy()
+    assert np.allclose(sp, ref, atol=1e-12, rtol=0), np.abs(sp - ref).max()
+    assert np.allclose(dn, ref, atol=1e-12, rtol=0), np.abs(dn - ref).max()
+
+
+def check_attention_subset_library(o):
+    """A proper subset of blocks equals torch SDPA over exactly those keys."""
+    rng = np.random.default_rng(22)
+    Nq, Nk, d, block = 20, 77, 8, 8
+    Q, K, V = (rng.normal(size=(1, 1, n, d)) for n in (Nq, Nk, Nk))
+    keep = [1, 4, 9]  # block 9 is the 5-token partial tail
+    idx = np.tile(np.asarray(keep, dtype=np.int32), (1, 1, 3, 1))
+    toks = np.concatenate([np.arange(J * block, min((J + 1) * block, Nk)) for J in keep])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q), torch.from_numpy(K[:, :, toks]), torch.from_numpy(V[:, :, toks])).numpy()
+    got = o.sparse_attention(Q, K, V, idx, block)
+    assert np.allclose(got, ref, atol=1e-12, rtol=0)
+
+
+def check_attention_identical_keys(o):
+    """Identical keys in the kept blocks give uniform weights: O = mean of their v."""
+    rng = np.random.default_rng(23)
+    Nq, Nk, d, block = 8, 32, 4, 8
+    Q = rng.normal(size=(1, 1, Nq, d))
+    K = np.tile(rng.normal(size=(1, 1, 1, d)), (1, 1, Nk, 1))
+    V = rng.normal(size=(1, 1, Nk, d))
+    idx = np.asarray([[[[0, 3]]]], dtype=np.int32)
+    got = o.sparse_attention(Q, K, V, idx, block)
+    want = np.concatenate([V[0, 0, 0:8], V[0, 0, 24:32]]).mean(axis=0)
+    assert np.allclose(got[0, 0], want[None, :], atol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# readout and absorption
+# ---------------------------------------------------------------------------
+def check_absorb_readout_golden(o):
+    g = _golden()["absorb_readout"]
+    S, z = o.absorb_batch(_as4(g["K_ev"]), _as4(g["V_ev"]))
+    assert np.allclose(S[0, 0], g["S"], atol=1e-14, rtol=0), S[0, 0]
+    assert np.allclose(z[0, 0], g["z"], atol=1e-14, rtol=0), z[0, 0]
+    got = o.linear_readout(_as4(g["Q"]), S, z)[0, 0]
+    assert np.allclose(got, g["O_lin"], atol=1e-13, rtol=0), got
+
+
+def check_absorb_incremental_equals_batch(o):
+    rng = np.random.default_rng(31)
+    B, H, d = 2, 3, 16
+    Ks = [rng.normal(size=(B, H, n, d)) for n in (5, 1, 17, 64)]
+    Vs = [rng.normal(size=(B, H, n, d)) for n in (5, 1, 17, 64)]
+    S = np.zeros((B, H, d, d))
+    z = np.zeros((B, H, d))
+    for k, v in zip(Ks, Vs):
+        S, z = o.absorb(S, z, k, v)
+    Sb, zb = o.absorb_batch(np.concatenate(Ks, axis=2), np.concatenate(Vs, axis=2))
+    assert np.allclose(S, Sb, atol=1e-12, rtol=0) and np.allclose(z, zb, atol=1e-12, rtol=0)
+    assert np.all(z > 0), "z is a sum of positive features"
+    assert S.shape == (B, H, d, d) and z.shape == (B, H, d), "state size independent of tokens"
+
+
+def check_absorb_single_token(o):
+    """One token: S = phi(k) v^T, z = phi(k), phi written out branch by branch."""
+    k = np.array([0.5, -1.25, 0.0, 2.0])
+    v = np.array([1.0, -2.0, 3.0, 0.25])
+    ph = np.array([1.5, math.exp(-1.25), 1.0, 3.0])
+    S, z = o.absorb_batch(_as4([k]), _as4([v]))
+    assert np.allclose(S[0, 0], np.outer(ph, v), atol=1e-15, rtol=0)
+    assert np.allclose(z[0, 0], ph, atol=1e-15, rtol=0)
+
+
+def check_readout_closed_forms(o):
+    """Single-token state: O_lin = v * a / (a + 1e-6) with a = phi(q).phi(k).
+    Empty state: O_lin = 0."""
+    rng = np.random.default_rng(41)
+    d = 8
+    k = rng.normal(size=d)
+    v = rng.normal(size=d)
+    q = rng.normal(size=(5, d))
+    S, z = o.absorb_batch(_as4([k]), _as4([v]))
+    got = o.linear_readout(_as4(q), S, z)[0, 0]
+    pk = np.where(k > 0, k + 1, np.exp(np.minimum(k, 0)))
+    pq = np.where(q > 0, q + 1, np.exp(np.minimum(q, 0)))
+    a = pq @ pk
+    assert np.allclose(got, (a / (a + 1e-6))[:, None] * v[None, :], atol=1e-14, rtol=0)
+    zero = o.linear_readout(_as4(q), np.zeros((1, 1, d, d)), np.zeros((1, 1, d)))
+    assert np.all(zero == 0.0)
+
+
+def check_hybrid_sum(o):
+    """O = O_s + O_lin; with an empty state O = O_s."""
+    rng = np.random.default_rng(51)
+    Q, K, V = (rng.normal(size=(1, 2, n, 8)) for n in (16, 40, 40))
+    idx, _ = o.select_blocks(Q, K, 8, 2)
+    S, z = o.absorb_batch(rng.normal(size=(1, 2, 30, 8)), rng.normal(size=(1, 2, 30, 8)))
+    hyb = o.hybrid_attention(Q, K, V, idx, S, z, 8)
+    assert np.allclose(hyb, o.sparse_attention(Q, K, V, idx, 8) + o.linear_readout(Q, S, z), atol=1e-14)
+    empty = o.hybrid_attention(Q, K, V, idx, np.zeros((1, 2, 8, 8)), np.zeros((1, 2, 8)), 8)
+    assert np.allclose(empty, o.sparse_attention(Q, K, V, idx, 8), atol=0, rtol=0)
+    tile = o.hybrid_attention_tile(Q, K, V, idx, S, z, 8, 0, 1, 1)
+    assert np.allclose(tile, hyb[0, 1, 8:16], atol=1e-14)
+
+
+ALL_CHECKS = [
+    check_phi_library, check_pool_by_hand, check_selection_golden, check_selection_bruteforce,
+    check_selection_ties_constructed, check_selection_output_form, check_attention_golden,
+    check_attention_dense_equivalence, check_attention_subset_library,
+    check_attention_identical_keys, check_absorb_readout_golden,
+    check_absorb_incremental_equals_batch, check_absorb_single_token,
+    check_readout_closed_forms, check_hybrid_sum,
+]

@@ -1,0 +1,148 @@
+"""The fp64 oracle against its pins, and planted mistakes against the pins.
+
+CPU only. A planted mistake lives in a private copy of the oracle module loaded
+for the test; the real oracle is never modified.
+"""
+import importlib.util
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.hf_oracle as real_oracle
+from tests import oracle_pins as pins
+
+ORACLE_PATH = os.path.abspath(real_oracle.__file__)
+
+
+@pytest.mark.parametrize("check", pins.ALL_CHECKS, ids=lambda c: c.__name__)
+def test_oracle_pin(check):
+    check(real_oracle)
+
+
+def _fresh_copy(name):
+    spec = importlib.util.spec_from_file_location(f"_oracle_mutant_{name}", ORACLE_PATH)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def _mut_phi_no_plus_one(m):
+    m.phi = lambda x: np.where(np.asarray(x) > 0, np.asarray(x, float), np.exp(np.minimum(x, 0.0)))
+
+
+def _mut_phi_exp(m):
+    m.phi = lambda x: np.exp(np.asarray(x, float))
+
+
+def _mut_readout_no_eps(m):
+    def f(Q, S, z):
+        ph = m.phi(Q)
+        return (ph @ np.asarray(S, float)) / (ph @ np.asarray(z, float)[..., :, None])
+    m.linear_readout = f
+
+
+def _mut_readout_transposed(m):
+    def f(Q, S, z):
+        ph = m.phi(Q)
+        return (ph @ np.swapaxes(np.asarray(S, float), -1, -2)) / (ph @ np.asarray(z, float)[..., :, None] + 1e-6)
+    m.linear_readout = f
+
+
+def _mut_readout_no_phi_q(m):
+    def f(Q, S, z):
+        q = np.asarray(Q, float)
+        return (q @ np.asarray(S, float)) / (q @ np.asarray(z, float)[..., :, None] + 1e-6)
+    m.linear_readout = f
+
+
+def _mut_select_ties_high(m):
+    orig_lexsort = np.lexsort
+
+    class _NP:
+        def __getattr__(self, k):
+            return getattr(np, k)
+
+        @staticmethod
+        def lexsort(keys):
+            a, b = keys
+            return orig_lexsort((-a, b))
+    m.np = _NP()
+
+
+def _mut_select_bottom(m):
+    orig = m.block_scores
+    m.block_scores = lambda Q, K, block: -orig(Q, K, block)
+
+
+def _mut_pool_sum(m):
+    def f(X, block):
+        X = np.asarray(X, float)
+        B, H, N, d = X.shape
+        out = np.empty((B, H, -(-N // block), d))
+        for t, (lo, hi) in enumerate(m.block_ranges(N, block)):
+            out[:, :, t] = X[:, :, lo:hi].sum(axis=2)
+        return out
+    m.pool_blocks = f
+
+
+def _mut_attention_no_scale(m):
+    m.default_scale = lambda d: 1.0
+
+
+def _mut_attention_sqrt_d(m):
+    m.default_scale = lambda d: float(np.sqrt(d))
+
+
+def _mut_attention_all_keys(m):
+    m._selected_tokens = lambda kept, Nk, block: np.arange(Nk)
+
+
+def _mut_absorb_transposed(m):
+    def f(S, z, K_ev, V_ev):
+        pk = m.phi(K_ev)
+        v = np.asarray(V_ev, float)
+        return np.asarray(S, float) + np.swapaxes(v, -1, -2) @ pk, np.asarray(z, float) + pk.sum(axis=-2)
+    m.absorb = f
+
+
+def _mut_absorb_z_raw(m):
+    def f(S, z, K_ev, V_ev):
+        pk = m.phi(K_ev)
+        v = np.asarray(V_ev, float)
+        return (np.asarray(S, float) + np.swapaxes(pk, -1, -2) @ v,
+                np.asarray(z, float) + np.asarray(K_ev, float).sum(axis=-2))
+    m.absorb = f
+
+
+def _mut_hybrid_difference(m):
+    def f(Q, K, V, idx, S, z, block, scale=None):
+        return m.sparse_attention(Q, K, V, idx, block, scale) - m.linear_readout(Q, S, z)
+    m.hybrid_attention = f
+
+
+MUTANTS = [
+    _mut_phi_no_plus_one, _mut_phi_exp, _mut_readout_no_eps, _mut_readout_transposed,
+    _mut_readout_no_phi_q, _mut_select_ties_high, _mut_select_bottom, _mut_pool_sum,
+    _mut_attention_no_scale, _mut_attention_sqrt_d, _mut_attention_all_keys,
+    _mut_absorb_transposed, _mut_absorb_z_raw, _mut_hybrid_difference,
+]
+
+
+@pytest.mark.parametrize("mutate", MUTANTS, ids=lambda f: f.__name__[5:])
+def test_planted_mistake_is_caught(mutate):
+    m = _fresh_copy(mutate.__name__)
+    mutate(m)
+    failures = []
+    for check in pins.ALL_CHECKS:
+        try:
+            check(m)
+        except (AssertionError, ValueError, IndexError):
+            failures.append(check.__name__)
+    assert failures, f"no pin caught the planted mistake {mutate.__name__}"
+
+
+def test_oracle_package_exports():
+    for name in oracle.__all__:
+        assert hasattr(oracle, name)
