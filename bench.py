@@ -1,0 +1,420 @@
+"""Benchmark of the hybrid attention chunk step on B200.
+
+One step = one pass of the whole hot path over one chunk of the 832x480-shaped
+workload (B=1, H=12, d=128, 4680 queries, 32760-key window, block 128, top-64 of 256
+key blocks, state built from 60 evicted frames):
+    hf_select_blocks      block mean pooling, scores, top-r          (2 kernels)
+    hf_hybrid_attn_fwd    sparse attention + linear readout, summed  (1 kernel)
+    hf_absorb_evicted     the chunk step's 3 evicted frames -> state (2 kernels)
+Metric: query tokens/s per chunk step (whole job, all GPUs), with the roofline fraction
+of the dominant kernel (hf_hybrid_attn_fwd, tensor-bound) against the measured bf16
+peak. Inputs are resident in HBM; L2 is flushed between timed steps (outside the
+timed events). Multi-GPU (torchrun): every rank runs its own chunk stream (weak
+scaling, no collective on the data path); time = max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+``--impl reference`` times the fp64 CPU oracle instead (a bounded sample of heads of
+the same step, scaled to the whole step) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from hybrid_sparse_linear_hf_b200.inputs import WORKLOADS, draw_step_inputs, frame_structured  # noqa: E402
+
+METRIC = "hybrid attn query tokens/s per chunk step; % of bf16 tensor / HBM roofline"
+UNIT = "query tokens/s"
+WORKLOAD = "832x480"
+L2_FLUSH_BYTES = 256 << 20
+LAUNCHES_PER_STEP = 5  # pool, score+select, hybrid attention, absorb partials, state reduce
+
+
+# ----------------------------------------------------------------------------- helpers
+def load_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                "bf16_tflops_sustained": pk.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def attn_flops(idx: np.ndarray, wl) -> float:
+    """Algorithmic FLOPs of one hf_hybrid_attn_fwd launch: 4*d*L_I*L_J per kept (I, J)
+    pair (QK^T and PV), plus 2d^2 + 3d per query for the linear readout."""
+    L_I = np.array([min(wl.block, wl.Nq - I * wl.block) for I in range(wl.nQB)], dtype=np.float64)
+    L_J = np.array([min(wl.block, wl.Nk - J * wl.block) for J in range(wl.nKB)], dtype=np.float64)
+    kept_len = L_J[idx].sum(axis=-1)  # [B,H,nQB]
+    sparse = 4.0 * wl.d * float((kept_len * L_I[None, None, :]).sum())
+    readout = wl.B * wl.H * wl.Nq * (2.0 * wl.d * wl.d + 3.0 * wl.d)
+    return sparse + readout
+
+
+def attn_bytes(wl) -> float:
+    """Algorithmic bytes of one launch: Q and O once, the whole K/V window once, S and z."""
+    return 2.0 * wl.B * wl.H * (2 * wl.Nq * wl.d + 2 * wl.Nk * wl.d) + 4.0 * wl.B * wl.H * (wl.d * wl.d + wl.d)
+
+
+def select_bytes(wl) -> float:
+    return 2.0 * wl.B * wl.H * (wl.Nq + wl.Nk) * wl.d
+
+
+def absorb_bytes(wl, n_tokens) -> float:
+    """K_ev and V_ev read once plus a read and a write of S and z."""
+    return 2.0 * 2 * wl.B * wl.H * n_tokens * wl.d + 2 * 4.0 * wl.B * wl.H * (wl.d * wl.d + wl.d)
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.out = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self) -> dict:
+        if not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm), "sm_mhz_min": min(sm)}
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
+        return int(n)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+# ----------------------------------------------------------------------------- oracle leg
+def oracle_sample(wl, x: dict, S0: torch.Tensor, z0: torch.Tensor, heads, ev_k, ev_v) -> float:
+    """Seconds the fp64 oracle takes for the whole step on the given heads (select,
+    hybrid attention, absorption of the step's evicted tokens)."""
+    import oracle
+
+    f64 = lambda t: t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
+    total = 0.0
+    for h in heads:
+        Q = f64(x["Q"][:, h:h + 1])
+        K = f64(x["K"][:, h:h + 1])
+        V = f64(x["V"][:, h:h + 1])
+        S = f64(S0[:, h:h + 1])
+        z = f64(z0[:, h:h + 1])
+        Ke = f64(ev_k[:, h:h + 1])
+        Ve = f64(ev_v[:, h:h + 1])
+        t0 = time.perf_counter()
+        idx, _ = oracle.select_blocks(Q, K, wl.block, wl.r)
+        oracle.hybrid_attention(Q, K, V, idx, S, z, wl.block)
+        oracle.absorb(S, z, Ke, Ve)
+        total += time.perf_counter() - t0
+    return total
+
+
+def run_reference(args, wl) -> None:
+    """Reference arm: the fp64 CPU oracle, one head per step, scaled to the whole step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    x = draw_step_inputs(wl, n_evicted=wl.Ne_step)
+    g = torch.Generator().manual_seed(wl.seed + 77)
+    S0 = torch.randn(wl.B, wl.H, wl.d, wl.d, generator=g).abs() * 50.0
+    z0 = torch.rand(wl.B, wl.H, wl.d, generator=g) * 1e5
+    for i in range(args.warmup):
+        oracle_sample(wl, x, S0, z0, [i % wl.H], x["K_ev"], x["V_ev"])
+    times = [oracle_sample(wl, x, S0, z0, [i % wl.H], x["K_ev"], x["V_ev"]) for i in range(args.steps)]
+    t_step = statistics.mean(times) * wl.H  # one head per step, scaled to all heads
+    value = wl.B * wl.Nq / t_step
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(wl),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"fp64 numpy oracle, 1 of {wl.H} heads per step (select + hybrid attention + "
+                                   f"absorb of {wl.Ne_step} evicted tokens), scaled x{wl.H}"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(wl) -> dict:
+    return {"workload": f"{wl.name} hybrid attention chunk step", "B": wl.B, "H": wl.H, "d": wl.d,
+            "Nq": wl.Nq, "Nk": wl.Nk, "block": wl.block, "keep": wl.keep, "r": wl.r,
+            "state_frames": wl.state_frames, "evict_frames_per_step": wl.evict_frames,
+            "l2": "flushed between timed steps (256 MiB write)", "parallelism": "independent streams per GPU"}
+
+
+# ----------------------------------------------------------------------------- GPU leg
+def run_gpu(args, wl) -> None:
+    import hybrid_sparse_linear_hf_b200 as hf
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist_mod.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist = dist_mod
+    dev = torch.device("cuda", local_rank if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- inputs, drawn on the device (same recipe, device generator), resident in HBM
+    x = draw_step_inputs(wl, seed=wl.seed + 1000 * rank, n_evicted=wl.Ne_step, device=dev)
+    Q, K, V, K_ev, V_ev = (x[k] for k in ("Q", "K", "V", "K_ev", "V_ev"))
+    S = torch.empty(wl.B, wl.H, wl.d, wl.d, dtype=torch.float32, device=dev)
+    z = torch.empty(wl.B, wl.H, wl.d, dtype=torch.float32, device=dev)
+    st = hf.hf_state_init(S, z)
+    # the state is built from `state_frames` evicted frames (absorbed in slices)
+    gen = torch.Generator(device=dev).manual_seed(wl.seed + 5000 + rank)
+    build_K = frame_structured(gen, wl.B, wl.H, wl.Ne_state, wl.d, wl.tokens_per_frame, wl.w, device=dev)
+    build_V = frame_structured(gen, wl.B, wl.H, wl.Ne_state, wl.d, wl.tokens_per_frame, wl.w, device=dev)
+    ws_abs_build = torch.empty(hf.hf_workspace_size(hf.HF_WS_ABSORB, wl.B, wl.H, 0, wl.Ne_state, wl.d, 0, 0),
+                               dtype=torch.uint8, device=dev)
+    # time the full state build (the absorption's HBM roofline case) on a scratch state
+    Sb = torch.empty_like(S)
+    zb = torch.empty_like(z)
+    stb = hf.hf_state_init(Sb, zb)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    build_times = []
+    for i in range(4):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        hf.hf_absorb_evicted(stb, build_K, build_V, ws=ws_abs_build)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if i > 0:
+            build_times.append(e0.elapsed_time(e1) * 1e-3)
+    hf.hf_absorb_evicted(st, build_K, build_V, ws=ws_abs_build)
+    del build_K, build_V, ws_abs_build
+    ws_sel = torch.empty(hf.hf_workspace_size(hf.HF_WS_SELECT, wl.B, wl.H, wl.Nq, wl.Nk, wl.d, wl.block, wl.r),
+                         dtype=torch.uint8, device=dev)
+    ws_abs = torch.empty(hf.hf_workspace_size(hf.HF_WS_ABSORB, wl.B, wl.H, 0, wl.Ne_step, wl.d, 0, 0),
+                         dtype=torch.uint8, device=dev)
+    idx = torch.empty(wl.B, wl.H, wl.nQB, wl.r, dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        hf.hf_select_blocks(Q, K, wl.block, wl.r, idx_out=idx, ws=ws_sel)
+        if ev:
+            ev[1].record(stream)
+        hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wl.r, idx, st, O=O)
+        if ev:
+            ev[2].record(stream)
+        hf.hf_absorb_evicted(st, K_ev, V_ev, ws=ws_abs)
+        if ev:
+            ev[3].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    rc, word = hf.hf_query_status()
+    if rc != hf.HF_OK:
+        raise RuntimeError(f"device status after warm-up: {hf.hf_status_string(rc)} ({word:#x})")
+    idx_host = idx.cpu().numpy()
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index) as clk:
+        for k in range(args.steps):
+            flush.zero_()
+            step(events[k])
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    rc, word = hf.hf_query_status()
+    if rc != hf.HF_OK:
+        raise RuntimeError(f"device status after timing: {hf.hf_status_string(rc)} ({word:#x})")
+    t_sel = [e[0].elapsed_time(e[1]) * 1e-3 for e in events]
+    t_fwd = [e[1].elapsed_time(e[2]) * 1e-3 for e in events]
+    t_abs = [e[2].elapsed_time(e[3]) * 1e-3 for e in events]
+    t_step_local = sum(e[0].elapsed_time(e[3]) for e in events) * 1e-3 / args.steps
+    t_step = t_step_local
+    if dist:
+        tt = torch.tensor([t_step_local], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_step = float(tt.item())
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    host = {k: v.cpu().pin_memory() for k, v in x.items()}
+    O_host = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = O_host.numel() * O_host.element_size()
+    n_e2e = max(3, min(args.steps, 20))
+    dQ, dK, dV, dKe, dVe = (torch.empty_like(x[k]) for k in ("Q", "K", "V", "K_ev", "V_ev"))
+
+    def e2e_step():
+        dQ.copy_(host["Q"], non_blocking=True)
+        dK.copy_(host["K"], non_blocking=True)
+        dV.copy_(host["V"], non_blocking=True)
+        dKe.copy_(host["K_ev"], non_blocking=True)
+        dVe.copy_(host["V_ev"], non_blocking=True)
+        hf.hf_select_blocks(dQ, dK, wl.block, wl.r, idx_out=idx, ws=ws_sel)
+        hf.hf_hybrid_attn_fwd(dQ, dK, dV, wl.block, wl.r, idx, st, O=O)
+        hf.hf_absorb_evicted(st, dKe, dVe, ws=ws_abs)
+        O_host.copy_(O, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_e2e = e0.elapsed_time(e1) * 1e-3 / n_e2e
+    if dist:
+        tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_e2e = float(tt.item())
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks = load_peaks()
+    F = attn_flops(idx_host, wl)
+    fwd_mean = statistics.mean(t_fwd)
+    achieved_tf = F / fwd_mean / 1e12
+    sel_mean, abs_mean = statistics.mean(t_sel), statistics.mean(t_abs)
+    build_mean = statistics.mean(build_times)
+    value = world * wl.B * wl.Nq / t_step
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_dict(wl),
+        "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved_tf / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "hybrid_attn_kernel<128,128>", "flops_per_launch": F,
+                     "peak_source": f"{peaks['source']} dense bf16 (burst)"},
+        "kernels": {
+            "hf_hybrid_attn_fwd": {"us": fwd_mean * 1e6, "tflops": achieved_tf,
+                                   "bytes": attn_bytes(wl), "gbs": attn_bytes(wl) / fwd_mean / 1e9},
+            "hf_select_blocks": {"us": sel_mean * 1e6, "bytes": select_bytes(wl),
+                                 "gbs": select_bytes(wl) / sel_mean / 1e9,
+                                 "hbm_frac": select_bytes(wl) / sel_mean / 1e9 / peaks["hbm_gbs"]},
+            "hf_absorb_evicted_step": {"us": abs_mean * 1e6, "tokens": wl.Ne_step,
+                                       "bytes": absorb_bytes(wl, wl.Ne_step),
+                                       "gbs": absorb_bytes(wl, wl.Ne_step) / abs_mean / 1e9},
+            "hf_absorb_evicted_state_build": {"us": build_mean * 1e6, "tokens": wl.Ne_state,
+                                              "bytes": absorb_bytes(wl, wl.Ne_state),
+                                              "gbs": absorb_bytes(wl, wl.Ne_state) / build_mean / 1e9,
+                                              "hbm_frac": absorb_bytes(wl, wl.Ne_state) / build_mean / 1e9
+                                              / peaks["hbm_gbs"]},
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+        },
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+        "e2e": {"value": world * wl.B * wl.Nq / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": n_e2e,
+                "note": "pinned host Q, K/V window, evicted K/V copied in and O copied out every step"},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        # bounded sample of the fp64 oracle on the host cores: whole heads until ~10 s
+        ev_k, ev_v = K_ev.cpu(), V_ev.cpu()
+        xs = {k: x[k].cpu() for k in ("Q", "K", "V")}
+        heads, spent = [], 0.0
+        for h in range(wl.H):
+            spent += oracle_sample(wl, xs, S.cpu(), z.cpu(), [h], ev_k, ev_v)
+            heads.append(h)
+            if spent >= 10.0:
+                break
+        t_cpu_step = spent / len(heads) * wl.H
+        line["cpu_baseline"] = {
+            "value": wl.B * wl.Nq / t_cpu_step, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle on {len(heads)} of {wl.H} heads (select + hybrid attention + absorb "
+                      f"of the step's {wl.Ne_step} evicted tokens), {spent:.1f} s, scaled to all heads"}
+    print(json.dumps(line), flush=True)
+
+
+def main() -> None:
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["hf", "reference"], default="hf")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle CPU-baseline leg")
+    args = ap.parse_args()
+    wl = WORKLOADS[WORKLOAD]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,213 @@
+"""ctypes binding of ``libhf.so`` (C ABI in ``include/hf.h``), same names as the C calls.
+
+Argument marshalling only: every step of the hybrid attention step runs in the CUDA
+kernels of the library. PyTorch supplies device memory (tensors) and streams. There is
+no CPU fallback: if the library is missing, the first call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libhf.so")
+
+HF_OK = 0
+HF_ERR_INVALID_ARG = 1
+HF_ERR_UNSUPPORTED = 2
+HF_ERR_ALIGNMENT = 3
+HF_ERR_WORKSPACE = 4
+HF_ERR_CUDA = 5
+HF_ERR_DEVICE_TIMEOUT = 6
+HF_ERR_DEVICE_BAD_INDEX = 7
+
+HF_WS_SELECT = 1
+HF_WS_ATTN = 2
+HF_WS_ABSORB = 3
+
+_SIZE_T_MAX = (1 << (8 * ctypes.sizeof(ctypes.c_size_t))) - 1
+
+
+class HfStateC(ctypes.Structure):
+    """Mirror of ``struct hf_state``."""
+
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
+                ("S", ctypes.c_void_p), ("z", ctypes.c_void_p), ("n_absorbed", ctypes.c_longlong)]
+
+
+class HfError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {hf_status_string(status)} (status {status})")
+
+
+_lib = None
+
+_SIGNATURES = {
+    "hf_workspace_size": (ctypes.c_size_t, [ctypes.c_int] * 8),
+    "hf_state_init": (ctypes.c_int, [ctypes.POINTER(HfStateC), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "hf_absorb_evicted": (ctypes.c_int, [ctypes.POINTER(HfStateC), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                         ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_select_blocks": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 +
+                         [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_hybrid_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
+                           [ctypes.c_void_p, ctypes.POINTER(HfStateC), ctypes.c_float, ctypes.c_void_p,
+                            ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_query_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "hf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "hf_version": (ctypes.c_char_p, []),
+    "hf_debug_inject_timeout": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_ulonglong]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if ``libhf.so`` has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m hybrid_sparse_linear_hf_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def hf_status_string(status: int) -> str:
+    return lib().hf_status_string(int(status)).decode()
+
+
+def hf_version() -> str:
+    return lib().hf_version().decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != HF_OK:
+        raise HfError(rc, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+class HfState:
+    """Python handle of ``hf_state``: keeps S [B,H,d,d] and z [B,H,d] (fp32, device) alive."""
+
+    def __init__(self, S: torch.Tensor, z: torch.Tensor):
+        self.S = S
+        self.z = z
+        self.c = HfStateC()
+
+    @property
+    def n_absorbed(self) -> int:
+        return int(self.c.n_absorbed)
+
+    @property
+    def shape(self):
+        return (self.c.B, self.c.H, self.c.d)
+
+
+def hf_workspace_size(which: int, B: int, H: int, Nq: int, Nk: int, d: int, block: int, r: int) -> int:
+    n = lib().hf_workspace_size(which, B, H, Nq, Nk, d, block, r)
+    if n == _SIZE_T_MAX:
+        raise HfError(HF_ERR_INVALID_ARG, "hf_workspace_size")
+    return int(n)
+
+
+def _workspace(nbytes: int, device, ws):
+    if nbytes == 0:
+        return None, 0
+    if ws is None:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws, ws.numel() * ws.element_size()
+
+
+def hf_state_init(S: torch.Tensor, z: torch.Tensor, stream=None) -> HfState:
+    """Bind S [B,H,d,d] and z [B,H,d] (fp32) as a state and zero them."""
+    if S.dim() != 4 or z.dim() != 3:
+        raise ValueError("S must be [B,H,d,d] and z [B,H,d]")
+    B, H, d, _ = S.shape
+    st = HfState(S, z)
+    _check(lib().hf_state_init(ctypes.byref(st.c), B, H, d, _dev(S, torch.float32, "S"),
+                               _dev(z, torch.float32, "z"), _stream(stream)), "hf_state_init")
+    return st
+
+
+def hf_absorb_evicted(state: HfState, K_ev: torch.Tensor, V_ev: torch.Tensor, ws=None, stream=None) -> None:
+    """S += phi(K_ev)^T V_ev, z += sum phi(K_ev) for K_ev, V_ev [B,H,n,d] bf16."""
+    B, H, d = state.shape
+    if K_ev.shape != V_ev.shape or K_ev.dim() != 4 or tuple(K_ev.shape[:2]) != (B, H) or K_ev.shape[3] != d:
+        raise ValueError("K_ev and V_ev must both be [B,H,n,d] matching the state")
+    n = K_ev.shape[2]
+    nbytes = hf_workspace_size(HF_WS_ABSORB, B, H, 0, n, d, 0, 0)
+    ws, ws_bytes = _workspace(nbytes, K_ev.device, ws)
+    _check(lib().hf_absorb_evicted(ctypes.byref(state.c), _dev(K_ev, torch.bfloat16, "K_ev"),
+                                   _dev(V_ev, torch.bfloat16, "V_ev"), n,
+                                   ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
+           "hf_absorb_evicted")
+
+
+def hf_select_blocks(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, idx_out=None, scores_out=None,
+                     ws=None, stream=None) -> torch.Tensor:
+    """Top-r key blocks per query block: int32 [B,H,nQB,r] (ascending)."""
+    B, H, Nq, d = Q.shape
+    Nk = K.shape[2]
+    nQB = -(-Nq // block)
+    if idx_out is None:
+        idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
+    nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, Nk, d, block, r)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    _check(lib().hf_select_blocks(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), B, H, Nq, Nk, d,
+                                  block, r, _dev(idx_out, torch.int32, "idx_out"),
+                                  _dev(scores_out, torch.float32, "scores_out") if scores_out is not None else None,
+                                  ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
+           "hf_select_blocks")
+    return idx_out
+
+
+def hf_hybrid_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block: int, r: int,
+                       idx: torch.Tensor, state: HfState, scale: float = 0.0, O=None, stream=None) -> torch.Tensor:
+    """Hybrid attention output O [B,H,Nq,d] bf16 = sparse term + linear term."""
+    B, H, Nq, d = Q.shape
+    Nk = K.shape[2]
+    if O is None:
+        O = torch.empty_like(Q)
+    _check(lib().hf_hybrid_attn_fwd(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"),
+                                    _dev(V, torch.bfloat16, "V"), B, H, Nq, Nk, d, block, r,
+                                    _dev(idx, torch.int32, "idx"), ctypes.byref(state.c), float(scale),
+                                    _dev(O, torch.bfloat16, "O"), None, 0, _stream(stream)),
+           "hf_hybrid_attn_fwd")
+    return O
+
+
+def hf_query_status(stream=None) -> tuple[int, int]:
+    """(status, raw device error word) after synchronising the stream; clears the word."""
+    detail = ctypes.c_uint32(0)
+    rc = lib().hf_query_status(_stream(stream), ctypes.byref(detail))
+    return int(rc), int(detail.value)
+
+
+def hf_debug_inject_timeout(kernel_id: int, count: int, timeout_ns: int) -> None:
+    """Test only: see ``hf_debug_inject_timeout`` in include/hf.h."""
+    _check(lib().hf_debug_inject_timeout(kernel_id, count, timeout_ns), "hf_debug_inject_timeout")

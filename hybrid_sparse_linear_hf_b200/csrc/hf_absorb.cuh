@@ -1,0 +1,330 @@
+// State absorption (hf_absorb_evicted): S += phi(K)^T V, z += sum_t phi(k_t).
+//
+// Source: "Long-Horizon Streaming Video Generation via Hybrid Attention with
+// Decoupled Distillation", German technical summary, section 2 A (frames evicted
+// from the sliding window are aggregated into a compact KV state through a linear
+// attention function, constant memory in the video length); English abstract
+// (a compact key-value state incrementally absorbs evicted tokens).
+//
+// Work split: the tokens of every (b,h) are cut into `nsplit` slices of whole
+// 64-token tiles; one CTA per (b,h,slice) accumulates its slice's phi(K)^T V in TMEM
+// and writes an fp32 partial; reduce_state_kernel adds the partials of a head to S
+// and z in slice order (deterministic).
+//
+// absorb_partial_kernel (192 threads, one CTA per SM):
+//   warp 0      TMA producer: K and V tiles [64 tokens][d] into a 4-stage ring.
+//   warp 1      TMEM owner + MMA issuer: for each tile, D += A_hi x V and D += A_lo x V
+//               with M = 128 (d-index of S, zero-padded for d = 64), N = d, K = 64
+//               tokens; both operands MN-major (d contiguous).
+//   warps 2..5  converters: phi(k) in fp32, split hi = bf16(phi), lo = bf16(phi - hi)
+//               written at the same swizzled offsets as the K tile (the A operand has
+//               the K tile's layout), z accumulated in fp32 registers. They also drain
+//               the accumulator: the tensor core's fp32 accumulation truncates, so a
+//               long chain of MMAs into one TMEM accumulator drifts (relative error
+//               grows with the chain length, ~2e-5 after 500 MMAs). The MMAs of every
+//               group of kAbsGroup tiles (16 MMAs) therefore go to one of two TMEM
+//               buffers, which the converters add into fp32 registers with
+//               round-to-nearest while the other buffer fills. Epilogue: registers ->
+//               fp32 partial in the workspace.
+// Rows past the end of the token range are zero-filled by TMA; their phi is forced
+// to 0 (phi(0) = 1 would otherwise leak into z).
+#pragma once
+
+#include "hf_ptx.cuh"
+
+namespace hf {
+
+constexpr uint32_t kKernAbsorb = 2;
+constexpr int kAbsTok = 64;        // tokens per tile
+constexpr int kAbsStages = 4;      // K/V ring depth
+constexpr int kAbsThreads = 192;
+constexpr int kAbsGroup = 2;       // tiles per TMEM accumulation chain
+
+template <int D>
+struct AbsorbCfg {
+  static constexpr int kChunks = D / 64;                  // 64-element column chunks of K/V
+  static constexpr int kChunkBytes = kAbsTok * 128;       // one chunk of a tile: 64 rows x 128 B
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes;      // K tile + V tile
+  static constexpr int kAOpBytes = 2 * kChunkBytes;       // A operand, M = 128 (2 chunks)
+  static constexpr int kABufBytes = 2 * kAOpBytes;        // hi + lo
+  static constexpr int kRingBytes = kAbsStages * kStageBytes;
+  static constexpr int kDynSmem = 1024 + kRingBytes + 2 * kABufBytes;
+};
+
+struct AbsorbParams {
+  float* part_S;  // [BH][nsplit][D][D]
+  float* part_z;  // [BH][nsplit][D]
+  int n_tokens;   // tokens per (b,h)
+  int tiles_per_split;
+  int nsplit;
+  unsigned long long timeout_ns;
+  int inject;     // test only: skip the first tile's load so a wait runs out
+};
+
+template <int D>
+__global__ void __launch_bounds__(kAbsThreads, 1)
+    absorb_partial_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                          AbsorbParams p) {
+  using C = AbsorbCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  uint8_t* abuf = smem + C::kRingBytes;  // [2][hi | lo]
+
+  __shared__ uint64_t full_bar[kAbsStages], empty_bar[kAbsStages];
+  __shared__ uint64_t afull_bar[2], aempty_bar[2];
+  __shared__ uint64_t dfull_bar[2], dempty_bar[2], drain_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ int abort_sh;
+  __shared__ float zred[128][8];
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int bh = blockIdx.x / p.nsplit;
+  const int split = blockIdx.x % p.nsplit;
+  const int tile0 = split * p.tiles_per_split;
+  const int tiles_total = (p.n_tokens + kAbsTok - 1) / kAbsTok;
+  const int ntiles = min(p.tiles_per_split, tiles_total - tile0);
+  volatile int* abort_flag = &abort_sh;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAbsStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&afull_bar[a], 128);
+      mbar_init(&aempty_bar[a], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&dfull_bar[b], 1);
+      mbar_init(&dempty_bar[b], 128);
+    }
+    mbar_init(&drain_bar, 1);
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, 256);
+    tmem_relinquish();
+  }
+  if (D < 128 && warp >= 2) {
+    // the upper 64 rows of the M = 128 A operand are zero padding for d = 64
+    for (int i = threadIdx.x - 64; i < 2 * 2 * C::kChunkBytes / 16; i += 128) {
+      const int a = i / (2 * C::kChunkBytes / 16), rem = i % (2 * C::kChunkBytes / 16);
+      const int op = rem / (C::kChunkBytes / 16), u = rem % (C::kChunkBytes / 16);
+      reinterpret_cast<uint4*>(abuf + a * C::kABufBytes + op * C::kAOpBytes + C::kChunkBytes)[u] =
+          make_uint4(0, 0, 0, 0);
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = tmem_base_sh;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kAbsStages, u = i / kAbsStages;
+        if (u >= 1 && !mbar_wait(&empty_bar[s], (u - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 1))
+          break;
+        if (*abort_flag) break;
+        if (p.inject && i == 0) continue;  // test only: tile 0 never arrives
+        uint8_t* st = ring + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
+        const int row = (tile0 + i) * kAbsTok;
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_3d(st + c * C::kChunkBytes, &mapK, &full_bar[s], c * 64, row, bh);
+          tma_load_3d(st + C::kTileBytes + c * C::kChunkBytes, &mapV, &full_bar[s], c * 64, row, bh);
+        }
+        issued = i + 1;
+      }
+      // drain: every issued copy must have landed before the CTA may exit
+      for (int i = max(0, issued - kAbsStages); i < issued; ++i) {
+        if (p.inject && i == 0) continue;
+        mbar_wait_drain(&full_bar[i % kAbsStages], (i / kAbsStages) & 1, p.timeout_ns, (kKernAbsorb << 8) | 2);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+      bool ok = true;
+      for (int i = 0; i < ntiles && ok; ++i) {
+        const int s = i % kAbsStages, a = i & 1;
+        const int g = i / kAbsGroup, b = g & 1;
+        const bool first = (i % kAbsGroup) == 0;
+        const bool last = (i % kAbsGroup) == kAbsGroup - 1 || i == ntiles - 1;
+        ok = mbar_wait(&full_bar[s], (i / kAbsStages) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 3) &&
+             mbar_wait(&afull_bar[a], (i >> 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 4);
+        if (ok && first && g >= 2)
+          ok = mbar_wait(&dempty_bar[b], ((g >> 1) - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 9);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(ring + s * C::kStageBytes + C::kTileBytes);
+        const uint32_t a_addr = smem_u32(abuf + a * C::kABufBytes);
+        const uint32_t d_tmem = tmem_d + b * 128;
+#pragma unroll
+        for (int op = 0; op < 2; ++op) {
+#pragma unroll
+          for (int ks = 0; ks < kAbsTok / 16; ++ks) {
+            const uint64_t adesc = sdesc_sw128(a_addr + op * C::kAOpBytes + ks * 2048, C::kChunkBytes, 1024);
+            const uint64_t bdesc = sdesc_sw128(v_addr + ks * 2048, C::kChunkBytes, 1024);
+            umma_ss(d_tmem, adesc, bdesc, idesc, (!first || op > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        umma_commit(&empty_bar[s]);
+        umma_commit(&aempty_bar[a]);
+        if (last) umma_commit(&dfull_bar[b]);
+      }
+      umma_commit(&drain_bar);
+      mbar_wait_drain(&drain_bar, 0, p.timeout_ns, (kKernAbsorb << 8) | 5);
+    }
+  } else {
+    // ---------------- converters + epilogue (128 threads) ----------------
+    const int t = threadIdx.x - 64;  // 0..127
+    constexpr int kUnits = D / 8;    // 16-byte units per row
+    constexpr int kPhases = 128 / kUnits;
+    const int ucol = t % kUnits;     // logical unit column: elements [8*ucol, 8*ucol + 8)
+    const int phase = t / kUnits;    // rows phase, phase + kPhases, ...
+    const int chunk = ucol / 8;
+    const uint32_t swz = static_cast<uint32_t>(((ucol % 8) ^ (phase & 7)) * 16);
+    float zacc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    // register accumulator of this thread's row m of phi(K)^T V (TMEM lane m)
+    const int quarter = warp & 3;
+    const int m = quarter * 32 + lane;
+    const uint32_t lane_base = tmem_d + (static_cast<uint32_t>(quarter * 32) << 16);
+    float acc[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) acc[c] = 0.f;
+    const int ngroups = (ntiles + kAbsGroup - 1) / kAbsGroup;
+    int flushed = 0;
+    bool ok = true;
+    auto flush_group = [&](int g) {
+      const int b = g & 1;
+      if (!mbar_wait(&dfull_bar[b], (g >> 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 8)) return false;
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + b * 128 + c0, r);
+        tmem_wait_ld();
+        reg_fence<32>(r);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[c0 + j] += __uint_as_float(r[j]);
+      }
+      tc_fence_before();
+      mbar_arrive(&dempty_bar[b]);
+      return true;
+    };
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int s = i % kAbsStages, a = i & 1;
+      ok = mbar_wait(&full_bar[s], (i / kAbsStages) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 6);
+      if (ok && i >= 2) ok = mbar_wait(&aempty_bar[a], ((i >> 1) - 1) & 1, abort_flag, p.timeout_ns,
+                                       (kKernAbsorb << 8) | 7);
+      if (!ok) break;
+      const uint8_t* ktile = ring + s * C::kStageBytes;
+      uint8_t* ahi = abuf + a * C::kABufBytes;
+      uint8_t* alo = ahi + C::kAOpBytes;
+      const int valid = min(kAbsTok, p.n_tokens - (tile0 + i) * kAbsTok);
+#pragma unroll 2
+      for (int row = phase; row < kAbsTok; row += kPhases) {
+        const uint32_t off = chunk * C::kChunkBytes + row * 128 + swz;
+        const uint4 kv = *reinterpret_cast<const uint4*>(ktile + off);
+        const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
+        uint32_t hi[4], lo[4];
+        const bool live = row < valid;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x0 = bf16_lo_to_f32(w[e]), x1 = bf16_hi_to_f32(w[e]);
+          float p0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
+          float p1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
+          if (!live) p0 = p1 = 0.f;
+          zacc[2 * e] += p0;
+          zacc[2 * e + 1] += p1;
+          const uint32_t h = pack_bf16x2(p0, p1);
+          hi[e] = h;
+          lo[e] = pack_bf16x2(p0 - bf16_lo_to_f32(h), p1 - bf16_hi_to_f32(h));
+        }
+        *reinterpret_cast<uint4*>(ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&afull_bar[a]);
+      // once group g is fully converted, drain group g - 1 (one group of lag keeps the
+      // tensor core busy on the other buffer)
+      const int g = i / kAbsGroup;
+      const bool group_done = (i % kAbsGroup) == kAbsGroup - 1 || i == ntiles - 1;
+      if (group_done && g >= 1) {
+        ok = flush_group(g - 1);
+        flushed = g;
+      }
+    }
+    if (ok) {
+      for (int g = flushed; g < ngroups && ok; ++g) ok = flush_group(g);
+    }
+    // z partial: reduce the kPhases row phases of each unit column
+#pragma unroll
+    for (int k = 0; k < 8; ++k) zred[t][k] = zacc[k];
+    named_bar_sync(1, 128);
+    if (t < D) {
+      const int uc = t / 8, e = t % 8;
+      float zs = 0.f;
+      for (int ph = 0; ph < kPhases; ++ph) zs += zred[ph * kUnits + uc][e];
+      p.part_z[(static_cast<size_t>(bh) * p.nsplit + split) * D + t] = zs;
+    }
+    // S partial: row m of this slice's phi(K)^T V
+    if (ok && m < D) {
+      float* dst = p.part_S + ((static_cast<size_t>(bh) * p.nsplit + split) * D + m) * D;
+#pragma unroll
+      for (int j = 0; j < D; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_d, 256);
+  }
+}
+
+// S[bh] += sum_s part_S[bh][s], z[bh] += sum_s part_z[bh][s], slices in order.
+template <int D>
+__global__ void __launch_bounds__(256) reduce_state_kernel(float* __restrict__ S, float* __restrict__ z,
+                                                           const float* __restrict__ part_S,
+                                                           const float* __restrict__ part_z, int nsplit) {
+  constexpr int kVec4PerHead = D * D / 4;
+  constexpr int kCtasPerHead = (kVec4PerHead + 255) / 256;
+  const int bh = blockIdx.x / kCtasPerHead;
+  const int e4 = (blockIdx.x % kCtasPerHead) * 256 + threadIdx.x;
+  if (e4 < kVec4PerHead) {
+    float4* s4 = reinterpret_cast<float4*>(S + static_cast<size_t>(bh) * D * D) + e4;
+    float4 acc = *s4;
+    const float4* p4 = reinterpret_cast<const float4*>(part_S + static_cast<size_t>(bh) * nsplit * D * D) + e4;
+    for (int s = 0; s < nsplit; ++s) {
+      const float4 v = p4[static_cast<size_t>(s) * kVec4PerHead];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    *s4 = acc;
+  }
+  if (blockIdx.x % kCtasPerHead == 0 && threadIdx.x < D) {
+    float acc = z[static_cast<size_t>(bh) * D + threadIdx.x];
+    for (int s = 0; s < nsplit; ++s) acc += part_z[(static_cast<size_t>(bh) * nsplit + s) * D + threadIdx.x];
+    z[static_cast<size_t>(bh) * D + threadIdx.x] = acc;
+  }
+}
+
+}  // namespace hf

@@ -1,0 +1,346 @@
+// C ABI of the hybrid attention chunk step (declared in include/hf.h).
+//
+// Host side: argument validation (before any launch), TMA tensor-map encoding, grid
+// sizing and kernel dispatch on (d, block). The whole library is this one translation
+// unit; the kernels live in the included headers.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "hf.h"
+#include "hf_absorb.cuh"
+#include "hf_attn.cuh"
+#include "hf_ptx.cuh"
+#include "hf_select.cuh"
+
+namespace {
+
+using hf::AttnCfg;
+
+constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;  // 1 s per wait
+// CTAs the absorption spreads a call over (one per SM of a B200). A constant, so the
+// workspace size is a pure function of the shapes.
+constexpr int kAbsorbTargetCtas = 148;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+
+struct Injection {
+  int kernel_id = 0;
+  int count = 0;
+  unsigned long long timeout_ns = kDefaultTimeoutNs;
+};
+Injection g_inject;
+
+// Returns (inject flag, timeout) for one launch of `kernel_id`.
+void take_injection(int kernel_id, int* inject, unsigned long long* timeout_ns) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  *inject = 0;
+  *timeout_ns = kDefaultTimeoutNs;
+  if (g_inject.kernel_id == kernel_id && g_inject.count > 0) {
+    *inject = 1;
+    *timeout_ns = g_inject.timeout_ns;
+    if (--g_inject.count == 0) g_inject.kernel_id = 0;
+  }
+}
+
+EncodeTiledFn encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  return g_encode;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool supported_d(int d) { return d == 64 || d == 128; }
+bool supported_block(int b) { return b == 32 || b == 64 || b == 128; }
+int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// 3-D bf16 tensor map over [BH][rows][d] with a (64 x box_rows x 1) box, 128-byte swizzle.
+hf_status make_map(CUtensorMap* m, const void* base, int d, long long rows, long long bh, int box_rows) {
+  EncodeTiledFn enc = encoder();
+  if (!enc) return HF_ERR_CUDA;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(rows) * d * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? HF_OK : HF_ERR_CUDA;
+}
+
+hf_status launch_status() { return cudaGetLastError() == cudaSuccess ? HF_OK : HF_ERR_CUDA; }
+
+// ---------------------------------------------------------------- select
+size_t select_ws_bytes(int B, int H, int Nq, int Nk, int d, int block) {
+  const long long bh = static_cast<long long>(B) * H;
+  return align256(static_cast<size_t>(bh) * ceil_div(Nq, block) * d * 4) +
+         align256(static_cast<size_t>(bh) * ceil_div(Nk, block) * d * 4);
+}
+
+template <int D>
+hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk, int block, int r,
+                        int32_t* idx, float* scores, void* ws, cudaStream_t st) {
+  const int nQB = ceil_div(Nq, block), nKB = ceil_div(Nk, block);
+  float* Qp = static_cast<float*>(ws);
+  float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(BH) * nQB * D * 4));
+  const long long grid1 = static_cast<long long>(BH) * (nQB + nKB);
+  hf::pool_blocks_kernel<D><<<static_cast<unsigned>(grid1), hf::kPoolThreads, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block, nQB,
+      nKB, Qp, Kp);
+  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  const size_t smem = static_cast<size_t>(nKB) * 8;
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(hf::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return HF_ERR_CUDA;
+  }
+  hf::score_select_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * nQB), hf::kSelectThreads, smem,
+                               st>>>(Qp, Kp, nQB, nKB, r, idx, scores);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- absorb
+struct AbsorbPlan {
+  int tiles_per_split, nsplit;
+};
+
+AbsorbPlan absorb_plan(long long BH, int n_tokens, int sms) {
+  const int tiles = ceil_div(n_tokens, hf::kAbsTok);
+  int nsplit = BH >= sms ? 1 : static_cast<int>(sms / BH);
+  if (nsplit > tiles) nsplit = tiles;
+  if (nsplit < 1) nsplit = 1;
+  const int per = ceil_div(tiles, nsplit);
+  return AbsorbPlan{per, ceil_div(tiles, per)};
+}
+
+size_t absorb_ws_bytes(int B, int H, int n_tokens, int d) {
+  const long long bh = static_cast<long long>(B) * H;
+  const AbsorbPlan pl = absorb_plan(bh, n_tokens, kAbsorbTargetCtas);
+  return align256(static_cast<size_t>(bh) * pl.nsplit * d * d * 4) +
+         align256(static_cast<size_t>(bh) * pl.nsplit * d * 4);
+}
+
+template <int D>
+hf_status launch_absorb(hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, int n_tokens, void* ws,
+                        cudaStream_t stream) {
+  using C = hf::AbsorbCfg<D>;
+  const long long BH = static_cast<long long>(st->B) * st->H;
+  const AbsorbPlan pl = absorb_plan(BH, n_tokens, kAbsorbTargetCtas);
+  CUtensorMap mk, mv;
+  if (make_map(&mk, K_ev, D, n_tokens, BH, hf::kAbsTok) != HF_OK) return HF_ERR_CUDA;
+  if (make_map(&mv, V_ev, D, n_tokens, BH, hf::kAbsTok) != HF_OK) return HF_ERR_CUDA;
+  hf::AbsorbParams p;
+  p.part_S = static_cast<float*>(ws);
+  p.part_z = reinterpret_cast<float*>(static_cast<char*>(ws) +
+                                      align256(static_cast<size_t>(BH) * pl.nsplit * D * D * 4));
+  p.n_tokens = n_tokens;
+  p.tiles_per_split = pl.tiles_per_split;
+  p.nsplit = pl.nsplit;
+  take_injection(2, &p.inject, &p.timeout_ns);
+  if (cudaFuncSetAttribute(hf::absorb_partial_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kDynSmem) != cudaSuccess)
+    return HF_ERR_CUDA;
+  hf::absorb_partial_kernel<D>
+      <<<static_cast<unsigned>(BH * pl.nsplit), hf::kAbsThreads, C::kDynSmem, stream>>>(mk, mv, p);
+  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  constexpr int kCtasPerHead = (D * D / 4 + 255) / 256;
+  hf::reduce_state_kernel<D><<<static_cast<unsigned>(BH * kCtasPerHead), 256, 0, stream>>>(st->S, st->z, p.part_S,
+                                                                                         p.part_z, pl.nsplit);
+  return launch_status();
+}
+
+// ---------------------------------------------------------------- attention
+template <int D, int BLK>
+hf_status launch_attn(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int BH, int Nq, int Nk, int r,
+                      const int32_t* idx, const hf_state* st, float scale, hf_bf16* O, cudaStream_t stream) {
+  using C = AttnCfg<D, BLK>;
+  const int nQB = ceil_div(Nq, BLK), nKB = ceil_div(Nk, BLK);
+  CUtensorMap mq, mk, mv, mo;
+  if (make_map(&mq, Q, D, Nq, BH, 128) != HF_OK || make_map(&mk, K, D, Nk, BH, BLK) != HF_OK ||
+      make_map(&mv, V, D, Nk, BH, BLK) != HF_OK || make_map(&mo, O, D, Nq, BH, BLK) != HF_OK)
+    return HF_ERR_CUDA;
+  hf::AttnParams p;
+  p.idx = idx;
+  p.S = st->S;
+  p.z = st->z;
+  p.nQB = nQB;
+  p.nKB = nKB;
+  p.r = r;
+  p.last_len = Nk - (nKB - 1) * BLK;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  take_injection(3, &p.inject, &p.timeout_ns);
+  if (cudaFuncSetAttribute(hf::hybrid_attn_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kDynSmem) != cudaSuccess)
+    return HF_ERR_CUDA;
+  hf::hybrid_attn_kernel<D, BLK>
+      <<<static_cast<unsigned>(static_cast<long long>(BH) * nQB), hf::kAttnThreads, C::kDynSmem, stream>>>(
+          mq, mk, mv, mo, p);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+HF_API const char* hf_version(void) { return "hf-b200 0.1.0 (sm_100a)"; }
+
+HF_API const char* hf_status_string(hf_status s) {
+  switch (s) {
+    case HF_OK: return "HF_OK";
+    case HF_ERR_INVALID_ARG: return "HF_ERR_INVALID_ARG: invalid argument";
+    case HF_ERR_UNSUPPORTED: return "HF_ERR_UNSUPPORTED: d must be 64 or 128, block 32, 64 or 128";
+    case HF_ERR_ALIGNMENT: return "HF_ERR_ALIGNMENT: pointers must be 16-byte aligned";
+    case HF_ERR_WORKSPACE: return "HF_ERR_WORKSPACE: workspace missing or too small";
+    case HF_ERR_CUDA: return "HF_ERR_CUDA: a CUDA call or kernel launch failed";
+    case HF_ERR_DEVICE_TIMEOUT: return "HF_ERR_DEVICE_TIMEOUT: a kernel gave up on an internal wait";
+    case HF_ERR_DEVICE_BAD_INDEX: return "HF_ERR_DEVICE_BAD_INDEX: a block index outside [0, nKB) was skipped";
+  }
+  return "unknown hf_status";
+}
+
+HF_API size_t hf_workspace_size(int which, int B, int H, int Nq, int Nk, int d, int block, int r) {
+  if (B < 1 || H < 1 || !supported_d(d)) return static_cast<size_t>(-1);
+  switch (which) {
+    case HF_WS_SELECT:
+      if (!supported_block(block) || Nq < 0 || Nk < 1 || r < 1 || r > ceil_div(Nk, block))
+        return static_cast<size_t>(-1);
+      return select_ws_bytes(B, H, Nq, Nk, d, block);
+    case HF_WS_ATTN:
+      if (!supported_block(block) || Nq < 0 || Nk < 1 || r < 1 || r > ceil_div(Nk, block))
+        return static_cast<size_t>(-1);
+      return 0;
+    case HF_WS_ABSORB:
+      if (Nk < 0) return static_cast<size_t>(-1);
+      if (Nk == 0) return 0;
+      return absorb_ws_bytes(B, H, Nk, d);
+  }
+  return static_cast<size_t>(-1);
+}
+
+HF_API hf_status hf_state_init(hf_state* st, int B, int H, int d, float* S_dev, float* z_dev, void* stream) {
+  if (!st || !S_dev || !z_dev || B < 1 || H < 1) return HF_ERR_INVALID_ARG;
+  if (!supported_d(d)) return HF_ERR_UNSUPPORTED;
+  if (!aligned16(S_dev) || !aligned16(z_dev)) return HF_ERR_ALIGNMENT;
+  const size_t bh = static_cast<size_t>(B) * H;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(S_dev, 0, bh * d * d * sizeof(float), s) != cudaSuccess) return HF_ERR_CUDA;
+  if (cudaMemsetAsync(z_dev, 0, bh * d * sizeof(float), s) != cudaSuccess) return HF_ERR_CUDA;
+  st->B = B;
+  st->H = H;
+  st->d = d;
+  st->S = S_dev;
+  st->z = z_dev;
+  st->n_absorbed = 0;
+  return HF_OK;
+}
+
+HF_API hf_status hf_absorb_evicted(hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, int n_tokens, void* ws,
+                                   size_t ws_bytes, void* stream) {
+  if (!st || !st->S || !st->z || st->B < 1 || st->H < 1 || n_tokens < 0) return HF_ERR_INVALID_ARG;
+  if (!supported_d(st->d)) return HF_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return HF_OK;
+  if (!K_ev || !V_ev) return HF_ERR_INVALID_ARG;
+  if (!aligned16(K_ev) || !aligned16(V_ev) || !aligned16(st->S) || !aligned16(st->z)) return HF_ERR_ALIGNMENT;
+  const size_t need = absorb_ws_bytes(st->B, st->H, n_tokens, st->d);
+  if (!ws || ws_bytes < need) return HF_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const hf_status rc = st->d == 128 ? launch_absorb<128>(st, K_ev, V_ev, n_tokens, ws, s)
+                                    : launch_absorb<64>(st, K_ev, V_ev, n_tokens, ws, s);
+  if (rc == HF_OK) st->n_absorbed += n_tokens;
+  return rc;
+}
+
+HF_API hf_status hf_select_blocks(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk, int d,
+                                  int block, int r, int32_t* idx_out, float* scores_out, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  if (B < 1 || H < 1 || Nq < 0 || Nk < 1) return HF_ERR_INVALID_ARG;
+  if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
+  const int nKB = ceil_div(Nk, block);
+  if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
+  if (nKB > hf::kMaxKeyBlocks) return HF_ERR_UNSUPPORTED;
+  if (Nq == 0) return HF_OK;
+  if (!Q || !K || !idx_out) return HF_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(idx_out) || (scores_out && !aligned16(scores_out)))
+    return HF_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < select_ws_bytes(B, H, Nq, Nk, d, block)) return HF_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_select<128>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s)
+                  : launch_select<64>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s);
+}
+
+HF_API hf_status hf_hybrid_attn_fwd(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H, int Nq,
+                                    int Nk, int d, int block, int r, const int32_t* idx, const hf_state* st,
+                                    float scale, hf_bf16* O, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (B < 1 || H < 1 || Nq < 0 || Nk < 1 || !st) return HF_ERR_INVALID_ARG;
+  if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
+  const int nKB = ceil_div(Nk, block);
+  if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
+  if (st->B != B || st->H != H || st->d != d || !st->S || !st->z) return HF_ERR_INVALID_ARG;
+  if (!(scale == scale) || std::isinf(scale)) return HF_ERR_INVALID_ARG;
+  if (Nq == 0) return HF_OK;
+  if (!Q || !K || !V || !idx || !O) return HF_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx) || !aligned16(st->S) ||
+      !aligned16(st->z))
+    return HF_ERR_ALIGNMENT;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH * ceil_div(Nq, block) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int bh = static_cast<int>(BH);
+#define HF_ATTN_CASE(DD, BB) \
+  if (d == DD && block == BB) return launch_attn<DD, BB>(Q, K, V, bh, Nq, Nk, r, idx, st, sc, O, s);
+  HF_ATTN_CASE(128, 128)
+  HF_ATTN_CASE(128, 64)
+  HF_ATTN_CASE(128, 32)
+  HF_ATTN_CASE(64, 128)
+  HF_ATTN_CASE(64, 64)
+  HF_ATTN_CASE(64, 32)
+#undef HF_ATTN_CASE
+  return HF_ERR_UNSUPPORTED;
+}
+
+HF_API hf_status hf_query_status(void* stream, uint32_t* detail_out) {
+  if (detail_out) *detail_out = 0;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HF_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpyFromSymbol(&word, hf::g_hf_error_word, sizeof(word)) != cudaSuccess) return HF_ERR_CUDA;
+  if (word == 0) return HF_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(hf::g_hf_error_word, &zero, sizeof(zero)) != cudaSuccess) return HF_ERR_CUDA;
+  if (detail_out) *detail_out = word;
+  return (word >> 16) == 0x7200u ? HF_ERR_DEVICE_BAD_INDEX : HF_ERR_DEVICE_TIMEOUT;
+}
+
+HF_API hf_status hf_debug_inject_timeout(int kernel_id, int count, unsigned long long timeout_ns) {
+  if (kernel_id < 0 || kernel_id > 3 || count < 0) return HF_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_inject.kernel_id = (kernel_id == 0 || count == 0) ? 0 : kernel_id;
+  g_inject.count = count;
+  g_inject.timeout_ns = timeout_ns ? timeout_ns : kDefaultTimeoutNs;
+  return HF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,174 @@
+/*
+ * hf.h - C ABI of the hybrid attention chunk step (B200, sm_100a).
+ *
+ * The step is the attention of "Hybrid Forcing": for each new chunk of query tokens
+ * the output is the SUM of
+ *   (1) block-sparse softmax attention over the local sliding window of cached
+ *       frames, restricted to the top-r key blocks of every query block, and
+ *   (2) a linear-attention readout of a compact key-value state (S, z) that has
+ *       absorbed the tokens of every frame evicted from the window.
+ * Sources: "Long-Horizon Streaming Video Generation via Hybrid Attention with
+ * Decoupled Distillation" - German technical summary, section 2 A (linear temporal
+ * attention over a compact KV state; Top-K block-sparse SWA; output = sum), English
+ * abstract (state absorbs evicted tokens incrementally), Portuguese technical summary
+ * section 2 A.1/A.2; "Light Forcing: Accelerating Autoregressive Video Diffusion via
+ * Sparse Attention" - German technical summary, section 2.2 (mean-pooled block
+ * scores, selection per query block).
+ *
+ * Fixed readings of the open details:
+ *   phi(x) = elu(x) + 1 evaluated in fp32;
+ *   blocks are `block` consecutive tokens of the flattened sequence, the last block of
+ *   a sequence may be partial (its padding is excluded from pooling and masked);
+ *   score(I, J) = mean(q in I) . mean(k in J), unscaled, fp32;
+ *   each query block keeps the r best key blocks, ties to the lower index, listed in
+ *   ascending order;
+ *   sparse term: softmax(scale * q.k) over the valid tokens of the kept blocks,
+ *   scale = 1/sqrt(d) unless given, no causal mask inside the window;
+ *   linear term: phi(q)^T S / (phi(q) . z + 1e-6);
+ *   state update: S += phi(K)^T V, z += sum_t phi(k_t).
+ *
+ * Conventions for every call
+ *   - Tensors are dense row-major [B][H][N][d] (d innermost), bf16 unless stated.
+ *   - Every pointer is a DEVICE pointer of the current CUDA device unless stated, and
+ *     must be 16-byte aligned (TMA requirement).
+ *   - Supported: d in {64, 128}; block in {32, 64, 128}; 1 <= r <= nKB.
+ *   - The caller owns every buffer, including workspaces (size from
+ *     hf_workspace_size). The library allocates no device memory. Its only state is
+ *     one 32-bit device error word per GPU, read by hf_query_status.
+ *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). Argument errors are returned before anything is launched; a failed
+ *     launch returns HF_ERR_CUDA. A kernel that gives up on an internal wait (bounded,
+ *     about one second) records HF_ERR_DEVICE_TIMEOUT in the device error word
+ *     instead of hanging; hf_query_status reports it.
+ *   - Calls on one stream are ordered; calls whose buffers overlap must not run
+ *     concurrently on different streams.
+ */
+#ifndef HF_H_
+#define HF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define HF_API __attribute__((visibility("default")))
+#else
+#define HF_API
+#endif
+
+/* bfloat16 bit pattern (1 sign, 8 exponent, 7 mantissa bits). */
+typedef uint16_t hf_bf16;
+
+typedef enum hf_status {
+  HF_OK = 0,
+  HF_ERR_INVALID_ARG = 1,     /* null pointer, bad size, r outside [1, nKB], ...      */
+  HF_ERR_UNSUPPORTED = 2,     /* d or block outside the supported set                 */
+  HF_ERR_ALIGNMENT = 3,       /* a pointer is not 16-byte aligned                     */
+  HF_ERR_WORKSPACE = 4,       /* workspace missing or smaller than hf_workspace_size  */
+  HF_ERR_CUDA = 5,            /* a CUDA runtime/driver call or a launch failed        */
+  HF_ERR_DEVICE_TIMEOUT = 6,  /* a kernel gave up on an internal wait (device word)   */
+  HF_ERR_DEVICE_BAD_INDEX = 7 /* hf_hybrid_attn_fwd met a block index outside [0,nKB) */
+} hf_status;
+
+/* Compact key-value state of the linear temporal attention, one per (b, h):
+ *   S[b][h][k][n] = sum over absorbed tokens t of phi(k_t)[k] * v_t[n]   (fp32, d x d)
+ *   z[b][h][k]    = sum over absorbed tokens t of phi(k_t)[k]           (fp32, d)
+ * S and z are caller-owned device buffers of B*H*d*d and B*H*d floats. n_absorbed is a
+ * host-side count of tokens absorbed per head (bookkeeping only; the kernels do not
+ * read it). The state's size does not depend on how many tokens it has absorbed. */
+typedef struct hf_state {
+  int B, H, d;
+  float* S;
+  float* z;
+  long long n_absorbed;
+} hf_state;
+
+/* Workspace kinds for hf_workspace_size. */
+enum { HF_WS_SELECT = 1, HF_WS_ATTN = 2, HF_WS_ABSORB = 3 };
+
+/* Bytes of device workspace the call `which` needs (0 = none; NULL may be passed).
+ * For HF_WS_ABSORB pass the number of evicted tokens as Nk (Nq, block, r ignored).
+ * Returns (size_t)-1 for arguments the call would reject. Host-only, no CUDA call. */
+HF_API size_t hf_workspace_size(int which, int B, int H, int Nq, int Nk, int d, int block, int r);
+
+/* Bind S_dev / z_dev to *st and zero them (stream-ordered memset): the empty state.
+ * Errors: HF_ERR_INVALID_ARG (st/S_dev/z_dev NULL, B/H < 1), HF_ERR_UNSUPPORTED (d),
+ * HF_ERR_ALIGNMENT, HF_ERR_CUDA. */
+HF_API hf_status hf_state_init(hf_state* st, int B, int H, int d, float* S_dev, float* z_dev, void* stream);
+
+/* Absorb n_tokens evicted tokens per (b, h) into the state:
+ *   S += phi(K_ev)^T V_ev, z += sum_t phi(K_ev[t])   (K_ev, V_ev: [B][H][n_tokens][d])
+ * Source: Hybrid Forcing, German technical summary section 2 A (evicted frames are
+ * aggregated into the compact state by a linear attention function); English abstract.
+ * phi is evaluated in fp32; phi(K)^T V runs on the tensor cores with phi(K) split
+ * into two bf16 terms (hi + lo) and fp32 accumulation; the per-head reduction is
+ * deterministic (same inputs -> bit-identical state). n_tokens == 0 is a no-op.
+ * st->n_absorbed += n_tokens on success. ws: HF_WS_ABSORB bytes.
+ * Errors: HF_ERR_INVALID_ARG, HF_ERR_ALIGNMENT, HF_ERR_WORKSPACE, HF_ERR_CUDA. */
+HF_API hf_status hf_absorb_evicted(hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, int n_tokens,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/* Top-r key-block selection for every query block.
+ *   nQB = ceil(Nq/block), nKB = ceil(Nk/block)
+ *   score[b][h][I][J] = mean(Q rows of block I) . mean(K rows of block J)   (fp32)
+ *   idx_out[b][h][I][0..r) = the r blocks J of largest score, ties to the lower J,
+ *                            in ascending order                           (int32)
+ * Sources: Light Forcing, German technical summary section 2.2 (mean pooling at block
+ * level, selection per query block); Hybrid Forcing, German technical summary
+ * section 2 A (Top-K blocks). Q: [B][H][Nq][d], K: [B][H][Nk][d].
+ * scores_out: optional [B][H][nQB][nKB] fp32 (NULL to skip). NaN scores rank last.
+ * Nq == 0 is a no-op. ws: HF_WS_SELECT bytes.
+ * Errors: HF_ERR_INVALID_ARG (Nk < 1, r outside [1, nKB], NULL), HF_ERR_UNSUPPORTED,
+ * HF_ERR_ALIGNMENT, HF_ERR_WORKSPACE, HF_ERR_CUDA. */
+HF_API hf_status hf_select_blocks(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk, int d,
+                                  int block, int r, int32_t* idx_out, float* scores_out, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/* Hybrid attention output for the query chunk:
+ *   O[b][h][i] = sum_{j in kept(I(i))} softmax_j(scale * q_i . k_j) v_j
+ *              + phi(q_i)^T S[b][h] / (phi(q_i) . z[b][h] + 1e-6)
+ * where kept(I) are the valid tokens of the key blocks idx[b][h][I][0..r).
+ * Sources: Hybrid Forcing, German technical summary section 2 A ("Kombination": output
+ * = sum of the compressed global history and the sparse local interaction);
+ * Portuguese technical summary section 2 A.
+ * Q, O: [B][H][Nq][d]; K, V: [B][H][Nk][d] (the window); idx: [B][H][nQB][r] int32,
+ * normally from hf_select_blocks (any order is accepted; an index outside [0, nKB) is
+ * skipped and flagged as HF_ERR_DEVICE_BAD_INDEX in the device error word);
+ * st: the state (read only). scale <= 0 selects 1/sqrt(d). O is written in bf16
+ * (round to nearest even). Nq == 0 is a no-op. ws: none (HF_WS_ATTN = 0 bytes).
+ * The attention uses the state as it stands: a frame must be either in the window or
+ * absorbed in the state, never both.
+ * Errors: HF_ERR_INVALID_ARG, HF_ERR_UNSUPPORTED, HF_ERR_ALIGNMENT, HF_ERR_CUDA. */
+HF_API hf_status hf_hybrid_attn_fwd(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H,
+                                    int Nq, int Nk, int d, int block, int r, const int32_t* idx,
+                                    const hf_state* st, float scale, hf_bf16* O, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/* Synchronise `stream`, then read and clear the device error word of the current
+ * device. Returns HF_OK, HF_ERR_DEVICE_TIMEOUT, HF_ERR_DEVICE_BAD_INDEX or HF_ERR_CUDA
+ * (an asynchronous CUDA error). If detail_out is not NULL it receives the raw word
+ * (high 16 bits: error tag, low 16 bits: kernel id << 8 | wait site), 0 if none. */
+HF_API hf_status hf_query_status(void* stream, uint32_t* detail_out);
+
+/* Static description of a status code. */
+HF_API const char* hf_status_string(hf_status s);
+
+/* Library version string. */
+HF_API const char* hf_version(void);
+
+/* TEST ONLY. Makes the next `count` launches of kernel `kernel_id` (1 = select,
+ * 2 = absorb, 3 = attention) skip one internal barrier arrival, so that one wait runs
+ * out after `timeout_ns` nanoseconds; the kernel then records HF_ERR_DEVICE_TIMEOUT,
+ * drains its own copies and MMAs, frees its tensor memory and returns. The context
+ * stays usable. kernel_id 0 clears the injection. The bound of every other wait of
+ * those launches is also `timeout_ns`. Host-side setting of this library instance. */
+HF_API hf_status hf_debug_inject_timeout(int kernel_id, int count, unsigned long long timeout_ns);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HF_H_ */

@@ -1,0 +1,136 @@
+"""The C-ABI library on the CPU machine: it loads, exports every declared entry point, and
+rejects bad arguments before any CUDA call (no GPU needed for these paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hybrid_sparse_linear_hf_b200 as hf
+from hybrid_sparse_linear_hf_b200 import _binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hf.h")
+SIZE_MAX = (1 << (8 * ctypes.sizeof(ctypes.c_size_t))) - 1
+A = 0x100000  # a 16-byte aligned fake device address; never dereferenced on these paths
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"HF_API\s+[\w\s\*]+?\b(hf_\w+)\s*\(", text)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = hf.lib()
+    names = declared_symbols()
+    core = {"hf_state_init", "hf_absorb_evicted", "hf_select_blocks", "hf_hybrid_attn_fwd", "hf_workspace_size",
+            "hf_query_status", "hf_status_string", "hf_version", "hf_debug_inject_timeout"}
+    assert core <= set(names), sorted(core - set(names))
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/hf.h but not exported"
+    assert hf.hf_version().startswith("hf-b200")
+
+
+def test_status_strings():
+    for code in range(8):
+        s = hf.hf_status_string(code)
+        assert s.startswith("HF_")
+    assert "unknown" in hf.hf_status_string(42)
+
+
+def test_workspace_sizes():
+    # select: pooled Q and K, fp32, each 256-byte aligned
+    n = hf.hf_workspace_size(B.HF_WS_SELECT, 1, 12, 4680, 32760, 128, 128, 64)
+    assert n == 12 * 37 * 128 * 4 + 12 * 256 * 128 * 4
+    assert hf.hf_workspace_size(B.HF_WS_ATTN, 1, 12, 4680, 32760, 128, 128, 64) == 0
+    assert hf.hf_workspace_size(B.HF_WS_ABSORB, 1, 1, 0, 0, 64, 0, 0) == 0
+    # absorb: 12 heads spread over 12 slices each (144 CTAs)
+    assert hf.hf_workspace_size(B.HF_WS_ABSORB, 1, 12, 0, 93600, 128, 0, 0) == 12 * 12 * (128 * 128 + 128) * 4
+    with pytest.raises(hf.HfError):
+        hf.hf_workspace_size(B.HF_WS_SELECT, 1, 1, 64, 256, 96, 32, 2)
+    with pytest.raises(hf.HfError):
+        hf.hf_workspace_size(B.HF_WS_SELECT, 1, 1, 64, 256, 64, 32, 9)
+    with pytest.raises(hf.HfError):
+        hf.hf_workspace_size(7, 1, 1, 64, 256, 64, 32, 2)
+
+
+def _sel(**kw):
+    a = dict(Q=A, K=A, B=1, H=1, Nq=64, Nk=256, d=64, block=32, r=2, idx=A, scores=None, ws=A, ws_bytes=1 << 20)
+    a.update(kw)
+    return hf.lib().hf_select_blocks(a["Q"], a["K"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], a["block"], a["r"],
+                                     a["idx"], a["scores"], a["ws"], a["ws_bytes"], None)
+
+
+def test_select_validation():
+    assert _sel(d=96) == B.HF_ERR_UNSUPPORTED
+    assert _sel(block=48) == B.HF_ERR_UNSUPPORTED
+    assert _sel(r=0) == B.HF_ERR_INVALID_ARG
+    assert _sel(r=9) == B.HF_ERR_INVALID_ARG
+    assert _sel(Nk=0) == B.HF_ERR_INVALID_ARG
+    assert _sel(B=0) == B.HF_ERR_INVALID_ARG
+    assert _sel(Q=None) == B.HF_ERR_INVALID_ARG
+    assert _sel(Q=A + 2) == B.HF_ERR_ALIGNMENT
+    assert _sel(scores=A + 4) == B.HF_ERR_ALIGNMENT
+    assert _sel(ws=None) == B.HF_ERR_WORKSPACE
+    assert _sel(ws_bytes=100) == B.HF_ERR_WORKSPACE
+    assert _sel(Nq=0) == B.HF_OK  # empty query chunk: nothing to launch
+
+
+def _state(Bn=1, H=1, d=64):
+    st = B.HfStateC()
+    st.B, st.H, st.d, st.S, st.z, st.n_absorbed = Bn, H, d, A, A, 0
+    return st
+
+
+def _fwd(st=None, **kw):
+    a = dict(Q=A, K=A, V=A, B=1, H=1, Nq=64, Nk=256, d=64, block=32, r=2, idx=A, scale=0.0, O=A)
+    a.update(kw)
+    st = st or _state()
+    return hf.lib().hf_hybrid_attn_fwd(a["Q"], a["K"], a["V"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"],
+                                       a["block"], a["r"], a["idx"], ctypes.byref(st), a["scale"], a["O"],
+                                       None, 0, None)
+
+
+def test_attention_validation():
+    assert _fwd(d=32) == B.HF_ERR_UNSUPPORTED
+    assert _fwd(block=16) == B.HF_ERR_UNSUPPORTED
+    assert _fwd(r=9) == B.HF_ERR_INVALID_ARG
+    assert _fwd(st=_state(H=2)) == B.HF_ERR_INVALID_ARG
+    assert _fwd(st=_state(d=128)) == B.HF_ERR_INVALID_ARG
+    assert _fwd(scale=float("nan")) == B.HF_ERR_INVALID_ARG
+    assert _fwd(scale=float("inf")) == B.HF_ERR_INVALID_ARG
+    assert _fwd(V=None) == B.HF_ERR_INVALID_ARG
+    assert _fwd(O=A + 8) == B.HF_ERR_ALIGNMENT
+    assert _fwd(idx=A + 4) == B.HF_ERR_ALIGNMENT
+    assert _fwd(Nq=0) == B.HF_OK
+    assert hf.lib().hf_hybrid_attn_fwd(A, A, A, 1, 1, 64, 256, 64, 32, 2, A, None, 0.0, A, None, 0, None) \
+        == B.HF_ERR_INVALID_ARG
+
+
+def test_state_and_absorb_validation():
+    lib = hf.lib()
+    st = B.HfStateC()
+    assert lib.hf_state_init(None, 1, 1, 64, A, A, None) == B.HF_ERR_INVALID_ARG
+    assert lib.hf_state_init(ctypes.byref(st), 1, 1, 32, A, A, None) == B.HF_ERR_UNSUPPORTED
+    assert lib.hf_state_init(ctypes.byref(st), 1, 1, 64, A + 4, A, None) == B.HF_ERR_ALIGNMENT
+    assert lib.hf_state_init(ctypes.byref(st), 0, 1, 64, A, A, None) == B.HF_ERR_INVALID_ARG
+    s = _state()
+    assert lib.hf_absorb_evicted(ctypes.byref(s), A, A, -1, A, 1 << 30, None) == B.HF_ERR_INVALID_ARG
+    assert lib.hf_absorb_evicted(ctypes.byref(s), A, A, 0, None, 0, None) == B.HF_OK
+    assert s.n_absorbed == 0
+    assert lib.hf_absorb_evicted(ctypes.byref(s), A, A, 100, A, 16, None) == B.HF_ERR_WORKSPACE
+    assert lib.hf_absorb_evicted(ctypes.byref(s), A + 2, A, 100, A, 1 << 30, None) == B.HF_ERR_ALIGNMENT
+    assert lib.hf_absorb_evicted(None, A, A, 100, A, 1 << 30, None) == B.HF_ERR_INVALID_ARG
+
+
+def test_debug_injection_arguments():
+    assert hf.lib().hf_debug_inject_timeout(9, 1, 1000) == B.HF_ERR_INVALID_ARG
+    assert hf.lib().hf_debug_inject_timeout(2, -1, 1000) == B.HF_ERR_INVALID_ARG
+    assert hf.lib().hf_debug_inject_timeout(0, 0, 0) == B.HF_OK
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(B, "_lib", None)
+    monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "libhf.so"))
+    with pytest.raises(ImportError):
+        B.lib()

@@ -1,0 +1,313 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Inputs are the seeded bf16 tensors of ``hybrid_sparse_linear_hf_b200.inputs`` drawn on
+the CPU; the oracle sees them widened exactly to float64. Tolerances (tests/parity.py):
+masks bit-exact except near-ties (pooled scores within 1e-4), outputs max-abs 2e-2 and
+rel-L2 5e-3, the fp32 state rel-L2 1e-5. Output parity is checked against the oracle
+run on the GPU's own kept-block lists, so a legal tie swap never confounds it.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import hybrid_sparse_linear_hf_b200 as hf
+from hybrid_sparse_linear_hf_b200.inputs import WORKLOADS, Workload, draw_step_inputs, frame_structured
+from tests.parity import (assert_masks_match, assert_output_close, assert_state_close, f64, SCORE_ABS)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _gen(seed, B, H, N, d, tpf=64, w=0.0):
+    g = torch.Generator().manual_seed(seed)
+    return frame_structured(g, B, H, N, d, tpf, w)
+
+
+def _run_select(Q, K, block, r):
+    nQB, nKB = -(-Q.shape[2] // block), -(-K.shape[2] // block)
+    scores = torch.empty(Q.shape[0], Q.shape[1], nQB, nKB, dtype=torch.float32, device=DEV)
+    idx = hf.hf_select_blocks(Q.to(DEV), K.to(DEV), block, r, scores_out=scores)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), scores.cpu().numpy().astype(np.float64)
+
+
+def _state_from(K_ev, V_ev, d):
+    B, H = K_ev.shape[:2]
+    S = torch.empty(B, H, d, d, dtype=torch.float32, device=DEV)
+    z = torch.empty(B, H, d, dtype=torch.float32, device=DEV)
+    st = hf.hf_state_init(S, z)
+    hf.hf_absorb_evicted(st, K_ev.to(DEV), V_ev.to(DEV))
+    torch.cuda.synchronize()
+    return st
+
+
+def _check_status():
+    rc, word = hf.hf_query_status()
+    assert rc == hf.HF_OK, f"device status {rc} word {word:#x}"
+
+
+# --------------------------------------------------------------------------- select
+@pytest.mark.parametrize("B,H,Nq,Nk,d,block,r", [
+    (1, 1, 64, 256, 64, 32, 2),        # the tiny workload's shape
+    (1, 2, 100, 300, 64, 32, 5),       # ragged query and key tails
+    (2, 3, 257, 1000, 128, 128, 3),    # ragged, several heads and batches
+    (1, 4, 128, 640, 128, 64, 10),
+    (1, 2, 33, 129, 128, 128, 2),      # 1-token key tail
+    (1, 1, 64, 4096, 64, 32, 128),     # many key blocks
+    (1, 2, 300, 2000, 128, 128, 16),   # r = nKB
+])
+def test_select_matches_oracle(B, H, Nq, Nk, d, block, r):
+    Q = _gen(1, B, H, Nq, d, w=0.5)
+    K = _gen(2, B, H, Nk, d, w=0.5)
+    idx, scores = _run_select(Q, K, block, r)
+    oidx, osc = oracle.select_blocks(f64(Q), f64(K), block, r)
+    assert np.abs(scores - osc).max() <= SCORE_ABS
+    assert_masks_match(idx, oidx, osc, r)
+    _check_status()
+
+
+def test_select_ties_lower_index():
+    """Duplicated key blocks produce exactly equal pooled scores: the lower index wins."""
+    d, block = 64, 32
+    base = _gen(3, 1, 1, 4 * block, d)
+    K = torch.cat([base, base], dim=2)  # block 4+i duplicates block i
+    Q = _gen(4, 1, 1, 2 * block, d)
+    for r in range(1, 9):
+        idx, scores = _run_select(Q, K, block, r)
+        oidx, osc = oracle.select_blocks(f64(Q), f64(K), block, r)
+        assert np.array_equal(idx, oidx), (r, idx, oidx)
+        for row in idx.reshape(-1, r):
+            for J in row:
+                if J >= 4:
+                    assert J - 4 in row
+
+
+# --------------------------------------------------------------------------- absorb
+@pytest.mark.parametrize("B,H,n,d", [(1, 1, 192, 64), (1, 2, 1000, 128), (2, 3, 77, 128), (1, 12, 4680, 128),
+                                     (1, 1, 1, 64), (1, 40, 130, 64),
+                                     (1, 148, 4000, 128)])  # one slice per head: 63 tiles per CTA
+def test_absorb_matches_oracle(B, H, n, d):
+    K_ev = _gen(5, B, H, n, d, w=0.5)
+    V_ev = _gen(6, B, H, n, d, w=0.5)
+    st = _state_from(K_ev, V_ev, d)
+    S_o, z_o = oracle.absorb_batch(f64(K_ev), f64(V_ev))
+    assert_state_close(f64(st.S), f64(st.z), S_o, z_o)
+    assert st.n_absorbed == n
+    _check_status()
+
+
+def test_absorb_deterministic_and_incremental():
+    d = 128
+    K_ev = _gen(7, 1, 3, 3000, d, w=0.5)
+    V_ev = _gen(8, 1, 3, 3000, d, w=0.5)
+    a = _state_from(K_ev, V_ev, d)
+    b = _state_from(K_ev, V_ev, d)
+    assert torch.equal(a.S, b.S) and torch.equal(a.z, b.z), "absorption must be bit-reproducible"
+    # incremental in uneven pieces == oracle batch
+    S = torch.empty(1, 3, d, d, device=DEV)
+    z = torch.empty(1, 3, d, device=DEV)
+    st = hf.hf_state_init(S, z)
+    for lo, hi in [(0, 1), (1, 65), (65, 1000), (1000, 3000)]:
+        hf.hf_absorb_evicted(st, K_ev[:, :, lo:hi].contiguous().to(DEV), V_ev[:, :, lo:hi].contiguous().to(DEV))
+    torch.cuda.synchronize()
+    S_o, z_o = oracle.absorb_batch(f64(K_ev), f64(V_ev))
+    assert_state_close(f64(st.S), f64(st.z), S_o, z_o)
+    _check_status()
+
+
+# --------------------------------------------------------------------------- attention
+def _attn_case(B, H, Nq, Nk, d, block, r, n_state, seed=10, w=0.5, scale=0.0):
+    Q = _gen(seed, B, H, Nq, d, w=w)
+    K = _gen(seed + 1, B, H, Nk, d, w=w)
+    V = _gen(seed + 2, B, H, Nk, d, w=w)
+    K_ev = _gen(seed + 3, B, H, n_state, d, w=w)
+    V_ev = _gen(seed + 4, B, H, n_state, d, w=w)
+    if n_state:
+        st = _state_from(K_ev, V_ev, d)
+    else:
+        S = torch.empty(B, H, d, d, device=DEV)
+        z = torch.empty(B, H, d, device=DEV)
+        st = hf.hf_state_init(S, z)
+    idx = hf.hf_select_blocks(Q.to(DEV), K.to(DEV), block, r)
+    O = hf.hf_hybrid_attn_fwd(Q.to(DEV), K.to(DEV), V.to(DEV), block, r, idx, st, scale=scale)
+    torch.cuda.synchronize()
+    _check_status()
+    return Q, K, V, st, idx.cpu().numpy(), O
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,d,block,r,n_state", [
+    (1, 1, 64, 256, 64, 32, 2, 192),        # the tiny workload's shape
+    (1, 2, 300, 1000, 128, 128, 3, 500),    # ragged query tail (44 rows) and key tail (104)
+    (1, 2, 200, 700, 128, 64, 4, 300),
+    (1, 2, 100, 300, 128, 32, 3, 64),
+    (1, 3, 130, 900, 64, 128, 5, 129),
+    (1, 2, 96, 400, 64, 64, 7, 0),          # empty state: O = sparse term
+    (2, 2, 256, 1024, 128, 128, 8, 256),    # r = nKB: dense window attention
+    (1, 1, 128, 129, 128, 128, 2, 10),      # 1-token key tail
+])
+def test_attention_matches_oracle(B, H, Nq, Nk, d, block, r, n_state):
+    Q, K, V, st, idx, O = _attn_case(B, H, Nq, Nk, d, block, r, n_state)
+    want = oracle.hybrid_attention(f64(Q), f64(K), f64(V), idx, f64(st.S), f64(st.z), block)
+    assert_output_close(f64(O), want)
+
+
+def test_attention_dense_equals_window_attention_plus_readout():
+    """Keeping every block equals dense sliding-window attention plus the readout."""
+    B, H, Nq, Nk, d, block = 1, 2, 64, 256, 64, 32
+    Q, K, V, st, idx, O = _attn_case(B, H, Nq, Nk, d, block, 8, 192, seed=20, w=0.0)
+    want = oracle.dense_swa(f64(Q), f64(K), f64(V)) + oracle.linear_readout(f64(Q), f64(st.S), f64(st.z))
+    assert_output_close(f64(O), want)
+
+
+def test_attention_custom_scale_and_unsorted_idx():
+    B, H, Nq, Nk, d, block, r = 1, 2, 128, 512, 128, 64, 3
+    Q, K, V, st, idx, O = _attn_case(B, H, Nq, Nk, d, block, r, 100, seed=30, scale=0.05)
+    want = oracle.hybrid_attention(f64(Q), f64(K), f64(V), idx, f64(st.S), f64(st.z), block, scale=0.05)
+    assert_output_close(f64(O), want)
+    # reversed index order gives the same result
+    ridx = torch.from_numpy(np.ascontiguousarray(idx[..., ::-1])).to(DEV)
+    O2 = hf.hf_hybrid_attn_fwd(Q.to(DEV), K.to(DEV), V.to(DEV), block, r, ridx, st, scale=0.05)
+    torch.cuda.synchronize()
+    assert_output_close(f64(O2), want)
+
+
+def test_attention_bad_index_is_skipped_and_flagged():
+    B, H, Nq, Nk, d, block, r = 1, 1, 64, 256, 64, 32, 3
+    Q, K, V, st, idx, O = _attn_case(B, H, Nq, Nk, d, block, r, 64, seed=40)
+    bad = idx.copy()
+    bad[0, 0, 0, 1] = 99   # out of range: skipped
+    bad[0, 0, 1, 0] = -1
+    O2 = hf.hf_hybrid_attn_fwd(Q.to(DEV), K.to(DEV), V.to(DEV), block, r, torch.from_numpy(bad).to(DEV), st)
+    rc, word = hf.hf_query_status()
+    assert rc == hf.HF_ERR_DEVICE_BAD_INDEX, (rc, hex(word))
+    assert hf.hf_query_status()[0] == hf.HF_OK  # cleared
+    for I, keep in [(0, [idx[0, 0, 0, 0], idx[0, 0, 0, 2]]), (1, [idx[0, 0, 1, 1], idx[0, 0, 1, 2]])]:
+        kidx = np.zeros((1, 1, 2, 2), dtype=np.int32)
+        kidx[0, 0, I] = keep
+        want = oracle.hybrid_attention_tile(f64(Q), f64(K), f64(V), kidx, f64(st.S), f64(st.z), block, 0, 0, I)
+        assert_output_close(f64(O2)[0, 0, I * block:(I + 1) * block], want)
+
+
+def test_empty_inputs_are_noops():
+    d = 64
+    S = torch.empty(1, 1, d, d, device=DEV)
+    z = torch.empty(1, 1, d, device=DEV)
+    st = hf.hf_state_init(S, z)
+    e = torch.empty(1, 1, 0, d, dtype=torch.bfloat16, device=DEV)
+    hf.hf_absorb_evicted(st, e, e)
+    K = _gen(1, 1, 1, 64, d).to(DEV)
+    idx = torch.empty(1, 1, 0, 1, dtype=torch.int32, device=DEV)
+    hf.hf_select_blocks(e, K, 32, 1, idx_out=idx)
+    O = hf.hf_hybrid_attn_fwd(e, K, K, 32, 1, idx, st)
+    torch.cuda.synchronize()
+    assert O.numel() == 0 and float(S.abs().sum()) == 0.0 and st.n_absorbed == 0
+    _check_status()
+
+
+# --------------------------------------------------------------------------- workloads
+def test_tiny_workload_step():
+    wl = WORKLOADS["tiny"]
+    x = draw_step_inputs(wl)
+    Q, K, V, K_ev, V_ev = (x[k] for k in ("Q", "K", "V", "K_ev", "V_ev"))
+    st = _state_from(K_ev, V_ev, wl.d)
+    idx, scores = _run_select(Q, K, wl.block, wl.r)
+    oidx, osc = oracle.select_blocks(f64(Q), f64(K), wl.block, wl.r)
+    assert_masks_match(idx, oidx, osc, wl.r)
+    O = hf.hf_hybrid_attn_fwd(Q.to(DEV), K.to(DEV), V.to(DEV), wl.block, wl.r, torch.from_numpy(idx).to(DEV), st)
+    torch.cuda.synchronize()
+    S_o, z_o = oracle.absorb_batch(f64(K_ev), f64(V_ev))
+    assert_state_close(f64(st.S), f64(st.z), S_o, z_o)
+    want = oracle.hybrid_attention(f64(Q), f64(K), f64(V), idx, S_o, z_o, wl.block)
+    assert_output_close(f64(O), want)
+    _check_status()
+
+
+@pytest.mark.parametrize("keep", [1.0, 0.5, 0.25, 0.125])
+def test_sparsity_sweep_tiny(keep):
+    wl = WORKLOADS["tiny"].with_keep(keep)
+    x = draw_step_inputs(wl)
+    Q, K, V, K_ev, V_ev = (x[k] for k in ("Q", "K", "V", "K_ev", "V_ev"))
+    st = _state_from(K_ev, V_ev, wl.d)
+    idx = hf.hf_select_blocks(Q.to(DEV), K.to(DEV), wl.block, wl.r)
+    O = hf.hf_hybrid_attn_fwd(Q.to(DEV), K.to(DEV), V.to(DEV), wl.block, wl.r, idx, st)
+    torch.cuda.synchronize()
+    idx = idx.cpu().numpy()
+    oidx, osc = oracle.select_blocks(f64(Q), f64(K), wl.block, wl.r)
+    assert_masks_match(idx, oidx, osc, wl.r)
+    want = oracle.hybrid_attention(f64(Q), f64(K), f64(V), idx, f64(st.S), f64(st.z), wl.block)
+    assert_output_close(f64(O), want)
+    if keep == 1.0:
+        dense = oracle.dense_swa(f64(Q), f64(K), f64(V)) + oracle.linear_readout(f64(Q), f64(st.S), f64(st.z))
+        assert_output_close(f64(O), dense)
+    _check_status()
+
+
+def test_streaming_300_steps():
+    """300 chunk steps at the tiny shape; each step evicts 3 fresh frames into the state.
+    The fp32 state is checked against a float64 batch recompute at steps 10, 100, 300,
+    and the step output against the oracle at the same steps."""
+    wl = WORKLOADS["tiny"]
+    d = wl.d
+    S = torch.empty(1, 1, d, d, device=DEV)
+    z = torch.empty(1, 1, d, device=DEV)
+    st = hf.hf_state_init(S, z)
+    ev_k, ev_v = [], []
+    for t in range(1, 301):
+        x = draw_step_inputs(wl, seed=10000 + t, n_evicted=wl.Ne_step)
+        Qd, Kd, Vd = x["Q"].to(DEV), x["K"].to(DEV), x["V"].to(DEV)
+        idx = hf.hf_select_blocks(Qd, Kd, wl.block, wl.r)
+        O = hf.hf_hybrid_attn_fwd(Qd, Kd, Vd, wl.block, wl.r, idx, st)
+        if t in (10, 100, 300):
+            torch.cuda.synchronize()
+            S_before, z_before = f64(st.S), f64(st.z)
+            want = oracle.hybrid_attention(f64(x["Q"]), f64(x["K"]), f64(x["V"]), idx.cpu().numpy(),
+                                           S_before, z_before, wl.block)
+            assert_output_close(f64(O), want, what=f"O at step {t}")
+        hf.hf_absorb_evicted(st, x["K_ev"].to(DEV), x["V_ev"].to(DEV))
+        ev_k.append(x["K_ev"])
+        ev_v.append(x["V_ev"])
+        if t in (10, 100, 300):
+            torch.cuda.synchronize()
+            S_o, z_o = oracle.absorb_batch(f64(torch.cat(ev_k, 2)), f64(torch.cat(ev_v, 2)))
+            assert_state_close(f64(st.S), f64(st.z), S_o, z_o)
+    assert st.n_absorbed == 300 * wl.Ne_step
+    _check_status()
+
+
+def _sample_tiles(wl, n, seed=0):
+    rng = np.random.default_rng(seed)
+    tiles = {(0, h, int(rng.integers(0, wl.nQB))) for h in rng.integers(0, wl.H, size=n)}
+    tiles.add((0, wl.H - 1, wl.nQB - 1))  # the partial last query block
+    tiles.add((0, 0, 0))
+    return sorted(tiles)
+
+
+@pytest.mark.parametrize("name", ["832x480"])
+def test_full_size_workload_sampled(name):
+    """The full 832x480-shaped step in the bench's launch configuration: every mask, the
+    whole state, and the outputs of sampled query blocks against the oracle."""
+    wl = WORKLOADS[name]
+    x = draw_step_inputs(wl)
+    Qd, Kd, Vd = x["Q"].to(DEV), x["K"].to(DEV), x["V"].to(DEV)
+    st = _state_from(x["K_ev"], x["V_ev"], wl.d)
+    nKB = wl.nKB
+    scores = torch.empty(wl.B, wl.H, wl.nQB, nKB, device=DEV)
+    idx_t = hf.hf_select_blocks(Qd, Kd, wl.block, wl.r, scores_out=scores)
+    O = hf.hf_hybrid_attn_fwd(Qd, Kd, Vd, wl.block, wl.r, idx_t, st)
+    torch.cuda.synchronize()
+    _check_status()
+    idx = idx_t.cpu().numpy()
+    Q64, K64, V64 = f64(x["Q"]), f64(x["K"]), f64(x["V"])
+    oidx, osc = oracle.select_blocks(Q64, K64, wl.block, wl.r)
+    assert np.abs(scores.cpu().numpy() - osc).max() <= SCORE_ABS
+    assert_masks_match(idx, oidx, osc, wl.r)
+    S_o, z_o = oracle.absorb_batch(f64(x["K_ev"]), f64(x["V_ev"]))
+    assert_state_close(f64(st.S), f64(st.z), S_o, z_o)
+    Og = f64(O)
+    for (b, h, I) in _sample_tiles(wl, 6):
+        lo, hi = I * wl.block, min((I + 1) * wl.block, wl.Nq)
+        want = oracle.hybrid_attention_tile(Q64, K64, V64, idx, S_o, z_o, wl.block, b, h, I)
+        assert_output_close(Og[b, h, lo:hi], want, what=f"O tile {(b, h, I)}")
