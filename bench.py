@@ -20,6 +20,7 @@ the same step, scaled to the whole step) on the host cores.
 from __future__ import annotations
 
 import argparse
+import faulthandler
 import json
 import math
 import os
@@ -45,6 +46,16 @@ LAUNCHES_PER_STEP = 5  # pool, score+select, hybrid attention, absorb partials, 
 
 
 # ----------------------------------------------------------------------------- helpers
+_T0 = time.time()
+_VERBOSE = False
+
+
+def log(msg: str) -> None:
+    """Progress line on stderr (``--verbose``)."""
+    if _VERBOSE:
+        print(f"[bench {time.time() - _T0:8.2f}s] {msg}", file=sys.stderr, flush=True)
+
+
 def load_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -224,6 +235,7 @@ def run_gpu(args, wl) -> None:
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
 
+    log(f"rank {rank}/{world} on {dev}")
     # ---- inputs, drawn on the device (same recipe, device generator), resident in HBM
     x = draw_step_inputs(wl, seed=wl.seed + 1000 * rank, n_evicted=wl.Ne_step, device=dev)
     Q, K, V, K_ev, V_ev = (x[k] for k in ("Q", "K", "V", "K_ev", "V_ev"))
@@ -241,6 +253,8 @@ def run_gpu(args, wl) -> None:
     zb = torch.empty_like(z)
     stb = hf.hf_state_init(Sb, zb)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    log("inputs drawn; timing the state build")
     build_times = []
     for i in range(4):
         flush.zero_()
@@ -251,8 +265,11 @@ def run_gpu(args, wl) -> None:
         torch.cuda.synchronize(dev)
         if i > 0:
             build_times.append(e0.elapsed_time(e1) * 1e-3)
+        log(f"state build {i}: {e0.elapsed_time(e1):.3f} ms")
     hf.hf_absorb_evicted(st, build_K, build_V, ws=ws_abs_build)
-    del build_K, build_V, ws_abs_build
+    torch.cuda.synchronize(dev)
+    del build_K, build_V, ws_abs_build, Sb, zb, stb
+    torch.cuda.empty_cache()
     ws_sel = torch.empty(hf.hf_workspace_size(hf.HF_WS_SELECT, wl.B, wl.H, wl.Nq, wl.Nk, wl.d, wl.block, wl.r),
                          dtype=torch.uint8, device=dev)
     ws_abs = torch.empty(hf.hf_workspace_size(hf.HF_WS_ABSORB, wl.B, wl.H, 0, wl.Ne_step, wl.d, 0, 0),
@@ -273,9 +290,13 @@ def run_gpu(args, wl) -> None:
         if ev:
             ev[3].record(stream)
 
-    for _ in range(max(args.warmup, 3)):
+    log("warm-up")
+    for i in range(max(args.warmup, 3)):
         flush.zero_()
         step()
+        if _VERBOSE:
+            torch.cuda.synchronize(dev)
+            log(f"warm-up step {i} done")
     torch.cuda.synchronize(dev)
     rc, word = hf.hf_query_status()
     if rc != hf.HF_OK:
@@ -286,6 +307,7 @@ def run_gpu(args, wl) -> None:
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
+    log("timed steps")
     with ClockSampler(dev.index) as clk:
         for k in range(args.steps):
             flush.zero_()
@@ -306,6 +328,7 @@ def run_gpu(args, wl) -> None:
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         t_step = float(tt.item())
 
+    log(f"timed: {t_step_local * 1e3:.3f} ms/step; end-to-end leg")
     # ---- end to end through the public API with host buffers (pinned), copies timed
     host = {k: v.cpu().pin_memory() for k, v in x.items()}
     O_host = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
@@ -383,6 +406,7 @@ def run_gpu(args, wl) -> None:
                 "d2h_bytes_per_step": d2h, "steps": n_e2e,
                 "note": "pinned host Q, K/V window, evicted K/V copied in and O copied out every step"},
     }
+    log("cpu baseline")
     if world == 1 and not args.no_cpu_baseline:
         # bounded sample of the fp64 oracle on the host cores: whole heads until ~10 s
         ev_k, ev_v = K_ev.cpu(), V_ev.cpu()
@@ -408,7 +432,14 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["hf", "reference"], default="hf")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle CPU-baseline leg")
+    ap.add_argument("--verbose", action="store_true", help="progress lines on stderr")
+    ap.add_argument("--watchdog", type=float, default=0.0,
+                    help="dump the Python stacks and exit if the run exceeds this many seconds")
     args = ap.parse_args()
+    global _VERBOSE
+    _VERBOSE = args.verbose
+    if args.watchdog > 0:
+        faulthandler.dump_traceback_later(args.watchdog, exit=True)
     wl = WORKLOADS[WORKLOAD]
     if args.impl == "reference":
         run_reference(args, wl)

@@ -210,7 +210,10 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     bool ok = true;
     auto flush_group = [&](int g) {
       const int b = g & 1;
-      if (!mbar_wait(&dfull_bar[b], (g >> 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 8)) return false;
+      // the TMEM loads below are warp-collective: the wait result is made warp-uniform
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&dfull_bar[b], (g >> 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 8)))
+        return false;
       tc_fence_after();
 #pragma unroll
       for (int c0 = 0; c0 < D; c0 += 32) {
@@ -230,6 +233,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       ok = mbar_wait(&full_bar[s], (i / kAbsStages) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 6);
       if (ok && i >= 2) ok = mbar_wait(&aempty_bar[a], ((i >> 1) - 1) & 1, abort_flag, p.timeout_ns,
                                        (kKernAbsorb << 8) | 7);
+      ok = __all_sync(0xffffffffu, ok);  // the warp stays converged for the collective drain
       if (!ok) break;
       const uint8_t* ktile = ring + s * C::kStageBytes;
       uint8_t* ahi = abuf + a * C::kABufBytes;

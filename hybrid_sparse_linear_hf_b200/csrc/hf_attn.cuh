@@ -241,7 +241,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    bool ok = mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 9);
+    // tcgen05.ld/st are warp-collective: every wait that guards one is made warp-uniform
+    bool ok = __all_sync(0xffffffffu, mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 9));
     float den = 1.0f;
     if (ok) {
       // ---- prologue: phi(q) hi/lo -> TMEM, den = phi(q).z + 1e-6, S -> bf16 hi/lo in smem
@@ -309,8 +310,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int J = __ldg(idx_row + jj);
       if (J < 0 || J >= p.nKB) continue;
       const int b = j & 1;
-      if (!(ok = mbar_wait(&sfull_bar[b], (j >> 1) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 10)))
-        break;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sfull_bar[b], (j >> 1) & 1, abort_flag, p.timeout_ns,
+                                             (kKernAttn << 8) | 10));
+      if (!ok) break;
       tc_fence_after();
       const uint32_t s_addr = lane_addr + (b ? C::kColS1 : C::kColS0);
       uint32_t sr[BLK];
@@ -331,22 +333,32 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mx *= p.scale_log2;
       if (j == 0) {
         m_run = mx;
-      } else if (mx > m_run + 8.0f) {
-        const float alpha = ex2_approx(m_run - mx);
-        if (!(ok = mbar_wait(&odone_bar, (j - 1) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 11))) break;
-        tc_fence_after();
+      } else {
+        // A row raises its running max only when the block max exceeds it by more than
+        // 8 (log2 units); the O rescale is done by the whole warp whenever any of its
+        // rows needs it (alpha = 1 for the others), since TMEM access is warp-collective.
+        const bool need = mx > m_run + 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m_run - mx) : 1.0f;
+          ok = __all_sync(0xffffffffu, mbar_wait(&odone_bar, (j - 1) & 1, abort_flag, p.timeout_ns,
+                                                 (kKernAttn << 8) | 11));
+          if (!ok) break;
+          tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + C::kColO + c, o);
-          tmem_wait_ld();
-          reg_fence<32>(o);
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + C::kColO + c, o);
+            tmem_wait_ld();
+            reg_fence<32>(o);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(lane_addr + C::kColO + c, o);
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(lane_addr + C::kColO + c, o);
+          }
+          if (need) {
+            l_run *= alpha;
+            m_run = mx;
+          }
         }
-        l_run *= alpha;
-        m_run = mx;
       }
       float lsum = 0.f;
       uint32_t pk[BLK / 2];
@@ -369,6 +381,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // ---- epilogue: O = O_s / l + O_lin / den -> bf16 -> TMA store of the block's rows
     if (ok) ok = mbar_wait(&final_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 12) &&
                  mbar_wait(&lin_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 13);
+    ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
       const float inv_l = (j > 0 && l_run > 0.f) ? 1.0f / l_run : 0.0f;

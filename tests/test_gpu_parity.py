@@ -311,3 +311,59 @@ def test_full_size_workload_sampled(name):
         lo, hi = I * wl.block, min((I + 1) * wl.block, wl.Nq)
         want = oracle.hybrid_attention_tile(Q64, K64, V64, idx, S_o, z_o, wl.block, b, h, I)
         assert_output_close(Og[b, h, lo:hi], want, what=f"O tile {(b, h, I)}")
+
+
+def test_attention_online_rescale_mixed_rows():
+    """Even query rows meet much larger scores in later blocks (their running max must be
+    raised twice, rescaling O) while odd rows do not: every warp mixes both cases."""
+    d, block, Nq, Nk = 128, 128, 256, 4 * 128
+    g = torch.Generator().manual_seed(77)
+    Q = torch.randn(1, 2, Nq, d, generator=g) * 0.3
+    Q[:, :, 0::2, 0] = 3.0
+    K = torch.randn(1, 2, Nk, d, generator=g) * 0.3
+    V = torch.randn(1, 2, Nk, d, generator=g)
+    K[:, :, 2 * block:3 * block, 0] = 40.0   # block 2: scores ~120 for even rows
+    K[:, :, 3 * block:4 * block, 0] = 70.0   # block 3: scores ~210 for even rows
+    Q, K, V = Q.bfloat16(), K.bfloat16(), V.bfloat16()
+    S = torch.empty(1, 2, d, d, device=DEV)
+    z = torch.empty(1, 2, d, device=DEV)
+    st = hf.hf_state_init(S, z)
+    hf.hf_absorb_evicted(st, _gen(1, 1, 2, 100, d).to(DEV), _gen(2, 1, 2, 100, d).to(DEV))
+    for order in ([0, 1, 2, 3], [3, 2, 1, 0], [1, 3, 0, 2]):
+        idx = torch.tensor(order, dtype=torch.int32).repeat(1, 2, 2, 1).contiguous()
+        O = hf.hf_hybrid_attn_fwd(Q.to(DEV), K.to(DEV), V.to(DEV), block, 4, idx.to(DEV), st)
+        torch.cuda.synchronize()
+        _check_status()
+        want = oracle.hybrid_attention(f64(Q), f64(K), f64(V), idx.numpy(), f64(st.S), f64(st.z), block)
+        assert_output_close(f64(O), want, what=f"O order {order}")
+
+
+def test_bench_step_sequence_on_device_drawn_inputs():
+    """The bench's loop (select -> hybrid attention -> absorb of the step's evicted
+    frames, back to back without host syncs) on inputs drawn by the device generator,
+    checked on sampled tiles after several steps."""
+    wl = WORKLOADS["832x480"]
+    x = draw_step_inputs(wl, seed=123, n_evicted=wl.Ne_step, device=DEV)
+    S = torch.empty(wl.B, wl.H, wl.d, wl.d, device=DEV)
+    z = torch.empty(wl.B, wl.H, wl.d, device=DEV)
+    st = hf.hf_state_init(S, z)
+    gen = torch.Generator(device=DEV).manual_seed(5)
+    bk = frame_structured(gen, wl.B, wl.H, 20 * wl.tokens_per_frame, wl.d, wl.tokens_per_frame, wl.w, device=DEV)
+    bv = frame_structured(gen, wl.B, wl.H, 20 * wl.tokens_per_frame, wl.d, wl.tokens_per_frame, wl.w, device=DEV)
+    hf.hf_absorb_evicted(st, bk, bv)
+    idx = torch.empty(wl.B, wl.H, wl.nQB, wl.r, dtype=torch.int32, device=DEV)
+    O = torch.empty_like(x["Q"])
+    for _ in range(4):
+        hf.hf_select_blocks(x["Q"], x["K"], wl.block, wl.r, idx_out=idx)
+        S_before, z_before = st.S.clone(), st.z.clone()
+        hf.hf_hybrid_attn_fwd(x["Q"], x["K"], x["V"], wl.block, wl.r, idx, st, O=O)
+        hf.hf_absorb_evicted(st, x["K_ev"], x["V_ev"])
+    torch.cuda.synchronize()
+    _check_status()
+    Q64, K64, V64 = f64(x["Q"]), f64(x["K"]), f64(x["V"])
+    idx_h = idx.cpu().numpy()
+    Og = f64(O)
+    for (b, h, I) in _sample_tiles(wl, 4, seed=1):
+        lo, hi = I * wl.block, min((I + 1) * wl.block, wl.Nq)
+        want = oracle.hybrid_attention_tile(Q64, K64, V64, idx_h, f64(S_before), f64(z_before), wl.block, b, h, I)
+        assert_output_close(Og[b, h, lo:hi], want, what=f"O tile {(b, h, I)}")
