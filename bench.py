@@ -91,6 +91,25 @@ def absorb_bytes(wl, n_tokens) -> float:
     return 2.0 * 2 * wl.B * wl.H * n_tokens * wl.d + 2 * 4.0 * wl.B * wl.H * (wl.d * wl.d + wl.d)
 
 
+def max_over_ranks(t_local: float, dist=None, device="cpu") -> float:
+    """The slowest rank's time (every rank takes the same collective step)."""
+    if dist is None:
+        return t_local
+    tt = torch.tensor([t_local], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_throughput(world: int, B: int, Nq: int, t_step: float) -> float:
+    """Whole-job query tokens/s: every rank processes its own B x Nq chunk per step."""
+    return world * B * Nq / t_step
+
+
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Each rank streams its own synthetic chunk (independent inputs, same recipe)."""
+    return base_seed + 1000 * rank
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -237,7 +256,7 @@ def run_gpu(args, wl) -> None:
 
     log(f"rank {rank}/{world} on {dev}")
     # ---- inputs, drawn on the device (same recipe, device generator), resident in HBM
-    x = draw_step_inputs(wl, seed=wl.seed + 1000 * rank, n_evicted=wl.Ne_step, device=dev)
+    x = draw_step_inputs(wl, seed=rank_seed(wl.seed, rank), n_evicted=wl.Ne_step, device=dev)
     Q, K, V, K_ev, V_ev = (x[k] for k in ("Q", "K", "V", "K_ev", "V_ev"))
     S = torch.empty(wl.B, wl.H, wl.d, wl.d, dtype=torch.float32, device=dev)
     z = torch.empty(wl.B, wl.H, wl.d, dtype=torch.float32, device=dev)
@@ -322,11 +341,7 @@ def run_gpu(args, wl) -> None:
     t_fwd = [e[1].elapsed_time(e[2]) * 1e-3 for e in events]
     t_abs = [e[2].elapsed_time(e[3]) * 1e-3 for e in events]
     t_step_local = sum(e[0].elapsed_time(e[3]) for e in events) * 1e-3 / args.steps
-    t_step = t_step_local
-    if dist:
-        tt = torch.tensor([t_step_local], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_step = float(tt.item())
+    t_step = max_over_ranks(t_step_local, dist, dev)
 
     log(f"timed: {t_step_local * 1e3:.3f} ms/step; end-to-end leg")
     # ---- end to end through the public API with host buffers (pinned), copies timed
@@ -358,11 +373,8 @@ def run_gpu(args, wl) -> None:
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    t_e2e = e0.elapsed_time(e1) * 1e-3 / n_e2e
+    t_e2e = max_over_ranks(e0.elapsed_time(e1) * 1e-3 / n_e2e, dist, dev)
     if dist:
-        tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_e2e = float(tt.item())
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
@@ -374,7 +386,7 @@ def run_gpu(args, wl) -> None:
     achieved_tf = F / fwd_mean / 1e12
     sel_mean, abs_mean = statistics.mean(t_sel), statistics.mean(t_abs)
     build_mean = statistics.mean(build_times)
-    value = world * wl.B * wl.Nq / t_step
+    value = job_throughput(world, wl.B, wl.Nq, t_step)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
@@ -402,7 +414,7 @@ def run_gpu(args, wl) -> None:
         },
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
-        "e2e": {"value": world * wl.B * wl.Nq / t_e2e, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": job_throughput(world, wl.B, wl.Nq, t_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": n_e2e,
                 "note": "pinned host Q, K/V window, evicted K/V copied in and O copied out every step"},
     }
