@@ -11,12 +11,12 @@
 // and writes an fp32 partial; reduce_state_kernel adds the partials of a head to S
 // and z in slice order (deterministic).
 //
-// absorb_partial_kernel (192 threads, one CTA per SM):
+// absorb_partial_kernel (320 threads, one CTA per SM):
 //   warp 0      TMA producer: K and V tiles [64 tokens][d] into a 4-stage ring.
 //   warp 1      TMEM owner + MMA issuer: for each tile, D += A_hi x V and D += A_lo x V
 //               with M = 128 (d-index of S, zero-padded for d = 64), N = d, K = 64
 //               tokens; both operands MN-major (d contiguous).
-//   warps 2..5  converters: phi(k) in fp32, split hi = bf16(phi), lo = bf16(phi - hi)
+//   warps 2..9  converters (two warps per SM sub-partition, for latency hiding): phi(k) in fp32, split hi = bf16(phi), lo = bf16(phi - hi)
 //               written at the same swizzled offsets as the K tile (the A operand has
 //               the K tile's layout), z accumulated in fp32 registers. They also drain
 //               the accumulator: the tensor core's fp32 accumulation truncates, so a
@@ -37,7 +37,8 @@ namespace hf {
 constexpr uint32_t kKernAbsorb = 2;
 constexpr int kAbsTok = 64;        // tokens per tile
 constexpr int kAbsStages = 4;      // K/V ring depth
-constexpr int kAbsThreads = 192;
+constexpr int kConvThreads = 256;  // converter warps 2..9
+constexpr int kAbsThreads = 64 + kConvThreads;
 constexpr int kAbsGroup = 2;       // tiles per TMEM accumulation chain
 
 template <int D>
@@ -77,7 +78,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
   __shared__ uint64_t dfull_bar[2], dempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float zred[128][8];
+  __shared__ float zred[kConvThreads][8];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x / p.nsplit;
@@ -93,12 +94,12 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       mbar_init(&empty_bar[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&afull_bar[a], 128);
+      mbar_init(&afull_bar[a], kConvThreads);
       mbar_init(&aempty_bar[a], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&dfull_bar[b], 1);
-      mbar_init(&dempty_bar[b], 128);
+      mbar_init(&dempty_bar[b], kConvThreads);
     }
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -114,7 +115,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
   }
   if (D < 128 && warp >= 2) {
     // the upper 64 rows of the M = 128 A operand are zero padding for d = 64
-    for (int i = threadIdx.x - 64; i < 2 * 2 * C::kChunkBytes / 16; i += 128) {
+    for (int i = threadIdx.x - 64; i < 2 * 2 * C::kChunkBytes / 16; i += kConvThreads) {
       const int a = i / (2 * C::kChunkBytes / 16), rem = i % (2 * C::kChunkBytes / 16);
       const int op = rem / (C::kChunkBytes / 16), u = rem % (C::kChunkBytes / 16);
       reinterpret_cast<uint4*>(abuf + a * C::kABufBytes + op * C::kAOpBytes + C::kChunkBytes)[u] =
@@ -157,6 +158,9 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
+      // descriptors built once; each MMA adds a constant offset to the start address
+      const uint64_t vdesc0 = sdesc_sw128(smem_u32(ring + C::kTileBytes), C::kChunkBytes, 1024);
+      const uint64_t adesc0 = sdesc_sw128(smem_u32(abuf), C::kChunkBytes, 1024);
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
         const int s = i % kAbsStages, a = i & 1;
@@ -169,17 +173,15 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
           ok = mbar_wait(&dempty_bar[b], ((g >> 1) - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 9);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(ring + s * C::kStageBytes + C::kTileBytes);
-        const uint32_t a_addr = smem_u32(abuf + a * C::kABufBytes);
+        const uint64_t bd = vdesc0 + static_cast<uint64_t>((s * C::kStageBytes) >> 4);
+        const uint64_t ad = adesc0 + static_cast<uint64_t>((a * C::kABufBytes) >> 4);
         const uint32_t d_tmem = tmem_d + b * 128;
 #pragma unroll
         for (int op = 0; op < 2; ++op) {
 #pragma unroll
-          for (int ks = 0; ks < kAbsTok / 16; ++ks) {
-            const uint64_t adesc = sdesc_sw128(a_addr + op * C::kAOpBytes + ks * 2048, C::kChunkBytes, 1024);
-            const uint64_t bdesc = sdesc_sw128(v_addr + ks * 2048, C::kChunkBytes, 1024);
-            umma_ss(d_tmem, adesc, bdesc, idesc, (!first || op > 0 || ks > 0) ? 1u : 0u);
-          }
+          for (int ks = 0; ks < kAbsTok / 16; ++ks)
+            umma_ss(d_tmem, ad + ((op * C::kAOpBytes) >> 4) + ks * 128, bd + ks * 128, idesc,
+                    (!first || op > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&empty_bar[s]);
         umma_commit(&aempty_bar[a]);
@@ -189,22 +191,25 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       mbar_wait_drain(&drain_bar, 0, p.timeout_ns, (kKernAbsorb << 8) | 5);
     }
   } else {
-    // ---------------- converters + epilogue (128 threads) ----------------
-    const int t = threadIdx.x - 64;  // 0..127
+    // ---------------- converters + epilogue (256 threads) ----------------
+    const int t = threadIdx.x - 64;  // 0..255
     constexpr int kUnits = D / 8;    // 16-byte units per row
-    constexpr int kPhases = 128 / kUnits;
+    constexpr int kPhases = kConvThreads / kUnits;
+    constexpr int kRowsPerThread = kAbsTok / kPhases;
     const int ucol = t % kUnits;     // logical unit column: elements [8*ucol, 8*ucol + 8)
     const int phase = t / kUnits;    // rows phase, phase + kPhases, ...
     const int chunk = ucol / 8;
     const uint32_t swz = static_cast<uint32_t>(((ucol % 8) ^ (phase & 7)) * 16);
-    float zacc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    // register accumulator of this thread's row m of phi(K)^T V (TMEM lane m)
+    uint64_t zacc[4] = {0ull, 0ull, 0ull, 0ull};  // fp32 pairs: elements (2e, 2e+1) of the unit
+    // register accumulator: row m of phi(K)^T V (TMEM lane m), columns [col0, col0 + D/2);
+    // the two warps that share a TMEM lane quarter take one half of the columns each
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
+    const int col0 = (warp >= 6) ? D / 2 : 0;
     const uint32_t lane_base = tmem_d + (static_cast<uint32_t>(quarter * 32) << 16);
-    float acc[D];
+    float acc[D / 2];
 #pragma unroll
-    for (int c = 0; c < D; ++c) acc[c] = 0.f;
+    for (int c = 0; c < D / 2; ++c) acc[c] = 0.f;
     const int ngroups = (ntiles + kAbsGroup - 1) / kAbsGroup;
     int flushed = 0;
     bool ok = true;
@@ -216,9 +221,9 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
         return false;
       tc_fence_after();
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {
         uint32_t r[32];
-        tmem_ld32(lane_base + b * 128 + c0, r);
+        tmem_ld32(lane_base + b * 128 + col0 + c0, r);
         tmem_wait_ld();
         reg_fence<32>(r);
 #pragma unroll
@@ -227,6 +232,25 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       tc_fence_before();
       mbar_arrive(&dempty_bar[b]);
       return true;
+    };
+    // phi(x) = x + 1 (x > 0) or exp(x) (x <= 0) for the two bf16 halves of w, in fp32;
+    // hi = bf16(phi), lo = bf16(phi - hi); z accumulates phi.
+    auto convert_pair = [&](uint32_t w, uint64_t& z2, uint32_t& hi, uint32_t& lo) {
+      const float x0 = bf16_lo_to_f32(w), x1 = bf16_hi_to_f32(w);
+      const uint64_t xl = ffma2(f32x2(x0, x1), f32x2(1.4426950408889634f, 1.4426950408889634f), 0ull);
+      float l0, l1;
+      f32x2_split(xl, l0, l1);
+      const float e0 = ex2_approx(l0), e1 = ex2_approx(l1);
+      float a0, a1;
+      f32x2_split(fadd2(f32x2(x0, x1), f32x2(1.0f, 1.0f)), a0, a1);
+      const float p0 = x0 > 0.f ? a0 : e0;
+      const float p1 = x1 > 0.f ? a1 : e1;
+      const uint64_t pp = f32x2(p0, p1);
+      z2 = fadd2(z2, pp);
+      hi = pack_bf16x2(p0, p1);
+      float r0, r1;
+      f32x2_split(ffma2(f32x2(bf16_lo_to_f32(hi), bf16_hi_to_f32(hi)), f32x2(-1.0f, -1.0f), pp), r0, r1);
+      lo = pack_bf16x2(r0, r1);
     };
     for (int i = 0; i < ntiles && ok; ++i) {
       const int s = i % kAbsStages, a = i & 1;
@@ -239,24 +263,21 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       uint8_t* ahi = abuf + a * C::kABufBytes;
       uint8_t* alo = ahi + C::kAOpBytes;
       const int valid = min(kAbsTok, p.n_tokens - (tile0 + i) * kAbsTok);
-#pragma unroll 2
-      for (int row = phase; row < kAbsTok; row += kPhases) {
+#pragma unroll
+      for (int k = 0; k < kRowsPerThread; ++k) {
+        const int row = phase + k * kPhases;
         const uint32_t off = chunk * C::kChunkBytes + row * 128 + swz;
         const uint4 kv = *reinterpret_cast<const uint4*>(ktile + off);
-        const uint32_t w[4] = {kv.x, kv.y, kv.z, kv.w};
         uint32_t hi[4], lo[4];
-        const bool live = row < valid;
+        if (valid == kAbsTok || row < valid) {
+          convert_pair(kv.x, zacc[0], hi[0], lo[0]);
+          convert_pair(kv.y, zacc[1], hi[1], lo[1]);
+          convert_pair(kv.z, zacc[2], hi[2], lo[2]);
+          convert_pair(kv.w, zacc[3], hi[3], lo[3]);
+        } else {
+          // rows past the end of the tokens (zero-filled by TMA): phi forced to 0
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float x0 = bf16_lo_to_f32(w[e]), x1 = bf16_hi_to_f32(w[e]);
-          float p0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
-          float p1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
-          if (!live) p0 = p1 = 0.f;
-          zacc[2 * e] += p0;
-          zacc[2 * e + 1] += p1;
-          const uint32_t h = pack_bf16x2(p0, p1);
-          hi[e] = h;
-          lo[e] = pack_bf16x2(p0 - bf16_lo_to_f32(h), p1 - bf16_hi_to_f32(h));
+          for (int e = 0; e < 4; ++e) hi[e] = lo[e] = 0u;
         }
         *reinterpret_cast<uint4*>(ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
@@ -277,19 +298,20 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     }
     // z partial: reduce the kPhases row phases of each unit column
 #pragma unroll
-    for (int k = 0; k < 8; ++k) zred[t][k] = zacc[k];
-    named_bar_sync(1, 128);
+    for (int e = 0; e < 4; ++e) f32x2_split(zacc[e], zred[t][2 * e], zred[t][2 * e + 1]);
+    named_bar_sync(1, kConvThreads);
     if (t < D) {
       const int uc = t / 8, e = t % 8;
       float zs = 0.f;
       for (int ph = 0; ph < kPhases; ++ph) zs += zred[ph * kUnits + uc][e];
       p.part_z[(static_cast<size_t>(bh) * p.nsplit + split) * D + t] = zs;
     }
-    // S partial: row m of this slice's phi(K)^T V
+    // S partial: row m, columns [col0, col0 + D/2) of this slice's phi(K)^T V
     if (ok && m < D) {
-      float* dst = p.part_S + ((static_cast<size_t>(bh) * p.nsplit + split) * D + m) * D;
+      float* dst = p.part_S + ((static_cast<size_t>(bh) * p.nsplit + split) * D + m) * D + col0;
 #pragma unroll
-      for (int j = 0; j < D; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+      for (int j = 0; j < D / 2; j += 4)
+        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
     }
   }
 

@@ -8,25 +8,28 @@
 // section 2 A.
 //
 // One CTA per (b, h, query block I); the 128-row query tile holds block I's rows (for
-// block < 128 the remaining rows are computed but never stored). 192 threads:
-//   warp 0      TMA producer: Q tile once, then K/V of each kept block J into a ring
-//               of kStages stages (row coordinate J*block; rows past Nk are zero-filled).
+// block < 128 the remaining rows are computed but never stored). 224 threads:
+//   warp 0      TMA producer of the Q tile (once) and of the K tile of each kept block J
+//               into a ring of kStages K slots (row coordinate J*block; rows past Nk are
+//               zero-filled); a K slot frees as soon as its QK^T is done.
+//   warp 6      TMA producer of the V tiles into a ring of kStages V slots; a V slot
+//               frees when its PV is done. Separate warps keep the two rings independent.
 //   warp 1      TMEM owner (512 columns) + single-thread tcgen05 MMA issuer.
-//   warps 2..5  128 "row" threads, thread <-> query row <-> TMEM lane: prologue
-//               (phi(q) split into bf16 hi/lo written to TMEM, the state S converted to
-//               bf16 hi/lo in shared memory, denominator phi(q).z + 1e-6 in fp32),
-//               online softmax per block, epilogue (sum of both terms, bf16, TMA store).
-// TMEM columns: [0,128) S buffer 0 (phi hi/lo during the prologue), [128,256) S
-// buffer 1, [256,256+d) O accumulator, [384,384+d) linear term.
-// Pipeline per kept block j: S_{j+1} = Q K_{j+1}^T is issued before O += P_j V_j so the
-// tensor core works on the next scores while the row threads run the softmax of j. P_j
-// is written as bf16 over the columns of S_j and read by the MMA straight from TMEM.
-// Softmax is online in the log2 domain with a lazily raised running max: O is rescaled
-// only when the block maximum exceeds the running max by more than 8 (a factor 256),
-// which keeps exp2 arguments <= 8 and is exact since numerator and denominator share it.
-// The linear term runs first: D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi (two-term
-// bf16 splits of phi(q) and S, fp32 accumulation); its S_hi/S_lo operands occupy the
-// first ring stages, which the producer fills only after those MMAs completed.
+//   warps 2..5  128 "row" threads, thread <-> query row <-> TMEM lane: online softmax
+//               per kept block, then the linear readout's operands and the epilogue.
+// TMEM columns: three S buffers [0,128) [128,256) [256,384) and the O accumulator
+// [384, 384+d). S_j = Q K_j^T goes to buffer j % 3; P_j (bf16) is written over S_j's
+// columns and O += P_j V_j reads it straight from TMEM. With three buffers the MMA
+// issuer keeps S two blocks ahead of the softmax: S_{j+3} is issued right after PV_j, so
+// the softmax of block j+1 never waits for the tensor core to finish PV_j first.
+// Softmax: online in the log2 domain with a lazily raised running max (O is rescaled only
+// when a block maximum exceeds the running max by more than 8, i.e. a factor 256; exact
+// since numerator and denominator share the max); the rescale is warp-uniform because
+// TMEM access is warp-collective; 3 exp2 pairs in 8 run on the FMA pipe.
+// Linear term, after the last block: phi(q) in fp32 split into bf16 hi + lo (TMEM, S
+// buffer 1), the state S split into bf16 hi + lo (shared memory, in the now idle ring),
+// D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi on the tensor cores (TMEM, S buffer
+// 0), denominator phi(q).z + 1e-6 in fp32; the epilogue writes O_s / l + D_lin / den.
 #pragma once
 
 #include "hf_ptx.cuh"
@@ -34,8 +37,10 @@
 namespace hf {
 
 constexpr uint32_t kKernAttn = 3;
-constexpr int kAttnThreads = 192;
+constexpr int kAttnThreads = 224;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
+constexpr int kPolyOf8 = 3;         // pairs (of every 8) that take exp2 on the FMA pipe
+constexpr int kSBufs = 3;           // S buffers in TMEM
 
 template <int D, int BLK>
 struct AttnCfg {
@@ -46,11 +51,12 @@ struct AttnCfg {
   static constexpr int kReadoutBytes = 2 * D * D * 2;  // S_hi + S_lo (bf16, d x d each)
   static constexpr int kStagesFit = (kSmemLimit - 2048 - 1024 - kQBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit < 4 ? kStagesFit : 4;
-  static constexpr int kReadoutStages = (kReadoutBytes + kStageBytes - 1) / kStageBytes;
   static_assert(kStages >= 2, "ring too small");
-  static_assert(kReadoutStages <= kStages, "readout operands must fit in the ring");
+  static_assert(kReadoutBytes <= kStages * kStageBytes, "readout operands must fit in the K and V rings");
   static constexpr int kDynSmem = 1024 + kQBytes + kStages * kStageBytes;
-  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColLin = 384;
+  static constexpr uint32_t kColO = 384;
+  static constexpr uint32_t kColLin = 0;    // linear term (after the last block)
+  static constexpr uint32_t kColPhi = 128;  // phi(q) hi | lo (after the last block)
 };
 
 struct AttnParams {
@@ -71,16 +77,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                        AttnParams p) {
   using C = AttnCfg<D, BLK>;
   constexpr int NS = C::kStages;
-  constexpr int KR = C::kReadoutStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                  // Q tile; reused as the output staging tile
-  uint8_t* ring = smem + C::kQBytes;   // NS stages of [K tile | V tile]; S_hi/S_lo first
+  uint8_t* kring = smem + C::kQBytes;             // NS K slots
+  uint8_t* vring = kring + NS * C::kKVTileBytes;  // NS V slots (S_hi/S_lo over both rings at the end)
 
-  __shared__ uint64_t q_bar, full_bar[NS], empty_bar[NS];
-  __shared__ uint64_t pro_bar, sfull_bar[2], pfull_bar[2], odone_bar, lin_bar, final_bar, drain_bar;
+  __shared__ uint64_t q_bar, kfull_bar[NS], kempty_bar[NS], vfull_bar[NS], vempty_bar[NS];
+  __shared__ uint64_t sfull_bar[kSBufs], pfull_bar[kSBufs], odone_bar[2];
+  __shared__ uint64_t final_bar, pro_bar, lin_bar, drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
+  __shared__ float z_sh[D];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x / p.nQB;
@@ -91,17 +99,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&q_bar, 1);
     for (int s = 0; s < NS; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], 1);
+      mbar_init(&kfull_bar[s], 1);
+      mbar_init(&kempty_bar[s], 1);
+      mbar_init(&vfull_bar[s], 1);
+      mbar_init(&vempty_bar[s], 1);
     }
-    mbar_init(&pro_bar, 128);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSBufs; ++b) {
       mbar_init(&sfull_bar[b], 1);
       mbar_init(&pfull_bar[b], 128);
     }
-    mbar_init(&odone_bar, 1);
-    mbar_init(&lin_bar, 1);
+    mbar_init(&odone_bar[0], 1);
+    mbar_init(&odone_bar[1], 1);
     mbar_init(&final_bar, 1);
+    mbar_init(&pro_bar, 128);
+    mbar_init(&lin_bar, 1);
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
     fence_mbar_init();
@@ -116,18 +127,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
+  for (int i = threadIdx.x; i < D; i += kAttnThreads) z_sh[i] = p.z[static_cast<size_t>(bh) * D + i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
-  if (warp == 0) {
-    // ============================ TMA producer ============================
+  if (warp == 0 || warp == 6) {
+    // ============================ TMA producers ============================
     if (lane == 0) {
-      mbar_arrive_expect_tx(&q_bar, C::kQBytes);
+      const bool is_k = warp == 0;  // warp 0: Q + K tiles, warp 6: V tiles
+      const CUtensorMap* map = is_k ? &mapK : &mapV;
+      uint64_t* full = is_k ? kfull_bar : vfull_bar;
+      uint64_t* empty = is_k ? kempty_bar : vempty_bar;
+      uint8_t* slots = is_k ? kring : vring;
+      if (is_k) {
+        mbar_arrive_expect_tx(&q_bar, C::kQBytes);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) tma_load_3d(sQ + c * 128 * 128, &mapQ, &q_bar, c * 64, I * BLK, bh);
-      int v = KR;  // virtual block index: the readout used virtual blocks [0, KR)
+        for (int c = 0; c < C::kChunks; ++c) tma_load_3d(sQ + c * 128 * 128, &mapQ, &q_bar, c * 64, I * BLK, bh);
+      }
+      int v = 0;  // kept-block counter (valid indices only)
       bool bad = false;
       for (int jj = 0; jj < p.r; ++jj) {
         const int J = __ldg(idx_row + jj);
@@ -136,25 +155,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           continue;
         }
         const int s = v % NS, u = v / NS;
-        if (u >= 1 && !mbar_wait(&empty_bar[s], (u - 1) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 1))
-          break;
+        if (u >= 1 && !mbar_wait(&empty[s], (u - 1) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 1)) break;
         if (*abort_flag) break;
-        uint8_t* st = ring + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
+        uint8_t* dst = slots + s * C::kKVTileBytes;
+        mbar_arrive_expect_tx(&full[s], C::kKVTileBytes);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
-          tma_load_3d(st + c * BLK * 128, &mapK, &full_bar[s], c * 64, J * BLK, bh);
-          tma_load_3d(st + C::kKVTileBytes + c * BLK * 128, &mapV, &full_bar[s], c * 64, J * BLK, bh);
-        }
+        for (int c = 0; c < C::kChunks; ++c) tma_load_3d(dst + c * BLK * 128, map, &full[s], c * 64, J * BLK, bh);
         ++v;
       }
-      if (bad) atomicCAS(&g_hf_error_word, 0u, (0x7200u << 16) | (kKernAttn << 8));
-      // drain: the last NS fills (and the Q tile) must have landed before exit
-      mbar_wait_drain(&q_bar, 0, p.timeout_ns, (kKernAttn << 8) | 2);
-      for (int vv = max(KR, v - NS); vv < v; ++vv) {
-        const int s = vv % NS, u = vv / NS;
-        mbar_wait_drain(&full_bar[s], (u - (s < KR ? 1 : 0)) & 1, p.timeout_ns, (kKernAttn << 8) | 3);
-      }
+      if (bad && is_k) atomicCAS(&g_hf_error_word, 0u, (0x7200u << 16) | (kKernAttn << 8));
+      // drain: the Q tile and the last NS fills must have landed before exit
+      if (is_k) mbar_wait_drain(&q_bar, 0, p.timeout_ns, (kKernAttn << 8) | 2);
+      for (int vv = max(0, v - NS); vv < v; ++vv)
+        mbar_wait_drain(&full[vv % NS], (vv / NS) & 1, p.timeout_ns, (kKernAttn << 8) | 3);
     }
   } else if (warp == 1) {
     // ============================ MMA issuer ============================
@@ -167,86 +180,200 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int J = __ldg(idx_row + jj);
         n += (J >= 0 && J < p.nKB);
       }
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t ring_addr = smem_u32(ring);
-      bool ok = mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 4) &&
-                mbar_wait(&pro_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 5);
-      if (ok) {
-        tc_fence_after();
-        // linear term: D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi
-        const uint32_t s_hi = ring_addr, s_lo = ring_addr + D * D * 2;
-        int step = 0;
-#pragma unroll
-        for (int term = 0; term < 3; ++term) {
-          const uint32_t a_col = (term == 2) ? D / 2 : 0;
-          const uint32_t b_base = (term == 1) ? s_lo : s_hi;
-#pragma unroll
-          for (int ks = 0; ks < D / 16; ++ks, ++step) {
-            const uint64_t bdesc = sdesc_sw128(b_base + ks * 2048, D * 128, 1024);
-            umma_ts(tmem + C::kColLin, tmem + C::kColS0 + a_col + ks * 8, bdesc, idesc_lin, step > 0 ? 1u : 0u);
-          }
-        }
-#pragma unroll
-        for (int s = 0; s < KR; ++s) umma_commit(&empty_bar[s]);
-        umma_commit(&lin_bar);
-      }
-      auto stage_of = [&](int j, int& s, uint32_t& par) {
-        const int vv = j + KR;
-        s = vv % NS;
-        par = static_cast<uint32_t>((vv / NS) - (s < KR ? 1 : 0)) & 1u;
-      };
+      // Descriptors are built once; an MMA only adds a constant offset (in 16-byte units)
+      // to the 14-bit start-address field (shared-memory addresses stay below 256 KB, so the
+      // field never carries). This keeps the single issuing thread far ahead of the tensor core.
+      const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t kdesc = sdesc_sw128(smem_u32(kring), 16, 1024);
+      const uint64_t vdesc = sdesc_sw128(smem_u32(vring), BLK * 128, 1024);
+      const uint32_t kring_addr = smem_u32(kring);
       auto issue_qk = [&](int j) {
-        int s;
-        uint32_t par;
-        stage_of(j, s, par);
-        if (!mbar_wait(&full_bar[s], par, abort_flag, p.timeout_ns, (kKernAttn << 8) | 6)) return false;
+        const int s = j % NS;
+        if (!mbar_wait(&kfull_bar[s], (j / NS) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 6)) return false;
         tc_fence_after();
-        const uint32_t k_addr = ring_addr + s * C::kStageBytes;
-        const uint32_t d_col = (j & 1) ? C::kColS1 : C::kColS0;
+        const uint64_t kd = kdesc + static_cast<uint64_t>((s * C::kKVTileBytes) >> 4);
+        const uint32_t d_tmem = tmem + (j % kSBufs) * 128;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t koff = (ks / 4) * (128 * 128) + (ks % 4) * 32;
-          const uint32_t boff = (ks / 4) * (BLK * 128) + (ks % 4) * 32;
-          umma_ss(tmem + d_col, sdesc_sw128(q_addr + koff, 16, 1024), sdesc_sw128(k_addr + boff, 16, 1024),
+          constexpr int kQChunk = (128 * 128) >> 4, kKChunk = (BLK * 128) >> 4;
+          umma_ss(d_tmem, qdesc + (ks / 4) * kQChunk + (ks % 4) * 2, kd + (ks / 4) * kKChunk + (ks % 4) * 2,
                   idesc_qk, ks > 0 ? 1u : 0u);
         }
-        if (!(p.inject && j == 0)) umma_commit(&sfull_bar[j & 1]);
+        umma_commit(&kempty_bar[s]);
+        if (!(p.inject && j == 0)) umma_commit(&sfull_bar[j % kSBufs]);
         return true;
       };
-      if (ok && n > 0) ok = issue_qk(0);
+      bool ok = mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 4);
+      for (int j = 0; j < kSBufs && j < n && ok; ++j) ok = issue_qk(j);
       for (int j = 0; j < n && ok; ++j) {
-        if (j + 1 < n && !(ok = issue_qk(j + 1))) break;
-        if (!(ok = mbar_wait(&pfull_bar[j & 1], (j >> 1) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 7)))
+        const int s = j % NS;
+        if (!(ok = mbar_wait(&pfull_bar[j % kSBufs], (j / kSBufs) & 1, abort_flag, p.timeout_ns,
+                             (kKernAttn << 8) | 7) &&
+                   mbar_wait(&vfull_bar[s], (j / NS) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 14)))
           break;
         tc_fence_after();
-        int s;
-        uint32_t par;
-        stage_of(j, s, par);
-        const uint32_t v_addr = ring_addr + s * C::kStageBytes + C::kKVTileBytes;
-        const uint32_t p_col = (j & 1) ? C::kColS1 : C::kColS0;
+        const uint64_t vd = vdesc + static_cast<uint64_t>((s * C::kKVTileBytes) >> 4);
+        const uint32_t p_tmem = tmem + (j % kSBufs) * 128;
 #pragma unroll
-        for (int ks = 0; ks < BLK / 16; ++ks) {
-          umma_ts(tmem + C::kColO, tmem + p_col + ks * 8, sdesc_sw128(v_addr + ks * 2048, BLK * 128, 1024),
-                  idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-        }
-        umma_commit(&empty_bar[s]);
-        umma_commit(&odone_bar);
+        for (int ks = 0; ks < BLK / 16; ++ks)
+          umma_ts(tmem + C::kColO, p_tmem + ks * 8, vd + ks * 128, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(&vempty_bar[s]);
+        umma_commit(&odone_bar[j & 1]);
+        // S_{j+3} reuses buffer j % 3: in issue order it follows PV_j, which reads P_j there
+        if (j + kSBufs < n) ok = issue_qk(j + kSBufs);
       }
-      if (ok) umma_commit(&final_bar);
+      if (ok) {
+        umma_commit(&final_bar);
+        // linear term: D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi
+        if ((ok = mbar_wait(&pro_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 5))) {
+          tc_fence_after();
+          const uint64_t sdesc_hi = sdesc_sw128(kring_addr, D * 128, 1024);
+          const uint64_t sdesc_lo = sdesc_hi + ((D * D * 2) >> 4);
+#pragma unroll
+          for (int term = 0; term < 3; ++term) {
+            const uint32_t a_col = C::kColPhi + ((term == 2) ? D / 2 : 0);
+            const uint64_t b = (term == 1) ? sdesc_lo : sdesc_hi;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks)
+              umma_ts(tmem + C::kColLin, tmem + a_col + ks * 8, b + ks * 128, idesc_lin,
+                      (term > 0 || ks > 0) ? 1u : 0u);
+          }
+          umma_commit(&lin_bar);
+        }
+      }
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0, p.timeout_ns, (kKernAttn << 8) | 8);
     }
   } else {
-    // ======================= row threads (softmax, epilogue) =======================
+    // ======================= row threads (softmax, readout, epilogue) =======================
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     // tcgen05.ld/st are warp-collective: every wait that guards one is made warp-uniform
     bool ok = __all_sync(0xffffffffu, mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 9));
+
+    // ---- online softmax over the kept blocks
+    float m_run = -INFINITY, l_run = 0.f;
+    int j = 0;
+    for (int jj = 0; jj < p.r && ok; ++jj) {
+      const int J = __ldg(idx_row + jj);
+      if (J < 0 || J >= p.nKB) continue;
+      const int b = j % kSBufs;
+      ok = __all_sync(0xffffffffu, mbar_wait(&sfull_bar[b], (j / kSBufs) & 1, abort_flag, p.timeout_ns,
+                                             (kKernAttn << 8) | 10));
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t s_addr = lane_addr + b * 128;
+      // S row in two halves: the second half's TMEM load overlaps the first half's max
+      uint32_t sr[BLK];
+      constexpr int kHalf = BLK / 2;
+#pragma unroll
+      for (int c = 0; c < kHalf; c += 32) tmem_ld32(s_addr + c, sr + c);
+      tmem_wait_ld();
+      reg_fence<kHalf>(sr);
+#pragma unroll
+      for (int c = kHalf; c < BLK; c += 32) tmem_ld32(s_addr + c, sr + c);
+      float* s = reinterpret_cast<float*>(sr);
+      const int valid = (J == p.nKB - 1) ? p.last_len : BLK;
+      // row max: 8 independent chains of 3-input max (no long dependency chain)
+      float mc[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mc[k] = fmaxf(s[k], s[k + 8]);
+#pragma unroll
+      for (int c = 16; c < kHalf; c += 16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mc[k] = fmax3(mc[k], s[c + k], s[c + 8 + k]);
+      }
+      tmem_wait_ld();
+      reg_fence<kHalf>(sr + kHalf);
+      if (valid < BLK) {  // partial last key block: padding columns are masked out
+#pragma unroll
+        for (int c = 0; c < BLK; ++c)
+          if (c >= valid) s[c] = -INFINITY;
+        float m0 = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < kHalf; ++c) m0 = fmaxf(m0, s[c]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mc[k] = m0;
+      }
+#pragma unroll
+      for (int c = kHalf; c < BLK; c += 16) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mc[k] = fmax3(mc[k], s[c + k], s[c + 8 + k]);
+      }
+      float mx = fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7]));
+      mx *= p.scale_log2;
+      if (j == 0) {
+        m_run = mx;
+      } else {
+        // A row raises its running max only when the block max exceeds it by more than
+        // 8 (log2 units); the O rescale is done by the whole warp whenever any of its
+        // rows needs it (alpha = 1 for the others). It waits for PV_{j-1}: two alternating
+        // barriers, since with S two blocks ahead PV_{j-2} may still be pending here.
+        const bool need = mx > m_run + 8.0f;
+        if (__any_sync(0xffffffffu, need)) {
+          const float alpha = need ? ex2_approx(m_run - mx) : 1.0f;
+          ok = __all_sync(0xffffffffu, mbar_wait(&odone_bar[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
+                                                 p.timeout_ns, (kKernAttn << 8) | 11));
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + C::kColO + c, o);
+            tmem_wait_ld();
+            reg_fence<32>(o);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(lane_addr + C::kColO + c, o);
+          }
+          if (need) {
+            l_run *= alpha;
+            m_run = mx;
+          }
+        }
+      }
+      // p = 2^(s * scale * log2 e - m): packed fp32 pairs; kPolyOf8 pairs of every 8 run
+      // exp2 on the FMA pipe, the others on MUFU, so neither unit alone sets the pace.
+      const uint64_t sl2 = f32x2(p.scale_log2, p.scale_log2);
+      const uint64_t nm2 = f32x2(-m_run, -m_run);
+      uint64_t lacc[4] = {0ull, 0ull, 0ull, 0ull};
+      uint32_t pk[BLK / 2];
+#pragma unroll
+      for (int c = 0; c < BLK; c += 2) {
+        const uint64_t x2 = ffma2(f32x2(s[c], s[c + 1]), sl2, nm2);
+        float p0, p1;
+        if (((c / 2) & 7) >= 8 - kPolyOf8) {
+          exp2_poly_x2(x2, p0, p1);
+        } else {
+          float x0, x1;
+          f32x2_split(x2, x0, x1);
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+        }
+        lacc[(c / 2) & 3] = fadd2(lacc[(c / 2) & 3], f32x2(p0, p1));
+        pk[c / 2] = pack_bf16x2(p0, p1);
+      }
+      {
+        const uint64_t l2 = fadd2(fadd2(lacc[0], lacc[1]), fadd2(lacc[2], lacc[3]));
+        float la, lb;
+        f32x2_split(l2, la, lb);
+        l_run += la + lb;
+      }
+#pragma unroll
+      for (int c = 0; c < BLK / 2; c += 16) tmem_st16(s_addr + c, pk + c);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&pfull_bar[b]);
+      ++j;
+    }
+
+    // ---- linear term operands (all PV done: the S buffers and both rings are free)
+    ok = ok && mbar_wait(&final_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 12);
+    ok = __all_sync(0xffffffffu, ok);
     float den = 1.0f;
     if (ok) {
-      // ---- prologue: phi(q) hi/lo -> TMEM, den = phi(q).z + 1e-6, S -> bf16 hi/lo in smem
-      const float* zrow = p.z + static_cast<size_t>(bh) * D;
+      tc_fence_after();
       float dacc = 0.f;
 #pragma unroll
       for (int g = 0; g < D / 32; ++g) {  // 32 elements -> 16 packed columns of hi and of lo
@@ -262,24 +389,23 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const float x0 = bf16_lo_to_f32(w[e]), x1 = bf16_hi_to_f32(w[e]);
             const float p0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
             const float p1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
-            const float2 zz = __ldg(reinterpret_cast<const float2*>(zrow + unit * 8 + 2 * e));
-            dacc = fmaf(p0, zz.x, dacc);
-            dacc = fmaf(p1, zz.y, dacc);
+            dacc = fmaf(p0, z_sh[unit * 8 + 2 * e], dacc);
+            dacc = fmaf(p1, z_sh[unit * 8 + 2 * e + 1], dacc);
             const uint32_t hh = pack_bf16x2(p0, p1);
             hi[h * 4 + e] = hh;
             lo[h * 4 + e] = pack_bf16x2(p0 - bf16_lo_to_f32(hh), p1 - bf16_hi_to_f32(hh));
           }
         }
         // TMEM column c holds elements (2c, 2c+1) of the row: hi at [0, D/2), lo at [D/2, D)
-        tmem_st16(lane_addr + C::kColS0 + g * 16, hi);
-        tmem_st16(lane_addr + C::kColS0 + D / 2 + g * 16, lo);
+        tmem_st16(lane_addr + C::kColPhi + g * 16, hi);
+        tmem_st16(lane_addr + C::kColPhi + D / 2 + g * 16, lo);
       }
       den = dacc + 1e-6f;
       // state rows: thread k < D converts S[bh][k][:] into MN-major bf16 hi/lo tiles
       if (row < D) {
         const float* srow = p.S + (static_cast<size_t>(bh) * D + row) * D;
-        uint8_t* s_hi = ring;
-        uint8_t* s_lo = ring + D * D * 2;
+        uint8_t* s_hi = kring;
+        uint8_t* s_lo = kring + D * D * 2;
 #pragma unroll 4
         for (int unit = 0; unit < D / 8; ++unit) {
           const float4 a = __ldg(reinterpret_cast<const float4*>(srow + unit * 8));
@@ -303,84 +429,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_arrive(&pro_bar);
     }
 
-    // ---- online softmax over the kept blocks
-    float m_run = -INFINITY, l_run = 0.f;
-    int j = 0;
-    for (int jj = 0; jj < p.r && ok; ++jj) {
-      const int J = __ldg(idx_row + jj);
-      if (J < 0 || J >= p.nKB) continue;
-      const int b = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sfull_bar[b], (j >> 1) & 1, abort_flag, p.timeout_ns,
-                                             (kKernAttn << 8) | 10));
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t s_addr = lane_addr + (b ? C::kColS1 : C::kColS0);
-      uint32_t sr[BLK];
-#pragma unroll
-      for (int c = 0; c < BLK; c += 32) tmem_ld32(s_addr + c, sr + c);
-      tmem_wait_ld();
-      reg_fence<BLK>(sr);
-      float* s = reinterpret_cast<float*>(sr);
-      const int valid = (J == p.nKB - 1) ? p.last_len : BLK;
-      if (valid < BLK) {
-#pragma unroll
-        for (int c = 0; c < BLK; ++c)
-          if (c >= valid) s[c] = -INFINITY;
-      }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < BLK; ++c) mx = fmaxf(mx, s[c]);
-      mx *= p.scale_log2;
-      if (j == 0) {
-        m_run = mx;
-      } else {
-        // A row raises its running max only when the block max exceeds it by more than
-        // 8 (log2 units); the O rescale is done by the whole warp whenever any of its
-        // rows needs it (alpha = 1 for the others), since TMEM access is warp-collective.
-        const bool need = mx > m_run + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2_approx(m_run - mx) : 1.0f;
-          ok = __all_sync(0xffffffffu, mbar_wait(&odone_bar, (j - 1) & 1, abort_flag, p.timeout_ns,
-                                                 (kKernAttn << 8) | 11));
-          if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + C::kColO + c, o);
-            tmem_wait_ld();
-            reg_fence<32>(o);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(lane_addr + C::kColO + c, o);
-          }
-          if (need) {
-            l_run *= alpha;
-            m_run = mx;
-          }
-        }
-      }
-      float lsum = 0.f;
-      uint32_t pk[BLK / 2];
-#pragma unroll
-      for (int c = 0; c < BLK; c += 2) {
-        const float p0 = ex2_approx(fmaf(s[c], p.scale_log2, -m_run));
-        const float p1 = ex2_approx(fmaf(s[c + 1], p.scale_log2, -m_run));
-        lsum += p0 + p1;
-        pk[c / 2] = pack_bf16x2(p0, p1);
-      }
-      l_run += lsum;
-#pragma unroll
-      for (int c = 0; c < BLK / 2; c += 16) tmem_st16(s_addr + c, pk + c);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&pfull_bar[b]);
-      ++j;
-    }
-
     // ---- epilogue: O = O_s / l + O_lin / den -> bf16 -> TMA store of the block's rows
-    if (ok) ok = mbar_wait(&final_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 12) &&
-                 mbar_wait(&lin_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 13);
+    ok = ok && mbar_wait(&lin_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 13);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
