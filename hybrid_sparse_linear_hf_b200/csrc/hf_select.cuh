@@ -12,11 +12,11 @@
 //   pool_blocks_kernel   one CTA per (b,h,block) of Q or K: fp32 mean of the valid rows.
 //                        HBM-bound: reads Q and K once with 16-byte loads, 8 in flight
 //                        per thread.
-//   score_select_kernel  one CTA per (b,h,I): s_IJ = Qbar_I . Kbar_J by warp-level
-//                        reductions (one warp per J, lanes over d, xor shuffles), then
-//                        rank_J = #{J': s_J' > s_J or (s_J' == s_J and J' < J)}; the
-//                        r blocks with rank < r are written in ascending J. NaN scores
-//                        are ranked as -inf so exactly r blocks are always written.
+//   score_select_kernel  one CTA per (b,h, 4 query blocks): s_IJ = Qbar_I . Kbar_J, a
+//                        thread per key block; then one warp per query block finds its
+//                        top r by a warp-wide bitwise search (ballots) for the r-th
+//                        largest (score, -J) key; the r blocks are written in ascending J.
+//                        NaN scores are ranked as -inf, so exactly r blocks are written.
 #pragma once
 
 #include "hf_ptx.cuh"
@@ -25,7 +25,7 @@ namespace hf {
 
 constexpr int kPoolThreads = 256;
 constexpr int kSelectThreads = 256;
-constexpr int kMaxKeyBlocks = 8192;  // score row + flags fit in shared memory
+constexpr int kMaxKeyBlocks = 8192;  // 4 score rows fit in shared memory; J fits the 13-bit key field
 
 __device__ __forceinline__ void acc_bf16x8(float* acc, uint4 v) {
   acc[0] += bf16_lo_to_f32(v.x);
@@ -102,67 +102,120 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bf
   }
 }
 
+// Scores of kSelQB query blocks of one head per CTA (each pooled K row is read once for
+// all of them), then one warp per query block selects its top r.
+constexpr int kSelQB = 4;
+constexpr int kSelRegKeys = 16;  // keys per lane held in registers (nKB <= 512)
+
+// Order-preserving map of a float to an unsigned integer (NaN has been replaced by -inf).
+__device__ __forceinline__ uint32_t ordered_bits(float f) {
+  const uint32_t b = __float_as_uint(f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Unique selection key of key block J: larger score first, lower index first on ties.
+__device__ __forceinline__ uint64_t select_key(float s, int J) {
+  return (static_cast<uint64_t>(ordered_bits(s)) << 13) | static_cast<uint64_t>(8191 - J);
+}
+
 // idx_out[bh][I][0..r) = top-r key blocks of query block I, ascending.
+// Scores: thread per key block J, s_IJ = Qbar_I . Kbar_J for the CTA's kSelQB query blocks
+// (pooled Q in shared memory, the pooled K row streamed with 16-byte loads, all in flight).
+// Selection: the warp of query block I finds the r-th largest of the unique 45-bit keys
+// (ordered score bits << 13) | (8191 - J) bit by bit (counting keys at or above a
+// candidate with ballots); the blocks at or above it are exactly the top r, written in
+// ascending J with ballot prefix counts.
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const float* __restrict__ Qp,
                                                                       const float* __restrict__ Kp, int nQB,
                                                                       int nKB, int r,
                                                                       int32_t* __restrict__ idx_out,
                                                                       float* __restrict__ scores_out) {
-  extern __shared__ float s_row[];  // [nKB] scores, then [nKB] int flags
-  int* flag = reinterpret_cast<int*>(s_row + nKB);
-  constexpr int kPer = D / 32;  // pooled elements per lane
-  const int bh = blockIdx.x / nQB;
-  const int I = blockIdx.x % nQB;
+  extern __shared__ float s_sc[];  // [kSelQB][nKB] scores
+  __shared__ __align__(16) float q_sh[kSelQB][D];
+  const int groups = (nQB + kSelQB - 1) / kSelQB;
+  const int bh = blockIdx.x / groups;
+  const int I0 = (blockIdx.x % groups) * kSelQB;
+  const int G = min(kSelQB, nQB - I0);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  constexpr int kWarps = kSelectThreads / 32;
 
-  float q[kPer];
-  const float* qrow = Qp + (static_cast<size_t>(bh) * nQB + I) * D + lane * kPer;
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) q[k] = qrow[k];
-
-  const float* kbase = Kp + static_cast<size_t>(bh) * nKB * D + lane * kPer;
-  for (int J = warp; J < nKB; J += kWarps) {
-    const float* krow = kbase + static_cast<size_t>(J) * D;
-    float dot = 0.f;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) dot = fmaf(q[k], krow[k], dot);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-    if (lane == 0) s_row[J] = dot;
+  for (int i = threadIdx.x; i < kSelQB * D; i += kSelectThreads) {
+    const int g = i / D;
+    q_sh[g][i % D] = Qp[(static_cast<size_t>(bh) * nQB + I0 + min(g, G - 1)) * D + i % D];
   }
   __syncthreads();
-
-  float* srow_out = scores_out ? scores_out + (static_cast<size_t>(bh) * nQB + I) * nKB : nullptr;
+  const float* kbase = Kp + static_cast<size_t>(bh) * nKB * D;
   for (int J = threadIdx.x; J < nKB; J += kSelectThreads) {
-    const float v = s_row[J];
-    if (srow_out) srow_out[J] = v;
-  }
-  __syncthreads();
-  // NaN ranks last; the order (score desc, index asc) is then a strict total order.
-  for (int J = threadIdx.x; J < nKB; J += kSelectThreads) {
-    if (s_row[J] != s_row[J]) s_row[J] = -INFINITY;
-  }
-  __syncthreads();
-
-  for (int J = threadIdx.x; J < nKB; J += kSelectThreads) {
-    const float v = s_row[J];
-    int rank = 0;
-    for (int Jp = 0; Jp < nKB; ++Jp) {
-      const float w = s_row[Jp];
-      rank += (w > v) || (w == v && Jp < J);
+    const float4* krow = reinterpret_cast<const float4*>(kbase + static_cast<size_t>(J) * D);
+    float acc[kSelQB];
+#pragma unroll
+    for (int g = 0; g < kSelQB; ++g) acc[g] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < D / 4; k0 += 8) {
+      float4 kv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) kv[u] = __ldg(krow + k0 + u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+#pragma unroll
+        for (int g = 0; g < kSelQB; ++g) {
+          const float4 qv = *reinterpret_cast<const float4*>(&q_sh[g][4 * (k0 + u)]);
+          acc[g] = fmaf(qv.x, kv[u].x, acc[g]);
+          acc[g] = fmaf(qv.y, kv[u].y, acc[g]);
+          acc[g] = fmaf(qv.z, kv[u].z, acc[g]);
+          acc[g] = fmaf(qv.w, kv[u].w, acc[g]);
+        }
+      }
     }
-    flag[J] = rank < r;
+#pragma unroll
+    for (int g = 0; g < kSelQB; ++g) s_sc[g * nKB + J] = acc[g];
   }
   __syncthreads();
 
-  int32_t* out = idx_out + (static_cast<size_t>(bh) * nQB + I) * r;
-  for (int J = threadIdx.x; J < nKB; J += kSelectThreads) {
-    if (!flag[J]) continue;
-    int pos = 0;
-    for (int Jp = 0; Jp < J; ++Jp) pos += flag[Jp];
-    if (pos < r) out[pos] = J;
+  if (warp < G) {
+    const int I = I0 + warp;
+    const float* srow = s_sc + warp * nKB;
+    float* sout = scores_out ? scores_out + (static_cast<size_t>(bh) * nQB + I) * nKB : nullptr;
+    if (sout)
+      for (int J = lane; J < nKB; J += 32) sout[J] = srow[J];
+    auto key_at = [&](int J) -> uint64_t {
+      const float v = srow[J];
+      return select_key(v != v ? -INFINITY : v, J);  // NaN ranks last
+    };
+    // largest T with #{keys >= T} >= r: the r-th largest key (keys are unique)
+    uint64_t T = 0;
+    if (nKB <= 32 * kSelRegKeys) {
+      uint64_t keys[kSelRegKeys];
+#pragma unroll
+      for (int k = 0; k < kSelRegKeys; ++k) keys[k] = (32 * k + lane < nKB) ? key_at(32 * k + lane) : 0ull;
+      for (int bit = 44; bit >= 0; --bit) {
+        const uint64_t cand = T | (1ull << bit);
+        int cnt = 0;
+#pragma unroll
+        for (int k = 0; k < kSelRegKeys; ++k) cnt += __popc(__ballot_sync(0xffffffffu, keys[k] >= cand));
+        if (cnt >= r) T = cand;
+      }
+    } else {
+      for (int bit = 44; bit >= 0; --bit) {
+        const uint64_t cand = T | (1ull << bit);
+        int cnt = 0;
+        for (int J0 = 0; J0 < nKB; J0 += 32) {
+          const int J = J0 + lane;
+          cnt += __popc(__ballot_sync(0xffffffffu, J < nKB && key_at(J) >= cand));
+        }
+        if (cnt >= r) T = cand;
+      }
+    }
+    int32_t* out = idx_out + (static_cast<size_t>(bh) * nQB + I) * r;
+    int base = 0;
+    for (int J0 = 0; J0 < nKB; J0 += 32) {
+      const int J = J0 + lane;
+      const bool keep = J < nKB && key_at(J) >= T;
+      const uint32_t m = __ballot_sync(0xffffffffu, keep);
+      const int pos = base + __popc(m & ((1u << lane) - 1u));
+      if (keep && pos < r) out[pos] = J;
+      base += __popc(m);
+    }
   }
 }
 
