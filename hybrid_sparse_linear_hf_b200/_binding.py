@@ -52,6 +52,8 @@ _SIGNATURES = {
                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "hf_select_blocks": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 +
                          [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_select_blocks_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 +
+                                 [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "hf_hybrid_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
                            [ctypes.c_void_p, ctypes.POINTER(HfStateC), ctypes.c_float, ctypes.c_void_p,
                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
@@ -185,6 +187,27 @@ def hf_select_blocks(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, idx_o
                                   _dev(scores_out, torch.float32, "scores_out") if scores_out is not None else None,
                                   ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
            "hf_select_blocks")
+    return idx_out
+
+
+# Largest select workspace hf_select_blocks_noalloc serves (HF_SELECT_NOALLOC_SCRATCH_BYTES).
+HF_SELECT_NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def hf_select_blocks_noalloc(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, idx_out: torch.Tensor,
+                             scores_out=None, stream=None) -> torch.Tensor:
+    """``hf_select_blocks`` without a workspace, for hosts that cannot allocate device
+    memory around the step: the library's fixed per-device scratch holds the pooled rows.
+    ``idx_out`` [B,H,nQB,r] int32 is caller-provided, so nothing is allocated here either.
+    The first call on a device does a one-off set-up (make it before any stream capture);
+    calls on one device share the scratch, so calls that overlap in time race."""
+    B, H, Nq, d = Q.shape
+    Nk = K.shape[2]
+    _check(lib().hf_select_blocks_noalloc(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), B, H, Nq,
+                                          Nk, d, block, r, _dev(idx_out, torch.int32, "idx_out"),
+                                          _dev(scores_out, torch.float32, "scores_out")
+                                          if scores_out is not None else None, _stream(stream)),
+           "hf_select_blocks_noalloc")
     return idx_out
 
 

@@ -213,6 +213,36 @@ __global__ void debug_exp2_kernel(const float* __restrict__ x, float* __restrict
 
 }  // namespace
 
+// ---------------------------------------------------------------- select without a caller workspace
+// Scratch of hf_select_blocks_noalloc: the pooled Q and K rows of one call, in place of
+// the caller's workspace. One copy per device (a module-scope __device__ array), so the
+// call needs no allocation; its address on a device is looked up once, with that device
+// current, and cached.
+static __device__ __align__(256) unsigned char g_select_scratch[HF_SELECT_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kScratchMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kScratchMaxDevices] = {};
+
+// Device address of g_select_scratch on the current device (set-up on first use).
+hf_status select_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return HF_ERR_CUDA;
+  if (dev < 0 || dev >= kScratchMaxDevices) return HF_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || !p) return HF_ERR_CUDA;
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return HF_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 HF_API const char* hf_version(void) { return "hf-b200 0.1.0 (sm_100a)"; }
@@ -366,6 +396,24 @@ HF_API hf_status hf_debug_inject_timeout(int kernel_id, int count, unsigned long
   g_inject.count = count;
   g_inject.timeout_ns = timeout_ns ? timeout_ns : kDefaultTimeoutNs;
   return HF_OK;
+}
+
+HF_API hf_status hf_select_blocks_noalloc(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk,
+                                          int d, int block, int r, int32_t* idx_out, float* scores_out,
+                                          void* stream) {
+  // The same argument checks as hf_select_blocks, so that a rejected call never reaches
+  // the set-up; then the size check against the fixed scratch.
+  if (B < 1 || H < 1 || Nq < 0 || Nk < 1) return HF_ERR_INVALID_ARG;
+  if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
+  if (r < 1 || r > ceil_div(Nk, block)) return HF_ERR_INVALID_ARG;
+  if (Nq == 0) return HF_OK;
+  const size_t need = select_ws_bytes(B, H, Nq, Nk, d, block);
+  if (need > HF_SELECT_NOALLOC_SCRATCH_BYTES) return HF_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const hf_status rc = select_scratch(&scratch);
+  if (rc != HF_OK) return rc;
+  return hf_select_blocks(Q, K, B, H, Nq, Nk, d, block, r, idx_out, scores_out, scratch,
+                          HF_SELECT_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

@@ -34,7 +34,8 @@
  *   - Supported: d in {64, 128}; block in {32, 64, 128}; 1 <= r <= nKB.
  *   - The caller owns every buffer, including workspaces (size from
  *     hf_workspace_size). The library allocates no device memory. Its only state is
- *     one 32-bit device error word per GPU, read by hf_query_status.
+ *     one 32-bit device error word per GPU, read by hf_query_status, and the fixed
+ *     scratch array of hf_select_blocks_noalloc.
  *   - All calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *     stream). Argument errors are returned before anything is launched; a failed
  *     launch returns HF_ERR_CUDA. A kernel that gives up on an internal wait (bounded,
@@ -126,6 +127,39 @@ HF_API hf_status hf_absorb_evicted(hf_state* st, const hf_bf16* K_ev, const hf_b
 HF_API hf_status hf_select_blocks(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk, int d,
                                   int block, int r, int32_t* idx_out, float* scores_out, void* ws,
                                   size_t ws_bytes, void* stream);
+
+/* Upper bound, in bytes, of the select workspace that hf_select_blocks_noalloc can
+ * serve: a call is accepted when hf_workspace_size(HF_WS_SELECT, ...) for its shapes
+ * is at most this (e.g. 12 heads x 4680 query x 32760 key tokens at d = 128, block
+ * 128 need 1.7 MiB; 40 heads x 10800 x 43200 need 8.3 MiB). */
+#define HF_SELECT_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/* hf_select_blocks for callers that cannot hand the library any device memory of
+ * their own: same arguments, results and errors, minus the workspace. The paper has
+ * no counterpart of this call; it exists for hosts that must not call cudaMalloc or
+ * an allocating library around the step (an allocation may synchronise the device or
+ * fail in the middle of a stream), or whose memory is owned by an allocator they
+ * cannot reach. Instead of a workspace it uses a fixed scratch array that the library
+ * holds in device memory, HF_SELECT_NOALLOC_SCRATCH_BYTES per device (present on
+ * every device the library's kernels are loaded on, whether this call is used or not).
+ *   - Shapes whose select workspace exceeds HF_SELECT_NOALLOC_SCRATCH_BYTES return
+ *     HF_ERR_WORKSPACE before anything runs; use hf_select_blocks for those.
+ *   - The first call on a device (that device current) does a one-off set-up: it looks
+ *     up the scratch's device address, which may load the library's kernels on that
+ *     device. Make that first call before any stream capture begins. A failed set-up
+ *     returns HF_ERR_CUDA and is retried by the next call.
+ *   - Nothing in the scratch needs to start at zero: every byte a call reads was
+ *     written earlier in that same call.
+ *   - All calls on one device share the one scratch. Two calls whose kernels overlap
+ *     in time (different streams, or different host threads, without ordering between
+ *     them) race on it and may return wrong blocks; calls on one stream are ordered
+ *     and safe.
+ *   - Device indices >= 64 return HF_ERR_UNSUPPORTED.
+ * Errors: those of hf_select_blocks, with HF_ERR_WORKSPACE meaning "too large for the
+ * fixed scratch". */
+HF_API hf_status hf_select_blocks_noalloc(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk,
+                                          int d, int block, int r, int32_t* idx_out, float* scores_out,
+                                          void* stream);
 
 /* Hybrid attention output for the query chunk:
  *   O[b][h][i] = sum_{j in kept(I(i))} softmax_j(scale * q_i . k_j) v_j
