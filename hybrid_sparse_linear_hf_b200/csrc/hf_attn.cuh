@@ -8,37 +8,35 @@
 // section 2 A.
 //
 // One CTA per (b, h, query block I); the 128-row query tile holds block I's rows (for
-// block < 128 the remaining rows are computed but never stored). 384 threads, three
-// warpgroups; setmaxnreg moves registers from the first to the other two:
+// block < 128 the remaining rows are computed but never stored). The kept blocks are
+// dealt alternately to two softmax pipelines A and B (positions 0, 2, 4, ... and
+// 1, 3, 5, ...), each with its own S buffer, O accumulator and running max / sum; the
+// two partial results merge after the last block, as two online-softmax states do. While
+// one pipeline exponentiates, the tensor cores run the other's MMAs, so the softmax of
+// a block only has to fit within the MMAs of two blocks.
+// 384 threads, three warpgroups; setmaxnreg moves registers from the first to the others:
 //   warp 0      TMA producer of the Q tile (once) and of the K tile of each kept block J
 //               into a ring of K slots (row coordinate J*block; rows past Nk are
 //               zero-filled); a K slot frees as soon as its QK^T is done.
 //   warp 1      TMEM owner (512 columns) + single-thread tcgen05 MMA issuer.
 //   warp 2      TMA producer of the V tiles into a ring of V slots. (warp 3 idles)
-//   warps 4..11 row threads: warps w and w+4 share TMEM lane quarter w % 4 (query rows
-//               32*(w%4) .. +31); warps 4..7 exponentiate the first half of every row's
-//               columns, warps 8..11 the second half: two softmax warps per sub-partition.
-// TMEM columns: S buffers [0,128) and [128,256), O [256, 256+d), Q [384, 384+d/2)
-// (bf16 pairs), P [448, 448+block/2) (bf16 pairs).
-// Shared-memory traffic is the binding resource at d = block = 128 (one SMEM operand of
-// 128x128x16 per 64 tensor cycles is already 128 B/clk): Q therefore lives in TMEM
-// (S = Q K^T reads only K from shared memory) and P too (O += P V reads only V).
-// Pipeline per kept block j: S_j -> buffer j%2; the row threads load S_j into registers
-// and release the buffer at once, so S_{j+2} is computed during softmax j; P_j goes to
-// the P region once PV_{j-1} has read P_{j-1}; PV_j follows P_j.
+//   warps 4..7  pipeline A, warps 8..11 pipeline B: one thread per query row (TMEM lane
+//               quarter = warp % 4), the whole row of S per thread.
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+d), O_B [384,384+d). P (bf16
+// pairs) overwrites the first block/2 columns of its S buffer once S is in registers.
+// MMA order: S_A0 S_B0 | PV_A0 S_A1 | PV_B0 S_B1 | PV_A1 S_A2 | ...; the commit after
+// S_p(i+1) also covers PV_p(i), so a softmax thread that sees S_p(i+1) knows O_p is
+// stable (its lazy rescale needs no other wait).
 // Softmax: online in the log2 domain with a lazily raised running max (O is rescaled only
 // when a block maximum exceeds the running max by more than 8, i.e. a factor 256; exact
-// since numerator and denominator share the max); both warps of a quarter read the whole
-// S row and take the same full-row max (no exchange, so they never wait on each other),
-// each exponentiating its half; the O rescale is warp-uniform because TMEM access is
-// warp-collective; 3 exp2 pairs in 8 run on the FMA pipe, the rest on MUFU.
-// Linear term, after the last block: phi(q) in fp32 split into bf16 hi + lo (TMEM, S
-// buffer 1), the state S split into bf16 hi + lo (shared memory, over the idle rings),
-// D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi on the tensor cores (TMEM, S buffer
-// 0), denominator phi(q).z + 1e-6 in fp32; the epilogue writes O_s / l + D_lin / den.
+// since numerator and denominator share the max); the O rescale is warp-uniform because
+// TMEM access is warp-collective; 3 exp2 pairs in 8 run on the FMA pipe, the rest on MUFU.
+// Linear term, after the last block: phi(q) in fp32 split into bf16 hi + lo (TMEM, over
+// S_B), the state S split into bf16 hi + lo (shared memory, over the idle rings),
+// D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi on the tensor cores (TMEM, over S_A),
+// denominator phi(q).z + 1e-6 in fp32; the epilogue writes
+// (w_A O_A + w_B O_B) / (w_A l_A + w_B l_B) + D_lin / den, w_p = 2^(m_p - max(m_A, m_B)).
 #pragma once
-
-#include <type_traits>
 
 #include "hf_ptx.cuh"
 
@@ -47,10 +45,12 @@ namespace hf {
 constexpr uint32_t kKernAttn = 3;
 constexpr int kAttnThreads = 384;
 constexpr int kRegsSupport = 104;   // registers per thread, producer/MMA warpgroup
-constexpr int kRegsRows = 200;     // registers per thread, row warpgroups
+constexpr int kRegsRows = 200;     // registers per thread, softmax warpgroups
 static_assert(128 * kRegsSupport + 256 * kRegsRows <= kAttnThreads * 168, "setmaxnreg split exceeds the launch");
-constexpr int kSmemLimit = 232448;  // max dynamic shared memory per CTA on sm_100
+constexpr int kSmemLimit = 232448;  // max shared memory per CTA on sm_100
+constexpr int kAttnStaticSmem = 1024;  // upper bound of the kernel's static shared memory
 constexpr int kPolyOf8 = 3;         // pairs (of every 8) that take exp2 on the FMA pipe
+constexpr int kMaxSlots = 6;
 
 template <int D, int BLK>
 struct AttnCfg {
@@ -58,22 +58,20 @@ struct AttnCfg {
   static constexpr int kQBytes = 128 * D * 2;
   static constexpr int kKVTileBytes = BLK * D * 2;
   static constexpr int kReadoutBytes = 2 * D * D * 2;  // S_hi + S_lo (bf16, d x d each)
-  // K slots free right after their QK^T, V slots only after their PV, two softmax periods
-  // before the slot is needed again: K gets the deeper ring.
-  static constexpr int kTiles = (kSmemLimit - 6144 - 1024 - kQBytes) / kKVTileBytes;
-  static constexpr int kKSlots = ((kTiles + 1) / 2) < 4 ? ((kTiles + 1) / 2) : 4;
-  static constexpr int kVSlots = (kTiles - kKSlots) < 4 ? (kTiles - kKSlots) : 4;
+  static constexpr int kXchBytes = 3 * 2 * 128 * 4;    // end-of-tile exchange [m | l | den][pipe][row]
+  static constexpr int kTiles = (kSmemLimit - kAttnStaticSmem - 1024 - kQBytes) / kKVTileBytes;
+  static constexpr int kKSlots = ((kTiles + 1) / 2) < kMaxSlots ? ((kTiles + 1) / 2) : kMaxSlots;
+  static constexpr int kVSlots = (kTiles - kKSlots) < kMaxSlots ? (kTiles - kKSlots) : kMaxSlots;
   static_assert(kKSlots >= 2 && kVSlots >= 2, "ring too small");
-  static_assert(kReadoutBytes <= (kKSlots + kVSlots) * kKVTileBytes, "readout operands must fit in the rings");
+  static_assert(kReadoutBytes + kXchBytes <= (kKSlots + kVSlots) * kKVTileBytes,
+                "readout operands and the exchange must fit in the rings");
   static constexpr int kDynSmem = 1024 + kQBytes + (kKSlots + kVSlots) * kKVTileBytes;
-  static constexpr uint32_t kColS = 0;      // S buffers at 0 and 128
-  static constexpr uint32_t kColO = 256;
-  static constexpr uint32_t kColQ = 384;
-  static constexpr uint32_t kColP = 448;
+  static_assert(kDynSmem + kAttnStaticSmem <= kSmemLimit, "shared memory");
+  static constexpr uint32_t kColS = 0;      // S_A at 0, S_B at 128
+  static constexpr uint32_t kColO = 256;    // O_A at 256, O_B at 384
   static constexpr uint32_t kColLin = 0;    // linear term (after the last block)
   static constexpr uint32_t kColPhi = 128;  // phi(q) hi | lo (after the last block)
-  static constexpr int kHB = BLK / 2;       // S columns per half-row thread
-  static constexpr int kHD = D / 2;         // O columns per half-row thread
+  static constexpr int kHD = D / 2;         // output / phi columns per pipeline thread at the end
 };
 
 struct AttnParams {
@@ -95,21 +93,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   using C = AttnCfg<D, BLK>;
   constexpr int NSK = C::kKSlots;
   constexpr int NSV = C::kVSlots;
-  constexpr int HB = C::kHB;
   constexpr int HD = C::kHD;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                             // Q tile; reused as the output staging tile
   uint8_t* kring = smem + C::kQBytes;              // NSK K slots
-  uint8_t* vring = kring + NSK * C::kKVTileBytes;  // NSV V slots (S_hi/S_lo over both rings at the end)
+  uint8_t* vring = kring + NSK * C::kKVTileBytes;  // NSV V slots (S_hi/S_lo + exchange over both rings at the end)
 
-  __shared__ uint64_t q_bar, qt_bar, kfull_bar[NSK], kempty_bar[NSK], vfull_bar[NSV], vempty_bar[NSV];
-  __shared__ uint64_t sfull_bar[2], sfree_bar[2], pfull_bar, pdone_bar[2], xch_bar[4];
-  __shared__ uint64_t final_bar, pro_bar, lin_bar, drain_bar;
+  __shared__ uint64_t q_bar, kfull_bar[NSK], kempty_bar[NSK], vfull_bar[NSV], vempty_bar[NSV];
+  __shared__ uint64_t sfull_bar[2], pfull_bar[2], final_bar, pro_bar, lin_bar, drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float z_sh[D];
-  __shared__ float xend[2][2][128];  // end-of-tile exchange: [den | l][half][row]
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x / p.nQB;
@@ -119,7 +113,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(&q_bar, 1);
-    mbar_init(&qt_bar, 256);
     for (int s = 0; s < NSK; ++s) {
       mbar_init(&kfull_bar[s], 1);
       mbar_init(&kempty_bar[s], 1);
@@ -128,13 +121,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&vfull_bar[s], 1);
       mbar_init(&vempty_bar[s], 1);
     }
-    for (int q = 0; q < 4; ++q) mbar_init(&xch_bar[q], 64);
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sfull_bar[b], 1);
-      mbar_init(&sfree_bar[b], 256);
-      mbar_init(&pdone_bar[b], 1);
+      mbar_init(&pfull_bar[b], 128);
     }
-    mbar_init(&pfull_bar, 256);
     mbar_init(&final_bar, 1);
     mbar_init(&pro_bar, 256);
     mbar_init(&lin_bar, 1);
@@ -152,14 +142,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tmem_alloc(&tmem_base_sh, 512);
     tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < D; i += kAttnThreads) z_sh[i] = p.z[static_cast<size_t>(bh) * D + i];
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
   if (warp < 4) {
-   // warpgroup 0: producers and MMA issuer give registers to the row warpgroups
+   // warpgroup 0: producers and MMA issuer give registers to the softmax warpgroups
    warpgroup_reg_dec<kRegsSupport>();
    if (warp == 0 || warp == 2) {
     // ============================ TMA producers ============================
@@ -201,7 +190,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
    } else if (warp == 1) {
     // ============================ MMA issuer ============================
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BLK, false, false);  // A=Q (TMEM), B=K: K-major
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, BLK, false, false);  // A=Q, B=K: both K-major
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);     // A=P (TMEM), B=V: MN-major
       constexpr uint32_t idesc_lin = idesc_bf16_f32(128, D, false, true);    // A=phi (TMEM), B=S: MN-major
       int n = 0;
@@ -212,44 +201,54 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // Descriptors are built once; an MMA only adds a constant offset (in 16-byte units)
       // to the 14-bit start-address field (shared-memory addresses stay below 256 KB, so the
       // field never carries). This keeps the single issuing thread ahead of the tensor core.
+      const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
       const uint64_t kdesc = sdesc_sw128(smem_u32(kring), 16, 1024);
       const uint64_t vdesc = sdesc_sw128(smem_u32(vring), BLK * 128, 1024);
-      auto issue_qk = [&](int j) {
-        const int s = j % NSK;
-        if (!mbar_wait(&kfull_bar[s], (j / NSK) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 6)) return false;
-        tc_fence_after();
-        const uint64_t kd = kdesc + static_cast<uint64_t>((s * C::kKVTileBytes) >> 4);
-        const uint32_t d_tmem = tmem + C::kColS + (j & 1) * 128;
+      // The tensor core's instruction queue is shallow: whatever this thread does between
+      // MMAs leaves it idle. So each kept block costs one wait and one commit here; the
+      // slot releases and the K / V arrival checks are done by the softmax threads.
+      // S of kept block v (valid position) into the S buffer of pipeline v % 2
+      auto qk = [&](int v) {
+        const uint64_t kd = kdesc + static_cast<uint64_t>(((v % NSK) * C::kKVTileBytes) >> 4);
+        const uint32_t d_tmem = tmem + C::kColS + (v & 1) * 128;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
+          constexpr int kQChunk = (128 * 128) >> 4;
           constexpr int kKChunk = (BLK * 128) >> 4;
-          umma_ts(d_tmem, tmem + C::kColQ + ks * 8, kd + (ks / 4) * kKChunk + (ks % 4) * 2, idesc_qk,
-                  ks > 0 ? 1u : 0u);
+          umma_ss(d_tmem, qdesc + (ks / 4) * kQChunk + (ks % 4) * 2, kd + (ks / 4) * kKChunk + (ks % 4) * 2,
+                  idesc_qk, ks > 0 ? 1u : 0u);
         }
-        umma_commit(&kempty_bar[s]);
-        if (!(p.inject && j == 0)) umma_commit(&sfull_bar[j & 1]);
-        return true;
       };
-      bool ok = mbar_wait(&qt_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 4);
-      for (int j = 0; j < 2 && j < n && ok; ++j) ok = issue_qk(j);
-      for (int j = 0; j < n && ok; ++j) {
-        // S_{j+2} into buffer j%2 as soon as the row threads hold S_j in registers
-        if (j + 2 < n) {
-          ok = mbar_wait(&sfree_bar[j & 1], (j >> 1) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 15) &&
-               issue_qk(j + 2);
-          if (!ok) break;
-        }
-        const int s = j % NSV;
-        if (!(ok = mbar_wait(&pfull_bar, j & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 7) &&
-                   mbar_wait(&vfull_bar[s], (j / NSV) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 14)))
-          break;
-        tc_fence_after();
-        const uint64_t vd = vdesc + static_cast<uint64_t>((s * C::kKVTileBytes) >> 4);
+      // O_p += P_p V for kept block v, p = v % 2 (P over the first columns of S_p)
+      auto pv = [&](int v) {
+        const int pp = v & 1;
+        const uint64_t vd = vdesc + static_cast<uint64_t>(((v % NSV) * C::kKVTileBytes) >> 4);
+        const uint32_t o_tmem = tmem + C::kColO + pp * 128;
+        const uint32_t p_tmem = tmem + C::kColS + pp * 128;
 #pragma unroll
         for (int ks = 0; ks < BLK / 16; ++ks)
-          umma_ts(tmem + C::kColO, tmem + C::kColP + ks * 8, vd + ks * 128, idesc_pv, (j > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(&vempty_bar[s]);
-        umma_commit(&pdone_bar[j & 1]);
+          umma_ts(o_tmem, p_tmem + ks * 8, vd + ks * 128, idesc_pv, (v > 1 || ks > 0) ? 1u : 0u);
+      };
+      bool ok = mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 4);
+      for (int v = 0; v < 2 && v < n && ok; ++v) {
+        if ((ok = mbar_wait(&kfull_bar[v], 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 6))) {
+          tc_fence_after();
+          qk(v);
+          if (!(p.inject && v == 0)) umma_commit(&sfull_bar[v]);
+        }
+      }
+      for (int v = 0; v < n && ok; ++v) {
+        // P_p(i) written, V(v) and K(v+2) landed (checked by the softmax threads)
+        if (!(ok = mbar_wait(&pfull_bar[v & 1], (v >> 1) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 7)))
+          break;
+        tc_fence_after();
+        pv(v);
+        // S_p(i+1) overwrites P_p(i): issued after PV_p(i), which the tensor core runs first;
+        // its commit also tells pipeline p that PV_p(i) is done (O_p stable, V slot free)
+        if (v + 2 < n) {
+          qk(v + 2);
+          umma_commit(&sfull_bar[v & 1]);
+        }
       }
       if (ok) {
         umma_commit(&final_bar);
@@ -276,57 +275,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
    }
   } else {
     warpgroup_reg_inc<kRegsRows>();
-    // ======================= row threads (softmax, readout, epilogue) =======================
+    // ======================= softmax pipelines, readout, epilogue =======================
     const int quarter = warp & 3;
-    const int half = (warp - 4) >> 2;     // 0: warps 4..7, 1: warps 8..11
+    const int pipe = (warp - 4) >> 2;     // 0: warps 4..7 (A), 1: warps 8..11 (B)
     const int row = quarter * 32 + lane;  // query row within the tile == TMEM lane
     const uint32_t lane_addr = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    // the two warps of a lane quarter meet once, at the end, on xch_bar[quarter]
-    // (an mbarrier: bounded wait)
-    uint64_t* pair_bar = &xch_bar[quarter];
-    // tcgen05.ld/st are warp-collective: every wait that guards one is made warp-uniform
-    bool ok = __all_sync(0xffffffffu, mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 9));
-    if (ok) {
-      // Q row -> TMEM as bf16 pairs (the A operand of S = Q K^T); this half's elements
-#pragma unroll
-      for (int g = 0; g < HD / 32; ++g) {
-        uint32_t w[16];
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const int unit = half * (HD / 8) + g * 4 + h;
-          const uint32_t off = (unit / 8) * (128 * 128) + row * 128 + (((unit % 8) ^ (row & 7)) * 16);
-          const uint4 qv = *reinterpret_cast<const uint4*>(sQ + off);
-          w[h * 4 + 0] = qv.x;
-          w[h * 4 + 1] = qv.y;
-          w[h * 4 + 2] = qv.z;
-          w[h * 4 + 3] = qv.w;
-        }
-        tmem_st16(lane_addr + C::kColQ + half * (HD / 2) + g * 16, w);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&qt_bar);
+    const uint32_t col_s = C::kColS + pipe * 128;
+    const uint32_t col_o = C::kColO + pipe * 128;
+    bool ok = true;
+    // lane 0 of the pipeline's first warp releases ring slots and checks tile arrivals
+    const bool elected = (warp & 3) == 0 && lane == 0;
+    int n_valid = 0;  // kept blocks with a valid index (the same count the MMA issuer uses)
+    for (int jj = 0; jj < p.r; ++jj) {
+      const int J = __ldg(idx_row + jj);
+      n_valid += (J >= 0 && J < p.nKB);
     }
 
-    // ---- online softmax over the kept blocks (this thread: columns [half*HB, half*HB+HB))
+    // ---- online softmax over this pipeline's kept blocks (the whole row per thread)
     float m_run = -INFINITY, l_run = 0.f;
-    int j = 0;
+    int v = 0, i = 0;  // valid kept position, blocks of this pipeline so far
     for (int jj = 0; jj < p.r && ok; ++jj) {
       const int J = __ldg(idx_row + jj);
       if (J < 0 || J >= p.nKB) continue;
-      const int b = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sfull_bar[b], (j >> 1) & 1, abort_flag, p.timeout_ns,
+      if ((v++ & 1) != pipe) continue;
+      // tcgen05.ld/st are warp-collective: every wait that guards one is made warp-uniform
+      ok = __all_sync(0xffffffffu, mbar_wait(&sfull_bar[pipe], i & 1, abort_flag, p.timeout_ns,
                                              (kKernAttn << 8) | 10));
       if (!ok) break;
       tc_fence_after();
-      // the whole row of S_j: the full-row max is computed by both warps of the quarter
-      // (no exchange between them); each keeps only its half for the exponentials
+      const int vb = v - 1;  // this block's valid position
+      if (elected) {
+        // S_p(i) done: QK(vb) has read its K slot; and PV_p(i-1), committed before it, its V slot
+        mbar_arrive(&kempty_bar[vb % NSK]);
+        if (i > 0) mbar_arrive(&vempty_bar[(vb - 2) % NSV]);
+      }
       uint32_t sr[BLK];
-      tmem_ld_cols<BLK>(lane_addr + C::kColS + b * 128, sr);
+      tmem_ld_cols<BLK>(lane_addr + col_s, sr);
       tmem_wait_ld();
       reg_fence<BLK>(sr);
-      tc_fence_before();
-      mbar_arrive(&sfree_bar[b]);  // S_j is in registers: the buffer may take S_{j+2}
       float* srow = reinterpret_cast<float*>(sr);
       const int valid = (J == p.nKB - 1) ? p.last_len : BLK;
       if (valid < BLK) {  // partial last key block: padding columns are masked out
@@ -334,142 +320,139 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int c = 0; c < BLK; ++c)
           if (c >= valid) srow[c] = -INFINITY;
       }
-      // row max: 8 independent chains of 3-input max
-      float mc[8];
+      // row max: independent chains of 3-input max
+      constexpr int kMC = BLK >= 64 ? 8 : 4;
+      float mc[kMC];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mc[k] = fmaxf(srow[k], srow[k + 8]);
+      for (int k = 0; k < kMC; ++k) mc[k] = fmaxf(srow[k], srow[k + kMC]);
 #pragma unroll
-      for (int c = 16; c < BLK; c += 16) {
+      for (int c = 2 * kMC; c < BLK; c += 2 * kMC) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mc[k] = fmax3(mc[k], srow[c + k], srow[c + 8 + k]);
+        for (int k = 0; k < kMC; ++k) mc[k] = fmax3(mc[k], srow[c + k], srow[c + kMC + k]);
       }
-      const float mx =
-          fmax3(fmax3(mc[0], mc[1], mc[2]), fmax3(mc[3], mc[4], mc[5]), fmaxf(mc[6], mc[7])) * p.scale_log2;
-      bool o_ready = j == 0;  // PV_{j-1} done (O final for j-1, P region free)
-      if (j == 0) {
+      float mx = mc[0];
+#pragma unroll
+      for (int k = 1; k < kMC; ++k) mx = fmaxf(mx, mc[k]);
+      mx *= p.scale_log2;
+      // A row raises its running max only when the block max exceeds it by more than 8
+      // (log2 units); O_p and l are then scaled by alpha = 2^(m_old - m_new).
+      float alpha = 1.0f;
+      const bool need = i > 0 && mx > m_run + 8.0f;
+      if (i == 0) {
         m_run = mx;
-      } else {
-        // A row raises its running max only when the block max exceeds it by more than
-        // 8 (log2 units); the O rescale is done by the whole warp whenever any of its
-        // rows needs it (alpha = 1 for the others); it waits for PV_{j-1}.
-        const bool need = mx > m_run + 8.0f;
-        if (__any_sync(0xffffffffu, need)) {
-          const float alpha = need ? ex2_approx(m_run - mx) : 1.0f;
-          ok = __all_sync(0xffffffffu, mbar_wait(&pdone_bar[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
-                                                 p.timeout_ns, (kKernAttn << 8) | 11));
-          if (!ok) break;
-          o_ready = true;
-          tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < HD; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + C::kColO + half * HD + c, o);
-            tmem_wait_ld();
-            reg_fence<32>(o);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(lane_addr + C::kColO + half * HD + c, o);
-          }
-          if (need) {
-            l_run *= alpha;
-            m_run = mx;
-          }
-        }
+      } else if (need) {
+        alpha = ex2_approx(m_run - mx);
+        l_run *= alpha;
+        m_run = mx;
       }
-      // p = 2^(s * scale * log2 e - m) over this warp's half of the row: packed fp32 pairs;
+      // p = 2^(s * scale * log2 e - m) as packed fp32 pairs, 32 columns at a time; each
+      // chunk of P goes to TMEM over the first columns of S_p at once (S is in registers).
       // kPolyOf8 pairs of every 8 run exp2 on the FMA pipe, the others on MUFU, so neither
-      // unit alone sets the pace. The half is a compile-time offset (a runtime index into
-      // the register array would move it to local memory).
-      uint32_t pk[HB / 2];
-      auto exp_half = [&](auto off) {
-        constexpr int OFF = decltype(off)::value;
+      // unit alone sets the pace.
+      {
         const uint64_t sl2 = f32x2(p.scale_log2, p.scale_log2);
         const uint64_t nm2 = f32x2(-m_run, -m_run);
         uint64_t lacc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-        for (int c = 0; c < HB; c += 2) {
-          const uint64_t x2 = ffma2(f32x2(srow[OFF + c], srow[OFF + c + 1]), sl2, nm2);
-          float p0, p1;
-          if (((c / 2) & 7) >= 8 - kPolyOf8) {
-            exp2_poly_x2(x2, p0, p1);
-          } else {
-            float x0, x1;
-            f32x2_split(x2, x0, x1);
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
+        for (int c0 = 0; c0 < BLK; c0 += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = c0; c < c0 + 32; c += 2) {
+            const uint64_t x2 = ffma2(f32x2(srow[c], srow[c + 1]), sl2, nm2);
+            float p0, p1;
+            if (((c / 2) & 7) >= 8 - kPolyOf8) {
+              exp2_poly_x2(x2, p0, p1);
+            } else {
+              float x0, x1;
+              f32x2_split(x2, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            lacc[(c / 2) & 3] = fadd2(lacc[(c / 2) & 3], f32x2(p0, p1));
+            pk[(c - c0) / 2] = pack_bf16x2(p0, p1);
           }
-          lacc[(c / 2) & 3] = fadd2(lacc[(c / 2) & 3], f32x2(p0, p1));
-          pk[c / 2] = pack_bf16x2(p0, p1);
+          tmem_st16(lane_addr + col_s + c0 / 2, pk);
         }
         const uint64_t l2 = fadd2(fadd2(lacc[0], lacc[1]), fadd2(lacc[2], lacc[3]));
         float la, lb;
         f32x2_split(l2, la, lb);
         l_run += la + lb;
-      };
-      // p = 2^(s * scale * log2 e - m) over this warp's half of the row: packed fp32 pairs;
-      // kPolyOf8 pairs of every 8 run exp2 on the FMA pipe, the others on MUFU, so neither
-      // unit alone sets the pace. The half is a compile-time offset (a runtime index into
-      // the register array would move it to local memory).
-      if (half == 0) {
-        exp_half(std::integral_constant<int, 0>{});
-      } else {
-        exp_half(std::integral_constant<int, HB>{});
       }
-      // P_j -> the P region once PV_{j-1} has read P_{j-1} (normally long done by now)
-      if (!o_ready) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&pdone_bar[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag,
-                                               p.timeout_ns, (kKernAttn << 8) | 16));
-        if (!ok) break;
-        tc_fence_after();
+      // lazy O rescale, by the whole warp whenever any of its rows needs it (alpha = 1 for
+      // the others); O_p is stable: PV_p(i-1) completed before S_p(i) was signalled
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + col_o + c, o);
+          tmem_wait_ld();
+          reg_fence<32>(o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_st32(lane_addr + col_o + c, o);
+        }
       }
-      tmem_st_cols<HB / 2>(lane_addr + C::kColP + half * (HB / 2), pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&pfull_bar);
-      ++j;
+      if (elected) {
+        // the MMA issuer runs PV(vb) and QK(vb+2) on this signal: their tiles must be there
+        bool tiles = mbar_wait(&vfull_bar[vb % NSV], (vb / NSV) & 1, abort_flag, p.timeout_ns,
+                               (kKernAttn << 8) | 14);
+        if (tiles && vb + 2 < n_valid)
+          tiles = mbar_wait(&kfull_bar[(vb + 2) % NSK], ((vb + 2) / NSK) & 1, abort_flag, p.timeout_ns,
+                            (kKernAttn << 8) | 15);
+        ok = tiles;
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      mbar_arrive(&pfull_bar[pipe]);
+      ++i;
     }
 
-    // ---- linear term operands (all PV done: the S buffers and both rings are free)
+    // ---- linear term operands (all MMAs done: the S buffers and both rings are free)
     ok = ok && mbar_wait(&final_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 12);
     ok = __all_sync(0xffffffffu, ok);
-    float den = 1.0f, l_tot = 0.f;
+    float dacc = 0.f;
     if (ok) {
       tc_fence_after();
-      float dacc = 0.f;
+      const float* zrow = p.z + static_cast<size_t>(bh) * D;
 #pragma unroll
       for (int g = 0; g < HD / 32; ++g) {  // 32 elements -> 16 packed columns of hi and of lo
         uint32_t hi[16], lo[16];
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          const int unit = half * (HD / 8) + g * 4 + h;  // elements [8*unit, 8*unit + 8)
+          const int unit = pipe * (HD / 8) + g * 4 + h;  // elements [8*unit, 8*unit + 8)
           const uint32_t off = (unit / 8) * (128 * 128) + row * 128 + (((unit % 8) ^ (row & 7)) * 16);
           const uint4 qv = *reinterpret_cast<const uint4*>(sQ + off);
+          const float4 za = __ldg(reinterpret_cast<const float4*>(zrow + unit * 8));
+          const float4 zb = __ldg(reinterpret_cast<const float4*>(zrow + unit * 8 + 4));
           const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
+          const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float x0 = bf16_lo_to_f32(w[e]), x1 = bf16_hi_to_f32(w[e]);
             const float p0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
             const float p1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
-            dacc = fmaf(p0, z_sh[unit * 8 + 2 * e], dacc);
-            dacc = fmaf(p1, z_sh[unit * 8 + 2 * e + 1], dacc);
+            dacc = fmaf(p0, zz[2 * e], dacc);
+            dacc = fmaf(p1, zz[2 * e + 1], dacc);
             const uint32_t hh = pack_bf16x2(p0, p1);
             hi[h * 4 + e] = hh;
             lo[h * 4 + e] = pack_bf16x2(p0 - bf16_lo_to_f32(hh), p1 - bf16_hi_to_f32(hh));
           }
         }
         // TMEM column c holds elements (2c, 2c+1) of the row: hi at [0, D/2), lo at [D/2, D)
-        tmem_st16(lane_addr + C::kColPhi + half * (HD / 2) + g * 16, hi);
-        tmem_st16(lane_addr + C::kColPhi + D / 2 + half * (HD / 2) + g * 16, lo);
+        tmem_st16(lane_addr + C::kColPhi + pipe * (HD / 2) + g * 16, hi);
+        tmem_st16(lane_addr + C::kColPhi + D / 2 + pipe * (HD / 2) + g * 16, lo);
       }
-      // state rows: thread (k, half) converts S[bh][k][half*D/2 .. +D/2) into MN-major bf16
-      // hi/lo tiles over the idle rings
+      // state rows: thread (k, pipe) converts S[bh][k][pipe*D/2 .. +D/2) into MN-major
+      // bf16 hi/lo tiles over the idle rings
       if (row < D) {
         const float* srow = p.S + (static_cast<size_t>(bh) * D + row) * D;
         uint8_t* s_hi = kring;
         uint8_t* s_lo = kring + D * D * 2;
 #pragma unroll 4
         for (int u = 0; u < HD / 8; ++u) {
-          const int unit = half * (HD / 8) + u;
+          const int unit = pipe * (HD / 8) + u;
           const float4 a = __ldg(reinterpret_cast<const float4*>(srow + unit * 8));
           const float4 b = __ldg(reinterpret_cast<const float4*>(srow + unit * 8 + 4));
           const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -489,29 +472,43 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&pro_bar);
-      // combine the two halves' partial denominators and row sums
-      xend[0][half][row] = dacc;
-      xend[1][half][row] = l_run;
-      mbar_arrive(pair_bar);  // the pair barrier's only phase
-      ok = __all_sync(0xffffffffu, mbar_wait(pair_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 18));
-      den = dacc + xend[0][half ^ 1][row] + 1e-6f;
-      l_tot = l_run + xend[1][half ^ 1][row];
     }
+    // ---- merge of the two pipelines' softmax states and denominators (every row thread
+    // reaches both named barriers, whatever happened before)
+    float* xch = reinterpret_cast<float*>(kring + C::kReadoutBytes);  // [3][2][128]
+    xch[(0 * 2 + pipe) * 128 + row] = m_run;
+    xch[(1 * 2 + pipe) * 128 + row] = l_run;
+    xch[(2 * 2 + pipe) * 128 + row] = dacc;
+    named_bar_sync(1, 256);
+    const float m_a = xch[(0 * 2 + 0) * 128 + row], m_b = xch[(0 * 2 + 1) * 128 + row];
+    const float l_a = xch[(1 * 2 + 0) * 128 + row], l_b = xch[(1 * 2 + 1) * 128 + row];
+    const float den = xch[(2 * 2 + 0) * 128 + row] + xch[(2 * 2 + 1) * 128 + row] + 1e-6f;
+    // a pipeline without blocks has m = -inf: weight 0, and its O (never written) unused
+    const float m_tot = fmaxf(m_a, m_b);
+    const bool has_a = m_a > -INFINITY, has_b = m_b > -INFINITY;
+    const float w_a = has_a ? ex2_approx(m_a - m_tot) : 0.f;
+    const float w_b = has_b ? ex2_approx(m_b - m_tot) : 0.f;
+    const float l_tot = (has_a ? l_a * w_a : 0.f) + (has_b ? l_b * w_b : 0.f);
+    const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.0f;
+    const float inv_den = 1.0f / den;
 
-    // ---- epilogue: O = O_s / l + O_lin / den -> bf16 -> TMA store of the block's rows
+    // ---- epilogue: this thread's half of the columns of
+    // O = (w_A O_A + w_B O_B) / l + O_lin / den -> bf16 -> TMA store of the block's rows
     ok = ok && mbar_wait(&lin_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 13);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       tc_fence_after();
-      const float inv_l = (j > 0 && l_tot > 0.f) ? 1.0f / l_tot : 0.0f;
-      const float inv_den = 1.0f / den;
+      const float sa = w_a * inv_l, sb = w_b * inv_l;
 #pragma unroll
       for (int c = 0; c < HD; c += 32) {
-        uint32_t o[32], lin[32];
-        tmem_ld32(lane_addr + C::kColO + half * HD + c, o);
-        tmem_ld32(lane_addr + C::kColLin + half * HD + c, lin);
+        const uint32_t col = pipe * HD + c;
+        uint32_t oa[32], ob[32], lin[32];
+        tmem_ld32(lane_addr + C::kColO + col, oa);
+        tmem_ld32(lane_addr + C::kColO + 128 + col, ob);
+        tmem_ld32(lane_addr + C::kColLin + col, lin);
         tmem_wait_ld();
-        reg_fence<32>(o);
+        reg_fence<32>(oa);
+        reg_fence<32>(ob);
         reg_fence<32>(lin);
         if (row < BLK) {
 #pragma unroll
@@ -519,13 +516,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int k = u * 8 + 2 * e;
-              const float y0 = (j > 0 ? __uint_as_float(o[k]) * inv_l : 0.f) + __uint_as_float(lin[k]) * inv_den;
-              const float y1 =
-                  (j > 0 ? __uint_as_float(o[k + 1]) * inv_l : 0.f) + __uint_as_float(lin[k + 1]) * inv_den;
-              w[e] = pack_bf16x2(y0, y1);
+              float y[2];
+#pragma unroll
+              for (int t = 0; t < 2; ++t) {
+                const int k = u * 8 + 2 * e + t;
+                const float s_a = has_a ? __uint_as_float(oa[k]) * sa : 0.f;
+                const float s_b = has_b ? __uint_as_float(ob[k]) * sb : 0.f;
+                y[t] = (s_a + s_b) + __uint_as_float(lin[k]) * inv_den;
+              }
+              w[e] = pack_bf16x2(y[0], y[1]);
             }
-            const int unit = (half * HD + c) / 8 + u;
+            const int unit = col / 8 + u;
             const uint32_t off = (unit / 8) * (BLK * 128) + row * 128 + (((unit % 8) ^ (row & 7)) * 16);
             *reinterpret_cast<uint4*>(sQ + off) = make_uint4(w[0], w[1], w[2], w[3]);
           }
