@@ -19,7 +19,11 @@
 //               into a ring of K slots (row coordinate J*block; rows past Nk are
 //               zero-filled); a K slot frees as soon as its QK^T is done.
 //   warp 1      TMEM owner (512 columns) + single-thread tcgen05 MMA issuer.
-//   warp 2      TMA producer of the V tiles into a ring of V slots. (warp 3 idles)
+//   warp 2      TMA producer of the V tiles into a ring of V slots.
+//   warp 3      ring bookkeeping, off the softmax threads' path: in kept-block order it
+//               waits for S of block v (so QK(v), and PV(v-2) before it, are done), frees
+//               their K and V slots, waits for V(v) and K(v+2) to land, and adds its arrival
+//               to pipeline v%2's P-ready barrier (which also counts the 128 softmax threads).
 //   warps 4..7  pipeline A, warps 8..11 pipeline B: one thread per query row (TMEM lane
 //               quarter = warp % 4), the whole row of S per thread.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+d), O_B [384,384+d). P (bf16
@@ -123,7 +127,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sfull_bar[b], 1);
-      mbar_init(&pfull_bar[b], 128);
+      mbar_init(&pfull_bar[b], 129);
     }
     mbar_init(&final_bar, 1);
     mbar_init(&pro_bar, 256);
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const uint64_t vdesc = sdesc_sw128(smem_u32(vring), BLK * 128, 1024);
       // The tensor core's instruction queue is shallow: whatever this thread does between
       // MMAs leaves it idle. So each kept block costs one wait and one commit here; the
-      // slot releases and the K / V arrival checks are done by the softmax threads.
+      // slot releases and the K / V arrival checks are done by warp 3.
       // S of kept block v (valid position) into the S buffer of pipeline v % 2
       auto qk = [&](int v) {
         const uint64_t kd = kdesc + static_cast<uint64_t>(((v % NSK) * C::kKVTileBytes) >> 4);
@@ -238,7 +242,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       for (int v = 0; v < n && ok; ++v) {
-        // P_p(i) written, V(v) and K(v+2) landed (checked by the softmax threads)
+        // P_p(i) written, V(v) and K(v+2) landed (checked by warp 3)
         if (!(ok = mbar_wait(&pfull_bar[v & 1], (v >> 1) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 7)))
           break;
         tc_fence_after();
@@ -272,6 +276,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0, p.timeout_ns, (kKernAttn << 8) | 8);
     }
+   } else {
+    // ============================ ring bookkeeping ============================
+    if (lane == 0) {
+      int n = 0;
+      for (int jj = 0; jj < p.r; ++jj) {
+        const int J = __ldg(idx_row + jj);
+        n += (J >= 0 && J < p.nKB);
+      }
+      // Every barrier below is waited on phase after phase, in order, by this one thread,
+      // so a parity wait can never be satisfied by an older phase.
+      for (int v = 0; v < n; ++v) {
+        const int pp = v & 1, i = v >> 1;
+        // S_p(i) done: QK(v) has read K(v); PV(v-2), committed before it, has read V(v-2).
+        // (P-ready phase i-1 of this pipeline is therefore complete too.)
+        if (!mbar_wait(&sfull_bar[pp], i & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 17)) break;
+        mbar_arrive(&kempty_bar[v % NSK]);
+        if (i > 0) mbar_arrive(&vempty_bar[(v - 2) % NSV]);
+        // the MMA issuer runs PV(v) and QK(v+2) on P-ready: their tiles must be there
+        if (!mbar_wait(&vfull_bar[v % NSV], (v / NSV) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 14)) break;
+        if (v + 2 < n &&
+            !mbar_wait(&kfull_bar[(v + 2) % NSK], ((v + 2) / NSK) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 15))
+          break;
+        mbar_arrive(&pfull_bar[pp]);
+      }
+    }
    }
   } else {
     warpgroup_reg_inc<kRegsRows>();
@@ -283,13 +312,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const uint32_t col_s = C::kColS + pipe * 128;
     const uint32_t col_o = C::kColO + pipe * 128;
     bool ok = true;
-    // lane 0 of the pipeline's first warp releases ring slots and checks tile arrivals
-    const bool elected = (warp & 3) == 0 && lane == 0;
-    int n_valid = 0;  // kept blocks with a valid index (the same count the MMA issuer uses)
-    for (int jj = 0; jj < p.r; ++jj) {
-      const int J = __ldg(idx_row + jj);
-      n_valid += (J >= 0 && J < p.nKB);
-    }
 
     // ---- online softmax over this pipeline's kept blocks (the whole row per thread)
     float m_run = -INFINITY, l_run = 0.f;
@@ -303,12 +325,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                              (kKernAttn << 8) | 10));
       if (!ok) break;
       tc_fence_after();
-      const int vb = v - 1;  // this block's valid position
-      if (elected) {
-        // S_p(i) done: QK(vb) has read its K slot; and PV_p(i-1), committed before it, its V slot
-        mbar_arrive(&kempty_bar[vb % NSK]);
-        if (i > 0) mbar_arrive(&vempty_bar[(vb - 2) % NSV]);
-      }
       uint32_t sr[BLK];
       tmem_ld_cols<BLK>(lane_addr + col_s, sr);
       tmem_wait_ld();
@@ -394,17 +410,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      if (elected) {
-        // the MMA issuer runs PV(vb) and QK(vb+2) on this signal: their tiles must be there
-        bool tiles = mbar_wait(&vfull_bar[vb % NSV], (vb / NSV) & 1, abort_flag, p.timeout_ns,
-                               (kKernAttn << 8) | 14);
-        if (tiles && vb + 2 < n_valid)
-          tiles = mbar_wait(&kfull_bar[(vb + 2) % NSK], ((vb + 2) / NSK) & 1, abort_flag, p.timeout_ns,
-                            (kKernAttn << 8) | 15);
-        ok = tiles;
-      }
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
       mbar_arrive(&pfull_bar[pipe]);
       ++i;
     }
