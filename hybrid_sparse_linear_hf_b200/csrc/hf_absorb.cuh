@@ -11,21 +11,28 @@
 // and writes an fp32 partial; reduce_state_kernel adds the partials of a head to S
 // and z in slice order (deterministic).
 //
-// absorb_partial_kernel (320 threads, one CTA per SM):
-//   warp 0      TMA producer: K and V tiles [64 tokens][d] into a 4-stage ring.
+// absorb_partial_kernel (576 threads, one CTA per SM):
+//   warp 0      TMA producer: K and V tiles [64 tokens][d] into a ring of stages. The
+//               kernel is bound by how many bytes each SM keeps in flight (HBM latency),
+//               so the ring takes all the shared memory left: 6 stages (192 KB) at d = 128.
 //   warp 1      TMEM owner + MMA issuer: for each tile, D += A_hi x V and D += A_lo x V
 //               with M = 128 (d-index of S, zero-padded for d = 64), N = d, K = 64
 //               tokens; both operands MN-major (d contiguous).
-//   warps 2..9  converters (two warps per SM sub-partition, for latency hiding): phi(k) in fp32, split hi = bf16(phi), lo = bf16(phi - hi)
-//               written at the same swizzled offsets as the K tile (the A operand has
-//               the K tile's layout), z accumulated in fp32 registers. They also drain
+//   warps 2..17 converters (four warps per SM sub-partition: the conversion is issue- and
+//               latency-bound, and it paces the whole kernel): phi(k) in
+//               fp32, split hi = bf16(phi), lo = bf16(phi - hi), z accumulated in fp32
+//               registers. The A operand has the K tile's layout, so at d = 128 hi
+//               overwrites the K tile in place and lo goes to one of two lo buffers; at
+//               d = 64 (M = 128 needs 64 zero rows after the tile) both go to separate
+//               zero-padded buffers. They also drain
 //               the accumulator: the tensor core's fp32 accumulation truncates, so a
 //               long chain of MMAs into one TMEM accumulator drifts (relative error
 //               grows with the chain length, ~2e-5 after 500 MMAs). The MMAs of every
 //               group of kAbsGroup tiles (16 MMAs) therefore go to one of two TMEM
 //               buffers, which the converters add into fp32 registers with
-//               round-to-nearest while the other buffer fills. Epilogue: registers ->
-//               fp32 partial in the workspace.
+//               round-to-nearest while the other buffer fills; the four warps that share
+//               a TMEM lane quarter take a quarter of the columns each. Epilogue:
+//               registers -> fp32 partial in the workspace.
 // Rows past the end of the token range are zero-filled by TMA; their phi is forced
 // to 0 (phi(0) = 1 would otherwise leak into z).
 #pragma once
@@ -36,8 +43,8 @@ namespace hf {
 
 constexpr uint32_t kKernAbsorb = 2;
 constexpr int kAbsTok = 64;        // tokens per tile
-constexpr int kAbsStages = 4;      // K/V ring depth
-constexpr int kConvThreads = 256;  // converter warps 2..9
+constexpr int kAbsMaxStages = 8;   // K/V ring depth cap
+constexpr int kConvThreads = 512;  // converter warps 2..17
 constexpr int kAbsThreads = 64 + kConvThreads;
 constexpr int kAbsGroup = 2;       // tiles per TMEM accumulation chain
 
@@ -48,8 +55,16 @@ struct AbsorbCfg {
   static constexpr int kTileBytes = kChunks * kChunkBytes;
   static constexpr int kStageBytes = 2 * kTileBytes;      // K tile + V tile
   static constexpr int kAOpBytes = 2 * kChunkBytes;       // A operand, M = 128 (2 chunks)
-  static constexpr int kABufBytes = 2 * kAOpBytes;        // hi + lo
-  static constexpr int kRingBytes = kAbsStages * kStageBytes;
+  static constexpr bool kInPlace = D == 128;              // hi over the K tile
+  static constexpr int kABufBytes = kInPlace ? kAOpBytes : 2 * kAOpBytes;  // [lo] or [hi | lo]
+  static constexpr int kZredBytes = kConvThreads * 8 * 4;  // end-of-kernel z reduction (over the ring)
+  static constexpr int kBudget = 232448 - 1024 - 1024;    // shared memory per CTA - alignment - static
+  static constexpr int kColsPerWarp = D / 4;              // drained accumulator columns per converter warp
+  static constexpr int kStagesFit = (kBudget - 2 * kABufBytes) / kStageBytes;
+  static constexpr int kStages = kStagesFit < kAbsMaxStages ? kStagesFit : kAbsMaxStages;
+  static_assert(kStages >= 2, "ring too small");
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static_assert(kZredBytes <= kRingBytes, "z reduction must fit over the ring");
   static constexpr int kDynSmem = 1024 + kRingBytes + 2 * kABufBytes;
 };
 
@@ -68,17 +83,17 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     absorb_partial_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                           AbsorbParams p) {
   using C = AbsorbCfg<D>;
+  constexpr int kAbsStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint8_t* abuf = smem + C::kRingBytes;  // [2][hi | lo]
+  uint8_t* abuf = smem + C::kRingBytes;  // [2][lo] (in place) or [2][hi | lo]
 
   __shared__ uint64_t full_bar[kAbsStages], empty_bar[kAbsStages];
   __shared__ uint64_t afull_bar[2], aempty_bar[2];
   __shared__ uint64_t dfull_bar[2], dempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
-  __shared__ float zred[kConvThreads][8];
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int bh = blockIdx.x / p.nsplit;
@@ -113,7 +128,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     tmem_alloc(&tmem_base_sh, 256);
     tmem_relinquish();
   }
-  if (D < 128 && warp >= 2) {
+  if (!C::kInPlace && warp >= 2) {
     // the upper 64 rows of the M = 128 A operand are zero padding for d = 64
     for (int i = threadIdx.x - 64; i < 2 * 2 * C::kChunkBytes / 16; i += kConvThreads) {
       const int a = i / (2 * C::kChunkBytes / 16), rem = i % (2 * C::kChunkBytes / 16);
@@ -160,6 +175,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
       // descriptors built once; each MMA adds a constant offset to the start address
       const uint64_t vdesc0 = sdesc_sw128(smem_u32(ring + C::kTileBytes), C::kChunkBytes, 1024);
+      const uint64_t kdesc0 = sdesc_sw128(smem_u32(ring), C::kChunkBytes, 1024);
       const uint64_t adesc0 = sdesc_sw128(smem_u32(abuf), C::kChunkBytes, 1024);
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
@@ -174,13 +190,16 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
         if (!ok) break;
         tc_fence_after();
         const uint64_t bd = vdesc0 + static_cast<uint64_t>((s * C::kStageBytes) >> 4);
-        const uint64_t ad = adesc0 + static_cast<uint64_t>((a * C::kABufBytes) >> 4);
+        const uint64_t ab = adesc0 + static_cast<uint64_t>((a * C::kABufBytes) >> 4);
+        // A operands: hi (over the K tile of stage s, or the first half of buffer a), lo
+        const uint64_t a_hi = C::kInPlace ? kdesc0 + static_cast<uint64_t>((s * C::kStageBytes) >> 4) : ab;
+        const uint64_t a_lo = C::kInPlace ? ab : ab + static_cast<uint64_t>(C::kAOpBytes >> 4);
         const uint32_t d_tmem = tmem_d + b * 128;
 #pragma unroll
         for (int op = 0; op < 2; ++op) {
 #pragma unroll
           for (int ks = 0; ks < kAbsTok / 16; ++ks)
-            umma_ss(d_tmem, ad + ((op * C::kAOpBytes) >> 4) + ks * 128, bd + ks * 128, idesc,
+            umma_ss(d_tmem, (op == 0 ? a_hi : a_lo) + ks * 128, bd + ks * 128, idesc,
                     (!first || op > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&empty_bar[s]);
@@ -201,15 +220,16 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     const int chunk = ucol / 8;
     const uint32_t swz = static_cast<uint32_t>(((ucol % 8) ^ (phase & 7)) * 16);
     uint64_t zacc[4] = {0ull, 0ull, 0ull, 0ull};  // fp32 pairs: elements (2e, 2e+1) of the unit
-    // register accumulator: row m of phi(K)^T V (TMEM lane m), columns [col0, col0 + D/2);
-    // the two warps that share a TMEM lane quarter take one half of the columns each
+    // register accumulator: row m of phi(K)^T V (TMEM lane m), columns [col0, col0 + D/4);
+    // the four warps that share a TMEM lane quarter (warp % 4) take a quarter each
+    constexpr int NC = C::kColsPerWarp;
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
-    const int col0 = (warp >= 6) ? D / 2 : 0;
+    const int col0 = ((warp - 2) / 4) * NC;
     const uint32_t lane_base = tmem_d + (static_cast<uint32_t>(quarter * 32) << 16);
-    float acc[D / 2];
+    float acc[NC];
 #pragma unroll
-    for (int c = 0; c < D / 2; ++c) acc[c] = 0.f;
+    for (int c = 0; c < NC; ++c) acc[c] = 0.f;
     const int ngroups = (ntiles + kAbsGroup - 1) / kAbsGroup;
     int flushed = 0;
     bool ok = true;
@@ -220,32 +240,29 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
                       mbar_wait(&dfull_bar[b], (g >> 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 8)))
         return false;
       tc_fence_after();
-#pragma unroll
-      for (int c0 = 0; c0 < D / 2; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(lane_base + b * 128 + col0 + c0, r);
+      {
+        uint32_t r[NC];
+        tmem_ld_cols<NC>(lane_base + b * 128 + col0, r);
         tmem_wait_ld();
-        reg_fence<32>(r);
+        reg_fence<NC>(r);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[c0 + j] += __uint_as_float(r[j]);
+        for (int j = 0; j < NC; ++j) acc[j] += __uint_as_float(r[j]);
       }
       tc_fence_before();
       mbar_arrive(&dempty_bar[b]);
       return true;
     };
-    // phi(x) = x + 1 (x > 0) or exp(x) (x <= 0) for the two bf16 halves of w, in fp32;
-    // hi = bf16(phi), lo = bf16(phi - hi); z accumulates phi.
+    // phi(x) = x + 1 (x > 0) or exp(x) (x <= 0) for the two bf16 halves of w, in fp32,
+    // written branch-free as max(x, 0) + 2^(min(x, 0) log2 e) (the exponential is 1 for
+    // x > 0); hi = bf16(phi), lo = bf16(phi - hi); z accumulates phi.
     auto convert_pair = [&](uint32_t w, uint64_t& z2, uint32_t& hi, uint32_t& lo) {
       const float x0 = bf16_lo_to_f32(w), x1 = bf16_hi_to_f32(w);
-      const uint64_t xl = ffma2(f32x2(x0, x1), f32x2(1.4426950408889634f, 1.4426950408889634f), 0ull);
       float l0, l1;
-      f32x2_split(xl, l0, l1);
-      const float e0 = ex2_approx(l0), e1 = ex2_approx(l1);
-      float a0, a1;
-      f32x2_split(fadd2(f32x2(x0, x1), f32x2(1.0f, 1.0f)), a0, a1);
-      const float p0 = x0 > 0.f ? a0 : e0;
-      const float p1 = x1 > 0.f ? a1 : e1;
-      const uint64_t pp = f32x2(p0, p1);
+      f32x2_split(ffma2(f32x2(fminf(x0, 0.f), fminf(x1, 0.f)),
+                        f32x2(1.4426950408889634f, 1.4426950408889634f), 0ull), l0, l1);
+      const uint64_t pp = fadd2(f32x2(fmaxf(x0, 0.f), fmaxf(x1, 0.f)), f32x2(ex2_approx(l0), ex2_approx(l1)));
+      float p0, p1;
+      f32x2_split(pp, p0, p1);
       z2 = fadd2(z2, pp);
       hi = pack_bf16x2(p0, p1);
       float r0, r1;
@@ -259,9 +276,9 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
                                        (kKernAbsorb << 8) | 7);
       ok = __all_sync(0xffffffffu, ok);  // the warp stays converged for the collective drain
       if (!ok) break;
-      const uint8_t* ktile = ring + s * C::kStageBytes;
-      uint8_t* ahi = abuf + a * C::kABufBytes;
-      uint8_t* alo = ahi + C::kAOpBytes;
+      uint8_t* ktile = ring + s * C::kStageBytes;
+      uint8_t* ahi = C::kInPlace ? ktile : abuf + a * C::kABufBytes;
+      uint8_t* alo = C::kInPlace ? abuf + a * C::kABufBytes : ahi + C::kAOpBytes;
       const int valid = min(kAbsTok, p.n_tokens - (tile0 + i) * kAbsTok);
 #pragma unroll
       for (int k = 0; k < kRowsPerThread; ++k) {
@@ -296,21 +313,24 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     if (ok) {
       for (int g = flushed; g < ngroups && ok; ++g) ok = flush_group(g);
     }
-    // z partial: reduce the kPhases row phases of each unit column
+    // z partial: reduce the kPhases row phases of each unit column (scratch over the ring,
+    // idle now: every tile has been converted and, once the last group was drained, every
+    // MMA is done)
+    float* zred = reinterpret_cast<float*>(ring);  // [kConvThreads][8]
 #pragma unroll
-    for (int e = 0; e < 4; ++e) f32x2_split(zacc[e], zred[t][2 * e], zred[t][2 * e + 1]);
+    for (int e = 0; e < 4; ++e) f32x2_split(zacc[e], zred[t * 8 + 2 * e], zred[t * 8 + 2 * e + 1]);
     named_bar_sync(1, kConvThreads);
     if (t < D) {
       const int uc = t / 8, e = t % 8;
       float zs = 0.f;
-      for (int ph = 0; ph < kPhases; ++ph) zs += zred[ph * kUnits + uc][e];
+      for (int ph = 0; ph < kPhases; ++ph) zs += zred[(ph * kUnits + uc) * 8 + e];
       p.part_z[(static_cast<size_t>(bh) * p.nsplit + split) * D + t] = zs;
     }
-    // S partial: row m, columns [col0, col0 + D/2) of this slice's phi(K)^T V
+    // S partial: row m, columns [col0, col0 + D/4) of this slice's phi(K)^T V
     if (ok && m < D) {
       float* dst = p.part_S + ((static_cast<size_t>(bh) * p.nsplit + split) * D + m) * D + col0;
 #pragma unroll
-      for (int j = 0; j < D / 2; j += 4)
+      for (int j = 0; j < NC; j += 4)
         *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
     }
   }
