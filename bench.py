@@ -43,6 +43,11 @@ UNIT = "query tokens/s"
 WORKLOAD = "832x480"
 L2_FLUSH_BYTES = 256 << 20
 LAUNCHES_PER_STEP = 5  # pool, score+select, hybrid attention, absorb partials, state reduce
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the current
+# hybrid_attn_kernel<128,128> on this workload, from one ncu capture of this script
+# (`ncu --set full --clock-control none -k regex:hybrid_attn -s 2 -c 1 ... bench.py
+# --steps 2 --warmup 3 --no-cpu-baseline`). Reset to None whenever the kernel changes.
+ATTN_TRAFFIC_BYTES = 161.3e6 + 12.8e6
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -393,7 +398,7 @@ def run_gpu(args, wl) -> None:
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_dict(wl),
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved_tf / peaks["bf16_tflops"], "traffic": None,
+                     "frac": achieved_tf / peaks["bf16_tflops"], "traffic": ATTN_TRAFFIC_BYTES,
                      "kernel": "hybrid_attn_kernel<128,128>", "flops_per_launch": F,
                      "peak_source": f"{peaks['source']} dense bf16 (burst)"},
         "kernels": {
