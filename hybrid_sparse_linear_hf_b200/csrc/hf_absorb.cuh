@@ -357,12 +357,22 @@ __global__ void __launch_bounds__(256) reduce_state_kernel(float* __restrict__ S
     float4* s4 = reinterpret_cast<float4*>(S + static_cast<size_t>(bh) * D * D) + e4;
     float4 acc = *s4;
     const float4* p4 = reinterpret_cast<const float4*>(part_S + static_cast<size_t>(bh) * nsplit * D * D) + e4;
-    for (int s = 0; s < nsplit; ++s) {
-      const float4 v = p4[static_cast<size_t>(s) * kVec4PerHead];
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
+    // all loads of a batch in flight, then the adds in slice order
+    constexpr int kBatch = 8;
+    for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
+      float4 v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (s0 + u < nsplit) v[u] = __ldg(p4 + static_cast<size_t>(s0 + u) * kVec4PerHead);
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        if (s0 + u < nsplit) {
+          acc.x += v[u].x;
+          acc.y += v[u].y;
+          acc.z += v[u].z;
+          acc.w += v[u].w;
+        }
+      }
     }
     *s4 = acc;
   }

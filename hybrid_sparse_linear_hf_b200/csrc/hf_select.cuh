@@ -13,9 +13,10 @@
 //                        HBM-bound: reads Q and K once with 16-byte loads, 8 in flight
 //                        per thread.
 //   score_select_kernel  one CTA per (b,h, 4 query blocks): s_IJ = Qbar_I . Kbar_J, a
-//                        thread per key block; then one warp per query block finds its
-//                        top r by a warp-wide bitwise search (ballots) for the r-th
-//                        largest (score, -J) key; the r blocks are written in ascending J.
+//                        thread per key block; then one warp per query block finds the
+//                        r-th largest score by a bitwise search (per-lane counts, one warp
+//                        reduction per bit), takes every block above it and the lowest-J
+//                        blocks equal to it, and writes the r blocks in ascending J.
 //                        NaN scores are ranked as -inf, so exactly r blocks are written.
 #pragma once
 
@@ -25,7 +26,7 @@ namespace hf {
 
 constexpr int kPoolThreads = 256;
 constexpr int kSelectThreads = 256;
-constexpr int kMaxKeyBlocks = 8192;  // 4 score rows fit in shared memory; J fits the 13-bit key field
+constexpr int kMaxKeyBlocks = 8192;  // 4 score rows of fp32 fit in shared memory
 
 __device__ __forceinline__ void acc_bf16x8(float* acc, uint4 v) {
   acc[0] += bf16_lo_to_f32(v.x);
@@ -105,7 +106,6 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bf
 // Scores of kSelQB query blocks of one head per CTA (each pooled K row is read once for
 // all of them), then one warp per query block selects its top r.
 constexpr int kSelQB = 4;
-constexpr int kSelRegKeys = 16;  // keys per lane held in registers (nKB <= 512)
 
 // Order-preserving map of a float to an unsigned integer (NaN has been replaced by -inf).
 __device__ __forceinline__ uint32_t ordered_bits(float f) {
@@ -113,18 +113,72 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Unique selection key of key block J: larger score first, lower index first on ties.
-__device__ __forceinline__ uint64_t select_key(float s, int J) {
-  return (static_cast<uint64_t>(ordered_bits(s)) << 13) | static_cast<uint64_t>(8191 - J);
+// Top-r of the scores srow[0..nKB) (larger score first, lower J first on ties), written
+// to out[0..r) in ascending J by one warp. NPL = ordered scores per lane held in registers
+// (lane l holds J = 32 k + l); NPL = 0 reads shared memory each time (any nKB).
+// 1. T = the r-th largest ordered score: the largest t with #{J : o_J >= t} >= r, found
+//    bit by bit from the top, each candidate counted per lane and summed over the warp.
+// 2. Keep every J with o_J > T, and the (r - #{o_J > T}) lowest J with o_J == T.
+template <int NPL>
+__device__ __forceinline__ void warp_top_r(const float* srow, int nKB, int r, int lane, int32_t* out) {
+  auto ob_at = [&](int J) -> uint32_t {
+    const float v = srow[J];
+    // NaN ranks last; -0 and +0 are one value (a tie, broken by J)
+    return ordered_bits(v != v ? -INFINITY : (v == 0.f ? 0.f : v));
+  };
+  constexpr int kRegs = NPL > 0 ? NPL : 1;
+  uint32_t o[kRegs];
+  if constexpr (NPL > 0) {
+#pragma unroll
+    for (int k = 0; k < NPL; ++k) o[k] = (32 * k + lane < nKB) ? ob_at(32 * k + lane) : 0u;
+  }
+  // Lanes past nKB are excluded from every count (their register holds 0).
+  auto count_ge = [&](uint32_t t) -> int {
+    int c = 0;
+    if constexpr (NPL > 0) {
+#pragma unroll
+      for (int k = 0; k < NPL; ++k) c += (32 * k + lane < nKB && o[k] >= t) ? 1 : 0;
+    } else {
+      for (int J = lane; J < nKB; J += 32) c += ob_at(J) >= t ? 1 : 0;
+    }
+    return static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
+  };
+  uint32_t T = 0;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = T | (1u << bit);
+    if (count_ge(cand) >= r) T = cand;
+  }
+  const int n_gt = T == 0xFFFFFFFFu ? 0 : count_ge(T + 1u);
+  const int n_eq_keep = r - n_gt;  // >= 1
+  int base = 0, eq_seen = 0;
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  for (int k = 0; 32 * k < nKB; ++k) {
+    const int J = 32 * k + lane;
+    uint32_t oj = 0;
+    if constexpr (NPL > 0) {
+#pragma unroll
+      for (int kk = 0; kk < NPL; ++kk)
+        if (kk == k) oj = o[kk];
+    } else {
+      oj = J < nKB ? ob_at(J) : 0u;
+    }
+    const bool valid = J < nKB;
+    const bool eq = valid && oj == T;
+    const uint32_t m_eq = __ballot_sync(0xffffffffu, eq);
+    const bool keep = valid && (oj > T || (eq && eq_seen + __popc(m_eq & lt_mask) < n_eq_keep));
+    const uint32_t m = __ballot_sync(0xffffffffu, keep);
+    const int pos = base + __popc(m & lt_mask);
+    if (keep) out[pos] = J;
+    base += __popc(m);
+    eq_seen += __popc(m_eq);
+  }
 }
 
 // idx_out[bh][I][0..r) = top-r key blocks of query block I, ascending.
 // Scores: thread per key block J, s_IJ = Qbar_I . Kbar_J for the CTA's kSelQB query blocks
 // (pooled Q in shared memory, the pooled K row streamed with 16-byte loads, all in flight).
-// Selection: the warp of query block I finds the r-th largest of the unique 45-bit keys
-// (ordered score bits << 13) | (8191 - J) bit by bit (counting keys at or above a
-// candidate with ballots); the blocks at or above it are exactly the top r, written in
-// ascending J with ballot prefix counts.
+// Selection: warp_top_r, one warp per query block.
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const float* __restrict__ Qp,
                                                                       const float* __restrict__ Kp, int nQB,
@@ -178,43 +232,13 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const floa
     float* sout = scores_out ? scores_out + (static_cast<size_t>(bh) * nQB + I) * nKB : nullptr;
     if (sout)
       for (int J = lane; J < nKB; J += 32) sout[J] = srow[J];
-    auto key_at = [&](int J) -> uint64_t {
-      const float v = srow[J];
-      return select_key(v != v ? -INFINITY : v, J);  // NaN ranks last
-    };
-    // largest T with #{keys >= T} >= r: the r-th largest key (keys are unique)
-    uint64_t T = 0;
-    if (nKB <= 32 * kSelRegKeys) {
-      uint64_t keys[kSelRegKeys];
-#pragma unroll
-      for (int k = 0; k < kSelRegKeys; ++k) keys[k] = (32 * k + lane < nKB) ? key_at(32 * k + lane) : 0ull;
-      for (int bit = 44; bit >= 0; --bit) {
-        const uint64_t cand = T | (1ull << bit);
-        int cnt = 0;
-#pragma unroll
-        for (int k = 0; k < kSelRegKeys; ++k) cnt += __popc(__ballot_sync(0xffffffffu, keys[k] >= cand));
-        if (cnt >= r) T = cand;
-      }
-    } else {
-      for (int bit = 44; bit >= 0; --bit) {
-        const uint64_t cand = T | (1ull << bit);
-        int cnt = 0;
-        for (int J0 = 0; J0 < nKB; J0 += 32) {
-          const int J = J0 + lane;
-          cnt += __popc(__ballot_sync(0xffffffffu, J < nKB && key_at(J) >= cand));
-        }
-        if (cnt >= r) T = cand;
-      }
-    }
     int32_t* out = idx_out + (static_cast<size_t>(bh) * nQB + I) * r;
-    int base = 0;
-    for (int J0 = 0; J0 < nKB; J0 += 32) {
-      const int J = J0 + lane;
-      const bool keep = J < nKB && key_at(J) >= T;
-      const uint32_t m = __ballot_sync(0xffffffffu, keep);
-      const int pos = base + __popc(m & ((1u << lane) - 1u));
-      if (keep && pos < r) out[pos] = J;
-      base += __popc(m);
+    if (nKB <= 256) {
+      warp_top_r<8>(srow, nKB, r, lane, out);
+    } else if (nKB <= 512) {
+      warp_top_r<16>(srow, nKB, r, lane, out);
+    } else {
+      warp_top_r<0>(srow, nKB, r, lane, out);
     }
   }
 }
