@@ -12,27 +12,29 @@
 // and z in slice order (deterministic).
 //
 // absorb_partial_kernel (576 threads, one CTA per SM):
-//   warp 0      TMA producer: K and V tiles [64 tokens][d] into a ring of stages. The
-//               kernel is bound by how many bytes each SM keeps in flight (HBM latency),
-//               so the ring takes all the shared memory left: 6 stages (192 KB) at d = 128.
+//   warp 0      TMA producer: K and V tiles [64 tokens][d] into a ring of stages taking
+//               the shared memory the A buffers leave (5 stages, 160 KB, at d = 128).
 //   warp 1      TMEM owner + MMA issuer: for each tile, D += A_hi x V and D += A_lo x V
 //               with M = 128 (d-index of S, zero-padded for d = 64), N = d, K = 64
-//               tokens; both operands MN-major (d contiguous).
+//               tokens; both operands MN-major (d contiguous). It waits only for the
+//               converters' "A written" barrier, which they arrive on after the tile's
+//               stage barrier (so the V tile has landed too).
 //   warps 2..17 converters (four warps per SM sub-partition: the conversion is issue- and
-//               latency-bound, and it paces the whole kernel): phi(k) in
-//               fp32, split hi = bf16(phi), lo = bf16(phi - hi), z accumulated in fp32
-//               registers. The A operand has the K tile's layout, so at d = 128 hi
-//               overwrites the K tile in place and lo goes to one of two lo buffers; at
-//               d = 64 (M = 128 needs 64 zero rows after the tile) both go to separate
-//               zero-padded buffers. They also drain
-//               the accumulator: the tensor core's fp32 accumulation truncates, so a
-//               long chain of MMAs into one TMEM accumulator drifts (relative error
-//               grows with the chain length, ~2e-5 after 500 MMAs). The MMAs of every
-//               group of kAbsGroup tiles (16 MMAs) therefore go to one of two TMEM
-//               buffers, which the converters add into fp32 registers with
-//               round-to-nearest while the other buffer fills; the four warps that share
-//               a TMEM lane quarter take a quarter of the columns each. Epilogue:
-//               registers -> fp32 partial in the workspace.
+//               latency-bound, and it paces the whole kernel): phi(k) in fp32, split
+//               hi = bf16(phi), lo = bf16(phi - hi), z accumulated in fp32 registers. The
+//               A operand has the K tile's layout, so at d = 128 hi overwrites the K tile
+//               in place and lo goes to one of four lo buffers (a buffer is reused once
+//               the MMAs of four tiles back are done; one wait every second tile covers
+//               two tiles); at d = 64 (M = 128 needs 64 zero rows after the tile) hi and
+//               lo go to two separate zero-padded buffers. They also drain the
+//               accumulator: the tensor core's fp32 accumulation truncates, so a long
+//               chain of MMAs into one TMEM accumulator drifts (relative error grows with
+//               the chain length, ~2e-5 after 500 MMAs). The MMAs of every group of
+//               kAbsGroup tiles (32 MMAs) therefore go to one of two TMEM buffers, which
+//               the converters add into fp32 registers with round-to-nearest while the
+//               other buffer fills; the four warps that share a TMEM lane quarter take a
+//               quarter of the columns each. Epilogue: registers -> fp32 partial in the
+//               workspace.
 // Rows past the end of the token range are zero-filled by TMA; their phi is forced
 // to 0 (phi(0) = 1 would otherwise leak into z).
 #pragma once
@@ -46,7 +48,7 @@ constexpr int kAbsTok = 64;        // tokens per tile
 constexpr int kAbsMaxStages = 8;   // K/V ring depth cap
 constexpr int kConvThreads = 512;  // converter warps 2..17
 constexpr int kAbsThreads = 64 + kConvThreads;
-constexpr int kAbsGroup = 2;       // tiles per TMEM accumulation chain
+constexpr int kAbsGroup = 4;       // tiles per TMEM accumulation chain
 
 template <int D>
 struct AbsorbCfg {
@@ -57,15 +59,16 @@ struct AbsorbCfg {
   static constexpr int kAOpBytes = 2 * kChunkBytes;       // A operand, M = 128 (2 chunks)
   static constexpr bool kInPlace = D == 128;              // hi over the K tile
   static constexpr int kABufBytes = kInPlace ? kAOpBytes : 2 * kAOpBytes;  // [lo] or [hi | lo]
+  static constexpr int kNA = kInPlace ? 4 : 2;            // A buffers
   static constexpr int kZredBytes = kConvThreads * 8 * 4;  // end-of-kernel z reduction (over the ring)
   static constexpr int kBudget = 232448 - 1024 - 1024;    // shared memory per CTA - alignment - static
   static constexpr int kColsPerWarp = D / 4;              // drained accumulator columns per converter warp
-  static constexpr int kStagesFit = (kBudget - 2 * kABufBytes) / kStageBytes;
+  static constexpr int kStagesFit = (kBudget - kNA * kABufBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit < kAbsMaxStages ? kStagesFit : kAbsMaxStages;
   static_assert(kStages >= 2, "ring too small");
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kZredBytes <= kRingBytes, "z reduction must fit over the ring");
-  static constexpr int kDynSmem = 1024 + kRingBytes + 2 * kABufBytes;
+  static constexpr int kDynSmem = 1024 + kRingBytes + kNA * kABufBytes;
 };
 
 struct AbsorbParams {
@@ -90,7 +93,8 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
   uint8_t* abuf = smem + C::kRingBytes;  // [2][lo] (in place) or [2][hi | lo]
 
   __shared__ uint64_t full_bar[kAbsStages], empty_bar[kAbsStages];
-  __shared__ uint64_t afull_bar[2], aempty_bar[2];
+  constexpr int NA = C::kNA;
+  __shared__ uint64_t afull_bar[NA], aempty_bar[NA];
   __shared__ uint64_t dfull_bar[2], dempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -108,7 +112,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NA; ++a) {
       mbar_init(&afull_bar[a], kConvThreads);
       mbar_init(&aempty_bar[a], 1);
     }
@@ -130,7 +134,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
   }
   if (!C::kInPlace && warp >= 2) {
     // the upper 64 rows of the M = 128 A operand are zero padding for d = 64
-    for (int i = threadIdx.x - 64; i < 2 * 2 * C::kChunkBytes / 16; i += kConvThreads) {
+    for (int i = threadIdx.x - 64; i < NA * 2 * C::kChunkBytes / 16; i += kConvThreads) {
       const int a = i / (2 * C::kChunkBytes / 16), rem = i % (2 * C::kChunkBytes / 16);
       const int op = rem / (C::kChunkBytes / 16), u = rem % (C::kChunkBytes / 16);
       reinterpret_cast<uint4*>(abuf + a * C::kABufBytes + op * C::kAOpBytes + C::kChunkBytes)[u] =
@@ -179,12 +183,12 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       const uint64_t adesc0 = sdesc_sw128(smem_u32(abuf), C::kChunkBytes, 1024);
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
-        const int s = i % kAbsStages, a = i & 1;
+        const int s = i % kAbsStages, a = i % NA;
         const int g = i / kAbsGroup, b = g & 1;
         const bool first = (i % kAbsGroup) == 0;
         const bool last = (i % kAbsGroup) == kAbsGroup - 1 || i == ntiles - 1;
-        ok = mbar_wait(&full_bar[s], (i / kAbsStages) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 3) &&
-             mbar_wait(&afull_bar[a], (i >> 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 4);
+        // A written implies the tile landed: the converters waited for the stage before arriving
+        ok = mbar_wait(&afull_bar[a], (i / NA) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 4);
         if (ok && first && g >= 2)
           ok = mbar_wait(&dempty_bar[b], ((g >> 1) - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 9);
         if (!ok) break;
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
                     (!first || op > 0 || ks > 0) ? 1u : 0u);
         }
         umma_commit(&empty_bar[s]);
-        umma_commit(&aempty_bar[a]);
+        if (NA == 2 || (i & 1)) umma_commit(&aempty_bar[a]);
         if (last) umma_commit(&dfull_bar[b]);
       }
       umma_commit(&drain_bar);
@@ -270,10 +274,17 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       lo = pack_bf16x2(r0, r1);
     };
     for (int i = 0; i < ntiles && ok; ++i) {
-      const int s = i % kAbsStages, a = i & 1;
+      const int s = i % kAbsStages, a = i % NA;
       ok = mbar_wait(&full_bar[s], (i / kAbsStages) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 6);
-      if (ok && i >= 2) ok = mbar_wait(&aempty_bar[a], ((i >> 1) - 1) & 1, abort_flag, p.timeout_ns,
-                                       (kKernAbsorb << 8) | 7);
+      // A buffer a is free once the MMAs of tile i - NA are done. With four buffers one wait
+      // every second tile suffices: at even i, MMA(i - 3) done covers tiles i and i + 1.
+      if (NA == 2) {
+        if (ok && i >= 2)
+          ok = mbar_wait(&aempty_bar[a], ((i >> 1) - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 7);
+      } else if (ok && i >= NA && (i & 1) == 0) {
+        const int t = i - NA + 1;
+        ok = mbar_wait(&aempty_bar[t % NA], (t / NA) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 7);
+      }
       ok = __all_sync(0xffffffffu, ok);  // the warp stays converged for the collective drain
       if (!ok) break;
       uint8_t* ktile = ring + s * C::kStageBytes;
