@@ -313,6 +313,50 @@ def test_full_size_workload_sampled(name):
         assert_output_close(Og[b, h, lo:hi], want, what=f"O tile {(b, h, I)}")
 
 
+def test_1280x720_workload_sampled():
+    """The 1280x720-shaped step (40 heads, 10800 query x 43200 key tokens, block 128, r 68):
+    every mask and the outputs of sampled query blocks against the oracle. The state holds
+    2 evicted frames here (the attention reads S and z the same way whatever they absorbed;
+    the 120-frame build is checked on two heads below)."""
+    wl = WORKLOADS["1280x720"]
+    x = draw_step_inputs(wl, n_evicted=2 * wl.tokens_per_frame)
+    Qd, Kd, Vd = x["Q"].to(DEV), x["K"].to(DEV), x["V"].to(DEV)
+    st = _state_from(x["K_ev"], x["V_ev"], wl.d)
+    scores = torch.empty(wl.B, wl.H, wl.nQB, wl.nKB, device=DEV)
+    idx_t = hf.hf_select_blocks(Qd, Kd, wl.block, wl.r, scores_out=scores)
+    O = hf.hf_hybrid_attn_fwd(Qd, Kd, Vd, wl.block, wl.r, idx_t, st)
+    torch.cuda.synchronize()
+    _check_status()
+    idx = idx_t.cpu().numpy()
+    Q64, K64, V64 = f64(x["Q"]), f64(x["K"]), f64(x["V"])
+    oidx, osc = oracle.select_blocks(Q64, K64, wl.block, wl.r)
+    assert np.abs(scores.cpu().numpy() - osc).max() <= SCORE_ABS
+    assert_masks_match(idx, oidx, osc, wl.r)
+    S_o, z_o = oracle.absorb_batch(f64(x["K_ev"]), f64(x["V_ev"]))
+    assert_state_close(f64(st.S), f64(st.z), S_o, z_o)
+    Og = f64(O)
+    for (b, h, I) in _sample_tiles(wl, 6, seed=1):
+        lo, hi = I * wl.block, min((I + 1) * wl.block, wl.Nq)
+        want = oracle.hybrid_attention_tile(Q64, K64, V64, idx, S_o, z_o, wl.block, b, h, I)
+        assert_output_close(Og[b, h, lo:hi], want, what=f"O tile {(b, h, I)}")
+
+
+def test_1280x720_state_build_sampled_heads():
+    """The 1280x720 state build as the bench would run it: 40 heads x 120 frames (432 000
+    tokens per head, 3 slices of 2250 tiles per head, so long per-CTA accumulations),
+    drawn on the device; two heads checked against the oracle."""
+    wl = WORKLOADS["1280x720"]
+    g = torch.Generator(device=DEV).manual_seed(wl.seed + 5000)
+    K = frame_structured(g, wl.B, wl.H, wl.Ne_state, wl.d, wl.tokens_per_frame, wl.w, DEV)
+    V = frame_structured(g, wl.B, wl.H, wl.Ne_state, wl.d, wl.tokens_per_frame, wl.w, DEV)
+    st = _state_from(K, V, wl.d)
+    _check_status()
+    for h in (0, wl.H - 1):
+        S_o, z_o = oracle.absorb_batch(f64(K[:, h:h + 1]), f64(V[:, h:h + 1]))
+        assert_state_close(f64(st.S[:, h:h + 1]), f64(st.z[:, h:h + 1]), S_o, z_o)
+    del K, V
+
+
 def test_attention_online_rescale_mixed_rows():
     """Even query rows meet much larger scores in later blocks (their running max must be
     raised twice, rescaling O) while odd rows do not: every warp mixes both cases."""
