@@ -20,7 +20,9 @@ Sources (page title, then the section used):
   [LF]     "Light Forcing: Accelerating Autoregressive Video Diffusion via
            Sparse Attention", German technical summary (gist.science),
            §2.2 Hierarchische Spärliche Attention (token compression by mean
-           pooling; per-query-block selection).
+           pooling at block and frame level; per-query-block selection; the
+           two-stage mask selection: frames first by frame-level compressed keys,
+           then blocks within the selected frames).
 
 The pages give the structure (a compact KV state absorbing evicted tokens
 through a linear attention function; Top-K block-sparse attention inside the
@@ -51,7 +53,8 @@ READOUT_EPS = 1e-6
 
 __all__ = [
     "READOUT_EPS", "phi", "block_ranges", "pool_blocks", "block_scores",
-    "select_blocks", "sparse_attention_tile", "sparse_attention", "linear_readout",
+    "select_blocks", "frame_ranges", "pool_frames", "frame_scores", "candidate_blocks",
+    "select_blocks_two_stage", "sparse_attention_tile", "sparse_attention", "linear_readout",
     "hybrid_attention", "hybrid_attention_tile", "absorb", "absorb_batch",
     "dense_swa", "default_scale",
 ]
@@ -126,6 +129,78 @@ def select_blocks(Q, K, block: int, r: int):
                 order = np.lexsort((order_key, -s[b, h, I]))
                 idx[b, h, I] = np.sort(order[:r])
     return idx, s
+
+
+def frame_ranges(n: int, tokens_per_frame: int) -> list[tuple[int, int]]:
+    """Token ranges [w*T, min((w+1)*T, n)) of the ceil(n/T) frames of a window."""
+    return block_ranges(n, tokens_per_frame)
+
+
+def pool_frames(K, tokens_per_frame: int) -> np.ndarray:
+    """Mean of the valid tokens of every frame: [B,H,N,d] -> [B,H,ceil(N/T),d].
+
+    [LF] §2.2: key tokens are also compressed by mean pooling at frame level.
+    """
+    return pool_blocks(K, tokens_per_frame)
+
+
+def frame_scores(Q, K, block: int, tokens_per_frame: int) -> np.ndarray:
+    """f[b,h,I,w] = pooled(Q, blocks)[I] . pooled(K, frames)[w] (unscaled), [B,H,nQB,W]."""
+    Qp = pool_blocks(Q, block)
+    Kf = pool_frames(K, tokens_per_frame)
+    return Qp @ np.swapaxes(Kf, -1, -2)
+
+
+def candidate_blocks(kept_frames, Nk: int, block: int, tokens_per_frame: int) -> np.ndarray:
+    """Key blocks whose token range intersects the token range of a kept frame (sorted)."""
+    frames = frame_ranges(Nk, tokens_per_frame)
+    out = []
+    for J, (lo, hi) in enumerate(block_ranges(Nk, block)):
+        if any(lo < frames[int(w)][1] and frames[int(w)][0] < hi for w in kept_frames):
+            out.append(J)
+    return np.asarray(out, dtype=np.int64)
+
+
+def select_blocks_two_stage(Q, K, block: int, r: int, tokens_per_frame: int, n_frames: int):
+    """Two-stage (frame, then block) top-r selection for every query block.
+
+    [LF] §2.2, "Zweistufige Maskenauswahl": for each query block the frames are
+    ranked by the frame-level compressed keys and a small set is kept; the blocks
+    within the kept frames are then ranked by the block-level compressed keys.
+    Readings: the n_frames frames of largest f_Iw are kept (equal scores: lower w
+    first); a key block lies within the kept frames when any of its tokens does; of
+    those candidate blocks the r of largest s_IJ are kept (equal scores: lower J
+    first) and returned in ascending J. Should fewer than r blocks touch the kept
+    frames (a short last frame), every candidate is kept and the remaining places go
+    to the best other blocks in the same order.
+
+    Returns (idx int32 [B,H,nQB,r], frames int32 [B,H,nQB,n_frames] ascending,
+    block scores float64 [B,H,nQB,nKB], frame scores float64 [B,H,nQB,W]).
+    """
+    s = block_scores(Q, K, block)
+    f = frame_scores(Q, K, block, tokens_per_frame)
+    B, H, nQB, nKB = s.shape
+    W = f.shape[-1]
+    Nk = np.asarray(K).shape[2]
+    if not 1 <= n_frames <= W:
+        raise ValueError(f"n_frames={n_frames} outside [1, {W}]")
+    if not 1 <= r <= nKB:
+        raise ValueError(f"r={r} outside [1, {nKB}]")
+    idx = np.empty((B, H, nQB, r), dtype=np.int32)
+    frames = np.empty((B, H, nQB, n_frames), dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            for I in range(nQB):
+                order = np.lexsort((np.arange(W), -f[b, h, I]))
+                kept = np.sort(order[:n_frames])
+                frames[b, h, I] = kept
+                cand = candidate_blocks(kept, Nk, block, tokens_per_frame)
+                is_cand = np.zeros(nKB, dtype=bool)
+                is_cand[cand] = True
+                # candidates first, then by decreasing score, then by increasing J
+                order = np.lexsort((np.arange(nKB), -s[b, h, I], ~is_cand))
+                idx[b, h, I] = np.sort(order[:r])
+    return idx, frames, s, f
 
 
 def _selected_tokens(kept_blocks, Nk: int, block: int) -> np.ndarray:

@@ -262,11 +262,95 @@ def check_hybrid_sum(o):
     assert np.allclose(tile, hyb[0, 1, 8:16], atol=1e-14)
 
 
+# ---------------------------------------------------------------------------
+# two-stage (frame, then block) selection
+# ---------------------------------------------------------------------------
+def check_two_stage_golden(o):
+    g = _golden()["two_stage_selection"]
+    Q, block, T = _as4(g["Q"]), g["block"], g["tokens_per_frame"]
+    for case in g["cases"]:
+        K = _as4(case["K"])
+        f = o.frame_scores(Q, K, block, T)[0, 0, 0]
+        assert np.allclose(f, case["frame_scores"], atol=1e-15, rtol=0), f"frame scores {f}"
+        s = o.block_scores(Q, K, block)[0, 0, 0]
+        assert np.allclose(s, case["block_scores"], atol=1e-15, rtol=0), f"block scores {s}"
+        for e in case["expect"]:
+            idx, frames, _, _ = o.select_blocks_two_stage(Q, K, block, e["r"], T, e["n_frames"])
+            assert frames[0, 0, 0].tolist() == e["frames"], (e, frames[0, 0, 0].tolist())
+            assert idx[0, 0, 0].tolist() == e["idx"], (e, idx[0, 0, 0].tolist())
+
+
+def check_two_stage_all_frames_is_one_stage(o):
+    """Keeping every frame makes every block a candidate: the one-stage selection."""
+    rng = np.random.default_rng(21)
+    Q = rng.standard_normal((1, 2, 70, 8))
+    K = rng.standard_normal((1, 2, 333, 8))
+    block, T = 16, 50
+    W = -(-333 // T)
+    for r in (1, 5, 21):
+        idx2, _, _, _ = o.select_blocks_two_stage(Q, K, block, r, T, W)
+        idx1, _ = o.select_blocks(Q, K, block, r)
+        assert np.array_equal(idx1, idx2), f"r={r}"
+
+
+def check_two_stage_frames_are_blocks(o):
+    """With frames of one block each and r frames kept, the frames are the top-r blocks."""
+    rng = np.random.default_rng(22)
+    Q = rng.standard_normal((1, 1, 64, 4))
+    K = rng.standard_normal((1, 1, 200, 4))
+    block, r = 16, 4
+    idx2, frames, _, _ = o.select_blocks_two_stage(Q, K, block, r, block, r)
+    idx1, _ = o.select_blocks(Q, K, block, r)
+    assert np.array_equal(idx1, idx2)
+    assert np.array_equal(frames, idx1)
+
+
+def _two_stage_brute(q_tokens, k_tokens, block, T, n_frames, r):
+    """Independent statement with python lists and sets: integer-valued inputs, exact means."""
+    qm = [sum(col) / len(q_tokens) for col in zip(*q_tokens)]
+    Nk = len(k_tokens)
+    frames = [list(range(w * T, min((w + 1) * T, Nk))) for w in range(-(-Nk // T))]
+    blocks = [list(range(J * block, min((J + 1) * block, Nk))) for J in range(-(-Nk // block))]
+    mean = lambda toks: [sum(k_tokens[t][c] for t in toks) / len(toks) for c in range(len(qm))]  # noqa: E731
+    dot = lambda a, b: sum(x * y for x, y in zip(a, b))  # noqa: E731
+    fs = [dot(qm, mean(fr)) for fr in frames]
+    kept = sorted(sorted(range(len(frames)), key=lambda w: (-fs[w], w))[:n_frames])
+    kept_tokens = set(t for w in kept for t in frames[w])
+    cand = [J for J, toks in enumerate(blocks) if kept_tokens.intersection(toks)]
+    bs = {J: dot(qm, mean(blocks[J])) for J in range(len(blocks))}
+    ranked = sorted(cand, key=lambda J: (-bs[J], J))
+    others = sorted((J for J in range(len(blocks)) if J not in cand), key=lambda J: (-bs[J], J))
+    return kept, sorted((ranked + others)[:r])
+
+
+def check_two_stage_bruteforce(o):
+    rng = np.random.default_rng(23)
+    for trial in range(12):
+        d = int(rng.integers(1, 4))
+        block = int(rng.integers(2, 6))
+        T = int(rng.integers(block, 3 * block + 2))
+        Nk = int(rng.integers(2 * T, 5 * T))
+        Nq = int(rng.integers(1, 2 * block + 1))
+        Q = rng.integers(-2, 3, size=(1, 1, Nq, d)).astype(np.float64)
+        K = rng.integers(-2, 3, size=(1, 1, Nk, d)).astype(np.float64)
+        W = -(-Nk // T)
+        n_frames = int(rng.integers(1, W + 1))
+        r = int(rng.integers(1, -(-Nk // block) + 1))  # may exceed the candidates: filled
+        idx, frames, _, _ = o.select_blocks_two_stage(Q, K, block, r, T, n_frames)
+        for I in range(-(-Nq // block)):
+            qt = Q[0, 0, I * block:min((I + 1) * block, Nq)].tolist()
+            kept, want = _two_stage_brute(qt, K[0, 0].tolist(), block, T, n_frames, r)
+            assert frames[0, 0, I].tolist() == kept, (trial, I, frames[0, 0, I].tolist(), kept)
+            assert idx[0, 0, I].tolist() == want, (trial, I, idx[0, 0, I].tolist(), want)
+
+
 ALL_CHECKS = [
     check_phi_library, check_pool_by_hand, check_selection_golden, check_selection_bruteforce,
     check_selection_ties_constructed, check_selection_output_form, check_attention_golden,
     check_attention_dense_equivalence, check_attention_subset_library,
     check_attention_identical_keys, check_absorb_readout_golden,
     check_absorb_incremental_equals_batch, check_absorb_single_token,
-    check_readout_closed_forms, check_hybrid_sum,
+    check_readout_closed_forms, check_hybrid_sum, check_two_stage_golden,
+    check_two_stage_all_frames_is_one_stage, check_two_stage_frames_are_blocks,
+    check_two_stage_bruteforce,
 ]

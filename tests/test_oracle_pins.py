@@ -122,11 +122,68 @@ def _mut_hybrid_difference(m):
     m.hybrid_attention = f
 
 
+def _mut_two_stage_inside_only(m):
+    def f(kept_frames, Nk, block, tokens_per_frame):
+        frames = m.frame_ranges(Nk, tokens_per_frame)
+        return np.asarray([J for J, (lo, hi) in enumerate(m.block_ranges(Nk, block))
+                           if any(frames[int(w)][0] <= lo and hi <= frames[int(w)][1] for w in kept_frames)],
+                          dtype=np.int64)
+    m.candidate_blocks = f
+
+
+def _mut_two_stage_ignore_frames(m):
+    m.candidate_blocks = lambda kept, Nk, block, T: np.arange(-(-Nk // block))
+
+
+def _mut_pool_frames_sum(m):
+    def f(K, T):
+        K = np.asarray(K, float)
+        B, H, N, d = K.shape
+        return np.stack([K[:, :, lo:hi].sum(axis=2) for lo, hi in m.frame_ranges(N, T)], axis=2)
+    m.pool_frames = f
+
+
+def _mut_two_stage_frame_ties_high(m):
+    def f(Q, K, block, r, T, n_frames):
+        # frame ranking with equal scores broken towards the higher frame index
+        fs = m.frame_scores(Q, K, block, T)
+        s = m.block_scores(Q, K, block)
+        B, H, nQB, nKB = s.shape
+        W = fs.shape[-1]
+        idx = np.empty((B, H, nQB, r), dtype=np.int32)
+        frames = np.empty((B, H, nQB, n_frames), dtype=np.int32)
+        for b in range(B):
+            for h in range(H):
+                for I in range(nQB):
+                    kept = np.sort(np.lexsort((-np.arange(W), -fs[b, h, I]))[:n_frames])
+                    frames[b, h, I] = kept
+                    is_cand = np.zeros(nKB, dtype=bool)
+                    is_cand[m.candidate_blocks(kept, np.asarray(K).shape[2], block, T)] = True
+                    idx[b, h, I] = np.sort(np.lexsort((np.arange(nKB), -s[b, h, I], ~is_cand))[:r])
+        return idx, frames, s, fs
+    m.select_blocks_two_stage = f
+
+
+def _mut_two_stage_no_fill(m):
+    orig = m.select_blocks_two_stage
+
+    def f(Q, K, block, r, T, n_frames):
+        idx, frames, s, fs = orig(Q, K, block, r, T, n_frames)
+        Nk = np.asarray(K).shape[2]
+        for b, h, I in np.ndindex(*idx.shape[:3]):
+            cand = set(m.candidate_blocks(frames[b, h, I], Nk, block, T).tolist())
+            keep = [J for J in idx[b, h, I].tolist() if J in cand]
+            idx[b, h, I] = np.asarray((keep + [keep[-1]] * r)[:r])  # short lists padded
+        return idx, frames, s, fs
+    m.select_blocks_two_stage = f
+
+
 MUTANTS = [
     _mut_phi_no_plus_one, _mut_phi_exp, _mut_readout_no_eps, _mut_readout_transposed,
     _mut_readout_no_phi_q, _mut_select_ties_high, _mut_select_bottom, _mut_pool_sum,
     _mut_attention_no_scale, _mut_attention_sqrt_d, _mut_attention_all_keys,
-    _mut_absorb_transposed, _mut_absorb_z_raw, _mut_hybrid_difference,
+    _mut_absorb_transposed, _mut_absorb_z_raw, _mut_hybrid_difference, _mut_two_stage_inside_only,
+    _mut_two_stage_ignore_frames, _mut_pool_frames_sum, _mut_two_stage_frame_ties_high, _mut_two_stage_no_fill,
 ]
 
 
