@@ -48,6 +48,9 @@ LAUNCHES_PER_STEP = 5  # pool, score+select, hybrid attention, absorb partials, 
 # (`ncu --set full --clock-control none -k regex:hybrid_attn -s 2 -c 1 ... bench.py
 # --steps 2 --warmup 3 --no-cpu-baseline`). Reset to None whenever the kernel changes.
 ATTN_TRAFFIC_BYTES = 161.3e6 + 12.8e6
+# frames kept per query block by the two-stage selection leg (8 of the window's 21 frames:
+# at least 12 blocks each, so the 64 kept blocks always come from the kept frames)
+TWO_STAGE_FRAMES = 8
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -348,7 +351,27 @@ def run_gpu(args, wl) -> None:
     t_step_local = sum(e[0].elapsed_time(e[3]) for e in events) * 1e-3 / args.steps
     t_step = max_over_ranks(t_step_local, dist, dev)
 
-    log(f"timed: {t_step_local * 1e3:.3f} ms/step; end-to-end leg")
+    log(f"timed: {t_step_local * 1e3:.3f} ms/step; two-stage selection leg")
+    # ---- two-stage (frame, then block) selection, timed alone beside the step
+    ws_sel2 = torch.empty(hf.hf_workspace_size(hf.HF_WS_SELECT_TWO_STAGE, wl.B, wl.H, wl.Nq, wl.Nk, wl.d, wl.block,
+                                               wl.r), dtype=torch.uint8, device=dev)
+    idx2 = torch.empty_like(idx)
+    t_sel2 = []
+    n_sel2 = max(3, min(args.steps, 50))
+    for k in range(n_sel2 + 3):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        hf.hf_select_blocks_two_stage(Q, K, wl.block, wl.r, wl.tokens_per_frame, TWO_STAGE_FRAMES, idx_out=idx2,
+                                      ws=ws_sel2)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        if k >= 3:
+            t_sel2.append(e0.elapsed_time(e1) * 1e-3)
+    rc, word = hf.hf_query_status()
+    if rc != hf.HF_OK:
+        raise RuntimeError(f"device status after the two-stage leg: {hf.hf_status_string(rc)} ({word:#x})")
+    log("end-to-end leg")
     # ---- end to end through the public API with host buffers (pinned), copies timed
     host = {k: v.cpu().pin_memory() for k, v in x.items()}
     O_host = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
@@ -407,6 +430,11 @@ def run_gpu(args, wl) -> None:
             "hf_select_blocks": {"us": sel_mean * 1e6, "bytes": select_bytes(wl),
                                  "gbs": select_bytes(wl) / sel_mean / 1e9,
                                  "hbm_frac": select_bytes(wl) / sel_mean / 1e9 / peaks["hbm_gbs"]},
+            "hf_select_blocks_two_stage": {"us": statistics.mean(t_sel2) * 1e6, "n_frames": TWO_STAGE_FRAMES,
+                                           "bytes": select_bytes(wl),
+                                           "gbs": select_bytes(wl) / statistics.mean(t_sel2) / 1e9,
+                                           "hbm_frac": select_bytes(wl) / statistics.mean(t_sel2) / 1e9
+                                           / peaks["hbm_gbs"]},
             "hf_absorb_evicted_step": {"us": abs_mean * 1e6, "tokens": wl.Ne_step,
                                        "bytes": absorb_bytes(wl, wl.Ne_step),
                                        "gbs": absorb_bytes(wl, wl.Ne_step) / abs_mean / 1e9},

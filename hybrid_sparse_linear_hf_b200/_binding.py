@@ -25,6 +25,7 @@ HF_ERR_DEVICE_BAD_INDEX = 7
 HF_WS_SELECT = 1
 HF_WS_ATTN = 2
 HF_WS_ABSORB = 3
+HF_WS_SELECT_TWO_STAGE = 4
 
 _SIZE_T_MAX = (1 << (8 * ctypes.sizeof(ctypes.c_size_t))) - 1
 
@@ -52,6 +53,8 @@ _SIGNATURES = {
                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "hf_select_blocks": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 +
                          [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_select_blocks_two_stage": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 9 +
+                                   [ctypes.c_void_p] * 4 + [ctypes.c_size_t, ctypes.c_void_p]),
     "hf_select_blocks_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 +
                                  [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "hf_hybrid_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
@@ -187,6 +190,27 @@ def hf_select_blocks(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, idx_o
                                   _dev(scores_out, torch.float32, "scores_out") if scores_out is not None else None,
                                   ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
            "hf_select_blocks")
+    return idx_out
+
+
+def hf_select_blocks_two_stage(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, tokens_per_frame: int,
+                               n_frames: int, idx_out=None, frames_out=None, scores_out=None, ws=None,
+                               stream=None) -> torch.Tensor:
+    """Two-stage top-r key blocks per query block (frames, then blocks within them):
+    int32 [B,H,nQB,r] (ascending). frames_out: optional int32 [B,H,nQB,n_frames]."""
+    B, H, Nq, d = Q.shape
+    Nk = K.shape[2]
+    nQB = -(-Nq // block)
+    if idx_out is None:
+        idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
+    nbytes = hf_workspace_size(HF_WS_SELECT_TWO_STAGE, B, H, Nq, Nk, d, block, r)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    _check(lib().hf_select_blocks_two_stage(
+        _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), B, H, Nq, Nk, d, block, r, tokens_per_frame,
+        n_frames, _dev(idx_out, torch.int32, "idx_out"),
+        _dev(frames_out, torch.int32, "frames_out") if frames_out is not None else None,
+        _dev(scores_out, torch.float32, "scores_out") if scores_out is not None else None,
+        ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)), "hf_select_blocks_two_stage")
     return idx_out
 
 

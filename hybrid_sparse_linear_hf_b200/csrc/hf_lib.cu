@@ -117,6 +117,46 @@ hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int 
   return launch_status();
 }
 
+// ---------------------------------------------------------------- two-stage select
+// Workspace: pooled Q, pooled K, the key blocks' frame parts and the frame means (fp32);
+// W <= nKB because tokens_per_frame >= block.
+size_t select2_ws_bytes(int B, int H, int Nq, int Nk, int d, int block) {
+  const long long bh = static_cast<long long>(B) * H;
+  const size_t nKB = ceil_div(Nk, block);
+  return align256(static_cast<size_t>(bh) * ceil_div(Nq, block) * d * 4) + align256(bh * nKB * d * 4) +
+         align256(bh * nKB * 2 * d * 4) + align256(bh * nKB * d * 4);
+}
+
+template <int D>
+hf_status launch_select2(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk, int block, int r, int T, int nf,
+                         int32_t* idx, int32_t* frames, float* scores, void* ws, cudaStream_t st) {
+  const int nQB = ceil_div(Nq, block), nKB = ceil_div(Nk, block), W = ceil_div(Nk, T);
+  char* base = static_cast<char*>(ws);
+  float* Qp = reinterpret_cast<float*>(base);
+  base += align256(static_cast<size_t>(BH) * nQB * D * 4);
+  float* Kp = reinterpret_cast<float*>(base);
+  base += align256(static_cast<size_t>(BH) * nKB * D * 4);
+  float* Kpart = reinterpret_cast<float*>(base);
+  base += align256(static_cast<size_t>(BH) * nKB * 2 * D * 4);
+  float* Kf = reinterpret_cast<float*>(base);
+  const long long grid1 = static_cast<long long>(BH) * (nQB + nKB);
+  hf::pool_blocks_kernel<D, true><<<static_cast<unsigned>(grid1), hf::kPoolThreads, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block, nQB,
+      nKB, Qp, Kp, T, Kpart);
+  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  hf::pool_frames_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * W), D, 0, st>>>(Kpart, Nk, block, T,
+                                                                                                nKB, W, Kf);
+  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  const size_t smem = static_cast<size_t>(hf::kSelQB) * (nKB + W) * (sizeof(float) + 1);
+  if (cudaFuncSetAttribute(hf::score_select2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return HF_ERR_CUDA;
+  const long long groups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
+  hf::score_select2_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * groups), hf::kSelectThreads, smem,
+                                st>>>(Qp, Kp, Kf, nQB, nKB, W, Nk, block, T, r, nf, idx, frames, scores);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------- absorb
 struct AbsorbPlan {
   int tiles_per_split, nsplit;
@@ -276,6 +316,10 @@ HF_API size_t hf_workspace_size(int which, int B, int H, int Nq, int Nk, int d, 
       if (Nk < 0) return static_cast<size_t>(-1);
       if (Nk == 0) return 0;
       return absorb_ws_bytes(B, H, Nk, d);
+    case HF_WS_SELECT_TWO_STAGE:
+      if (!supported_block(block) || Nq < 0 || Nk < 1 || r < 1 || r > ceil_div(Nk, block))
+        return static_cast<size_t>(-1);
+      return select2_ws_bytes(B, H, Nq, Nk, d, block);
   }
   return static_cast<size_t>(-1);
 }
@@ -333,6 +377,32 @@ HF_API hf_status hf_select_blocks(const hf_bf16* Q, const hf_bf16* K, int B, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_select<128>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s)
                   : launch_select<64>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s);
+}
+
+HF_API hf_status hf_select_blocks_two_stage(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk,
+                                            int d, int block, int r, int tokens_per_frame, int n_frames,
+                                            int32_t* idx_out, int32_t* frames_out, float* scores_out, void* ws,
+                                            size_t ws_bytes, void* stream) {
+  if (B < 1 || H < 1 || Nq < 0 || Nk < 1) return HF_ERR_INVALID_ARG;
+  if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
+  if (tokens_per_frame < block) return HF_ERR_INVALID_ARG;
+  const int nKB = ceil_div(Nk, block), W = ceil_div(Nk, tokens_per_frame);
+  if (r < 1 || r > nKB || n_frames < 1 || n_frames > W) return HF_ERR_INVALID_ARG;
+  if (nKB > hf::kMaxKeyBlocks2) return HF_ERR_UNSUPPORTED;
+  if (Nq == 0) return HF_OK;
+  if (!Q || !K || !idx_out) return HF_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(idx_out) || (frames_out && !aligned16(frames_out)) ||
+      (scores_out && !aligned16(scores_out)))
+    return HF_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < select2_ws_bytes(B, H, Nq, Nk, d, block)) return HF_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_select2<128>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, tokens_per_frame, n_frames,
+                                        idx_out, frames_out, scores_out, ws, s)
+                  : launch_select2<64>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, tokens_per_frame, n_frames,
+                                       idx_out, frames_out, scores_out, ws, s);
 }
 
 HF_API hf_status hf_hybrid_attn_fwd(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H, int Nq,

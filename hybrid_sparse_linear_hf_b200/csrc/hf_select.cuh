@@ -48,21 +48,28 @@ __device__ __forceinline__ uint4 ld_stream_16(const void* p) {
 }
 
 // Qp[bh][I][:] = mean of Q rows of block I; Kp[bh][J][:] likewise.
-template <int D>
+// kParts (two-stage selection): also Kpart[bh][J][0|1][:] = the sums of the rows of key
+// block J that lie in its first frame (J*block / T) and in the next frame (zero when the
+// block does not reach it); frames are runs of T >= block tokens, so a block touches at
+// most two. The block means are computed exactly as without kParts.
+template <int D, bool kParts = false>
 __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bfloat16* __restrict__ Q,
                                                                    const __nv_bfloat16* __restrict__ K,
                                                                    int Nq, int Nk, int block, int nQB, int nKB,
                                                                    float* __restrict__ Qp,
-                                                                   float* __restrict__ Kp) {
+                                                                   float* __restrict__ Kp,
+                                                                   int T = 0, float* __restrict__ Kpart = nullptr) {
   constexpr int kVec = 8;                       // bf16 per 16-byte load
   constexpr int kTpr = D / kVec;                // threads per row
   constexpr int kRows = kPoolThreads / kTpr;    // rows per pass
   constexpr int kUnroll = 8;                    // loads in flight per thread
   __shared__ float red[kRows * D];
+  __shared__ float red1[kParts ? kRows * D : 1];
 
   const int per_bh = nQB + nKB;
   const int bh = blockIdx.x / per_bh;
   int t = blockIdx.x % per_bh;
+  const bool is_key_block = t >= nQB;
   const __nv_bfloat16* X;
   int N;
   float* out;
@@ -80,8 +87,12 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bf
   const int hi = min(lo + block, N);
   const int c = threadIdx.x % kTpr;
   const int rr = threadIdx.x / kTpr;
+  // first row of the next frame, if this key block reaches it (kParts only)
+  const bool parts = kParts && is_key_block;
+  const int bnd = parts ? min(hi, (lo / T + 1) * T) : hi;
 
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float acc1[kParts ? 8 : 1] = {0.f};
   for (int base = lo + rr; base < hi; base += kRows * kUnroll) {
     uint4 v[kUnroll];
 #pragma unroll
@@ -90,17 +101,54 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bf
       v[u] = row < hi ? ld_stream_16(X + static_cast<size_t>(row) * D + c * kVec) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) acc_bf16x8(acc, v[u]);
+    for (int u = 0; u < kUnroll; ++u) {
+      acc_bf16x8(acc, v[u]);
+      if constexpr (kParts) {
+        if (base + u * kRows >= bnd) acc_bf16x8(acc1, v[u]);
+      }
+    }
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) red[rr * D + c * kVec + k] = acc[k];
+  if constexpr (kParts) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) red1[rr * D + c * kVec + k] = acc1[k];
+  }
   __syncthreads();
   if (threadIdx.x < D) {
     float s = 0.f;
 #pragma unroll 8
     for (int q = 0; q < kRows; ++q) s += red[q * D + threadIdx.x];
     out[threadIdx.x] = s / static_cast<float>(hi - lo);
+    if constexpr (kParts) {
+      if (parts) {
+        float s1 = 0.f;
+#pragma unroll 8
+        for (int q = 0; q < kRows; ++q) s1 += red1[q * D + threadIdx.x];
+        float* pt = Kpart + ((static_cast<size_t>(bh) * nKB + t) * 2) * D;
+        pt[threadIdx.x] = s - s1;
+        pt[D + threadIdx.x] = s1;
+      }
+    }
   }
+}
+
+// Kf[bh][w][:] = mean of the key rows of frame w (rows [w*T, min((w+1)*T, Nk))), summed
+// from the block parts in block order (deterministic). One CTA per (bh, w), D threads.
+template <int D>
+__global__ void __launch_bounds__(D) pool_frames_kernel(const float* __restrict__ Kpart, int Nk, int block, int T,
+                                                        int nKB, int W, float* __restrict__ Kf) {
+  const int bh = blockIdx.x / W, w = blockIdx.x % W;
+  const int f_lo = w * T, f_hi = min(f_lo + T, Nk);
+  const int J_lo = f_lo / block, J_hi = (f_hi - 1) / block;
+  const float* P = Kpart + static_cast<size_t>(bh) * nKB * 2 * D;
+  float s = 0.f;
+  for (int J = J_lo; J <= J_hi; ++J) {
+    // block J starts in frame w (its first part) or in frame w-1 and reaches w (second)
+    const int part = (J * block) / T == w ? 0 : 1;
+    s += P[(static_cast<size_t>(J) * 2 + part) * D + threadIdx.x];
+  }
+  Kf[(static_cast<size_t>(bh) * W + w) * D + threadIdx.x] = s / static_cast<float>(f_hi - f_lo);
 }
 
 // Scores of kSelQB query blocks of one head per CTA (each pooled K row is read once for
@@ -113,33 +161,31 @@ __device__ __forceinline__ uint32_t ordered_bits(float f) {
   return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Top-r of the scores srow[0..nKB) (larger score first, lower J first on ties), written
-// to out[0..r) in ascending J by one warp. NPL = ordered scores per lane held in registers
-// (lane l holds J = 32 k + l); NPL = 0 reads shared memory each time (any nKB).
-// 1. T = the r-th largest ordered score: the largest t with #{J : o_J >= t} >= r, found
-//    bit by bit from the top, each candidate counted per lane and summed over the warp.
-// 2. Keep every J with o_J > T, and the (r - #{o_J > T}) lowest J with o_J == T.
-template <int NPL>
-__device__ __forceinline__ void warp_top_r(const float* srow, int nKB, int r, int lane, int32_t* out) {
-  auto ob_at = [&](int J) -> uint32_t {
-    const float v = srow[J];
-    // NaN ranks last; -0 and +0 are one value (a tie, broken by J)
-    return ordered_bits(v != v ? -INFINITY : (v == 0.f ? 0.f : v));
-  };
+// Warp-wide top-r over n unique keys key_at(J) (J < n): larger key first, lower J first on
+// ties; emit(J, pos) is called for the r selected J in ascending J (pos = 0..r-1). Keys
+// are order-preserving 32-bit codes; a key of 0 ranks below every real score code
+// (ordered(-inf) = 0x007FFFFF), so it is chosen only when fewer than r keys are nonzero.
+// NPL = keys per lane held in registers (lane l holds J = 32 k + l); NPL = 0 calls key_at
+// each time (any n).
+// 1. T = the r-th largest key: the largest t with #{J : key_J >= t} >= r, found bit by
+//    bit from the top, each candidate counted per lane and summed over the warp.
+// 2. Keep every J with key_J > T, and the (r - #{key_J > T}) lowest J with key_J == T.
+template <int NPL, class KeyF, class EmitF>
+__device__ __forceinline__ void warp_top_r(int n, int r, int lane, KeyF key_at, EmitF emit) {
   constexpr int kRegs = NPL > 0 ? NPL : 1;
   uint32_t o[kRegs];
   if constexpr (NPL > 0) {
 #pragma unroll
-    for (int k = 0; k < NPL; ++k) o[k] = (32 * k + lane < nKB) ? ob_at(32 * k + lane) : 0u;
+    for (int k = 0; k < NPL; ++k) o[k] = (32 * k + lane < n) ? key_at(32 * k + lane) : 0u;
   }
-  // Lanes past nKB are excluded from every count (their register holds 0).
+  // Lanes past n are excluded from every count.
   auto count_ge = [&](uint32_t t) -> int {
     int c = 0;
     if constexpr (NPL > 0) {
 #pragma unroll
-      for (int k = 0; k < NPL; ++k) c += (32 * k + lane < nKB && o[k] >= t) ? 1 : 0;
+      for (int k = 0; k < NPL; ++k) c += (32 * k + lane < n && o[k] >= t) ? 1 : 0;
     } else {
-      for (int J = lane; J < nKB; J += 32) c += ob_at(J) >= t ? 1 : 0;
+      for (int J = lane; J < n; J += 32) c += key_at(J) >= t ? 1 : 0;
     }
     return static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(c)));
   };
@@ -153,7 +199,7 @@ __device__ __forceinline__ void warp_top_r(const float* srow, int nKB, int r, in
   const int n_eq_keep = r - n_gt;  // >= 1
   int base = 0, eq_seen = 0;
   const uint32_t lt_mask = (1u << lane) - 1u;
-  for (int k = 0; 32 * k < nKB; ++k) {
+  for (int k = 0; 32 * k < n; ++k) {
     const int J = 32 * k + lane;
     uint32_t oj = 0;
     if constexpr (NPL > 0) {
@@ -161,17 +207,66 @@ __device__ __forceinline__ void warp_top_r(const float* srow, int nKB, int r, in
       for (int kk = 0; kk < NPL; ++kk)
         if (kk == k) oj = o[kk];
     } else {
-      oj = J < nKB ? ob_at(J) : 0u;
+      oj = J < n ? key_at(J) : 0u;
     }
-    const bool valid = J < nKB;
+    const bool valid = J < n;
     const bool eq = valid && oj == T;
     const uint32_t m_eq = __ballot_sync(0xffffffffu, eq);
     const bool keep = valid && (oj > T || (eq && eq_seen + __popc(m_eq & lt_mask) < n_eq_keep));
     const uint32_t m = __ballot_sync(0xffffffffu, keep);
-    const int pos = base + __popc(m & lt_mask);
-    if (keep) out[pos] = J;
+    if (keep) emit(J, base + __popc(m & lt_mask));
     base += __popc(m);
     eq_seen += __popc(m_eq);
+  }
+}
+
+// Selection key of a score: NaN ranks last; -0 and +0 are one value (a tie, broken by J).
+__device__ __forceinline__ uint32_t score_key(float v) {
+  return ordered_bits(v != v ? -INFINITY : (v == 0.f ? 0.f : v));
+}
+
+// Top-r of the scores srow[0..nKB) written to out[0..r) in ascending J by one warp.
+__device__ __forceinline__ void warp_top_r_scores(const float* srow, int nKB, int r, int lane, int32_t* out) {
+  auto key = [&](int J) { return score_key(srow[J]); };
+  auto emit = [&](int J, int pos) { out[pos] = J; };
+  if (nKB <= 256) {
+    warp_top_r<8>(nKB, r, lane, key, emit);
+  } else if (nKB <= 512) {
+    warp_top_r<16>(nKB, r, lane, key, emit);
+  } else {
+    warp_top_r<0>(nKB, r, lane, key, emit);
+  }
+}
+
+// out[g * n + J] = q_sh[g] . rows[J] for the kSelQB query rows in shared memory and n fp32
+// rows of D: a thread per row J, the row read with 16-byte loads, 8 in flight.
+template <int D>
+__device__ __forceinline__ void score_rows(const float (*q_sh)[D], const float* __restrict__ rows, int n,
+                                           float* out) {
+  for (int J = threadIdx.x; J < n; J += kSelectThreads) {
+    const float4* krow = reinterpret_cast<const float4*>(rows + static_cast<size_t>(J) * D);
+    float acc[kSelQB];
+#pragma unroll
+    for (int g = 0; g < kSelQB; ++g) acc[g] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < D / 4; k0 += 8) {
+      float4 kv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) kv[u] = __ldg(krow + k0 + u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+#pragma unroll
+        for (int g = 0; g < kSelQB; ++g) {
+          const float4 qv = *reinterpret_cast<const float4*>(&q_sh[g][4 * (k0 + u)]);
+          acc[g] = fmaf(qv.x, kv[u].x, acc[g]);
+          acc[g] = fmaf(qv.y, kv[u].y, acc[g]);
+          acc[g] = fmaf(qv.z, kv[u].z, acc[g]);
+          acc[g] = fmaf(qv.w, kv[u].w, acc[g]);
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kSelQB; ++g) out[g * n + J] = acc[g];
   }
 }
 
@@ -198,32 +293,7 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const floa
     q_sh[g][i % D] = Qp[(static_cast<size_t>(bh) * nQB + I0 + min(g, G - 1)) * D + i % D];
   }
   __syncthreads();
-  const float* kbase = Kp + static_cast<size_t>(bh) * nKB * D;
-  for (int J = threadIdx.x; J < nKB; J += kSelectThreads) {
-    const float4* krow = reinterpret_cast<const float4*>(kbase + static_cast<size_t>(J) * D);
-    float acc[kSelQB];
-#pragma unroll
-    for (int g = 0; g < kSelQB; ++g) acc[g] = 0.f;
-#pragma unroll
-    for (int k0 = 0; k0 < D / 4; k0 += 8) {
-      float4 kv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) kv[u] = __ldg(krow + k0 + u);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-#pragma unroll
-        for (int g = 0; g < kSelQB; ++g) {
-          const float4 qv = *reinterpret_cast<const float4*>(&q_sh[g][4 * (k0 + u)]);
-          acc[g] = fmaf(qv.x, kv[u].x, acc[g]);
-          acc[g] = fmaf(qv.y, kv[u].y, acc[g]);
-          acc[g] = fmaf(qv.z, kv[u].z, acc[g]);
-          acc[g] = fmaf(qv.w, kv[u].w, acc[g]);
-        }
-      }
-    }
-#pragma unroll
-    for (int g = 0; g < kSelQB; ++g) s_sc[g * nKB + J] = acc[g];
-  }
+  score_rows<D>(q_sh, Kp + static_cast<size_t>(bh) * nKB * D, nKB, s_sc);
   __syncthreads();
 
   if (warp < G) {
@@ -232,13 +302,111 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const floa
     float* sout = scores_out ? scores_out + (static_cast<size_t>(bh) * nQB + I) * nKB : nullptr;
     if (sout)
       for (int J = lane; J < nKB; J += 32) sout[J] = srow[J];
-    int32_t* out = idx_out + (static_cast<size_t>(bh) * nQB + I) * r;
-    if (nKB <= 256) {
-      warp_top_r<8>(srow, nKB, r, lane, out);
-    } else if (nKB <= 512) {
-      warp_top_r<16>(srow, nKB, r, lane, out);
+    warp_top_r_scores(srow, nKB, r, lane, idx_out + (static_cast<size_t>(bh) * nQB + I) * r);
+  }
+}
+
+// ------------------------------------------------------------ two-stage selection
+constexpr int kMaxKeyBlocks2 = 4096;  // block and frame scores of 4 query blocks in shared memory
+
+template <int NPLMAX, class KeyF, class EmitF>
+__device__ __forceinline__ void warp_top_r_dispatch(int n, int r, int lane, KeyF key, EmitF emit) {
+  if (n <= 256) {
+    warp_top_r<8>(n, r, lane, key, emit);
+  } else if (NPLMAX >= 16 && n <= 512) {
+    warp_top_r<16>(n, r, lane, key, emit);
+  } else {
+    warp_top_r<0>(n, r, lane, key, emit);
+  }
+}
+
+// Source: "Light Forcing: Accelerating Autoregressive Video Diffusion via Sparse
+// Attention", German technical summary, section 2.2 (two-stage mask selection: for each
+// query block a small set of frames by the frame-level compressed keys, then the blocks
+// within those frames by the block-level compressed keys).
+// One CTA per (b, h, 4 query blocks): block scores s and frame scores f (a thread per
+// row), then one warp per query block: the nf frames of largest f (ties to the lower
+// frame; frames_out, ascending), candidate blocks = blocks with a token in a kept frame,
+// and the r candidates of largest s (ties to the lower J) in ascending J. With fewer than
+// r candidates every candidate is kept and the rest are the best other blocks.
+// Dynamic shared memory: s[4][nKB], f[4][W] (fp32), kept[4][W], sel[4][nKB] (bytes).
+template <int D>
+__global__ void __launch_bounds__(kSelectThreads) score_select2_kernel(
+    const float* __restrict__ Qp, const float* __restrict__ Kp, const float* __restrict__ Kf, int nQB, int nKB,
+    int W, int Nk, int block, int T, int r, int nf, int32_t* __restrict__ idx_out, int32_t* __restrict__ frames_out,
+    float* __restrict__ scores_out) {
+  extern __shared__ float dsm[];
+  float* s_sc = dsm;
+  float* f_sc = s_sc + kSelQB * nKB;
+  uint8_t* kept = reinterpret_cast<uint8_t*>(f_sc + kSelQB * W);
+  uint8_t* sel = kept + kSelQB * W;
+  __shared__ __align__(16) float q_sh[kSelQB][D];
+  const int groups = (nQB + kSelQB - 1) / kSelQB;
+  const int bh = blockIdx.x / groups;
+  const int I0 = (blockIdx.x % groups) * kSelQB;
+  const int G = min(kSelQB, nQB - I0);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  for (int i = threadIdx.x; i < kSelQB * D; i += kSelectThreads) {
+    const int g = i / D;
+    q_sh[g][i % D] = Qp[(static_cast<size_t>(bh) * nQB + I0 + min(g, G - 1)) * D + i % D];
+  }
+  __syncthreads();
+  score_rows<D>(q_sh, Kp + static_cast<size_t>(bh) * nKB * D, nKB, s_sc);
+  score_rows<D>(q_sh, Kf + static_cast<size_t>(bh) * W * D, W, f_sc);
+  __syncthreads();
+
+  if (warp < G) {
+    const int I = I0 + warp;
+    const size_t q = static_cast<size_t>(bh) * nQB + I;
+    const float* srow = s_sc + warp * nKB;
+    const float* frow = f_sc + warp * W;
+    uint8_t* krow = kept + warp * W;
+    uint8_t* selrow = sel + warp * nKB;
+    if (scores_out)
+      for (int J = lane; J < nKB; J += 32) scores_out[q * nKB + J] = srow[J];
+    for (int w = lane; w < W; w += 32) krow[w] = 0;
+    __syncwarp();
+    // stage 1: the nf frames of largest score
+    int32_t* fout = frames_out ? frames_out + q * nf : nullptr;
+    warp_top_r_dispatch<8>(
+        W, nf, lane, [&](int w) { return score_key(frow[w]); },
+        [&](int w, int pos) {
+          krow[w] = 1;
+          if (fout) fout[pos] = w;
+        });
+    __syncwarp();
+    // stage 2: candidate blocks (a token in a kept frame; a block touches at most 2 frames)
+    auto is_cand = [&](int J) -> bool {
+      const int f_lo = (J * block) / T;
+      const int f_hi = (min((J + 1) * block, Nk) - 1) / T;
+      return (krow[f_lo] | krow[f_hi]) != 0;
+    };
+    int nc = 0;
+    for (int J = lane; J < nKB; J += 32) nc += is_cand(J) ? 1 : 0;
+    nc = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<unsigned>(nc)));
+    int32_t* out = idx_out + q * r;
+    if (nc >= r) {
+      warp_top_r_dispatch<16>(
+          nKB, r, lane, [&](int J) { return is_cand(J) ? score_key(srow[J]) : 0u; },
+          [&](int J, int pos) { out[pos] = J; });
     } else {
-      warp_top_r<0>(srow, nKB, r, lane, out);
+      // every candidate, then the best r - nc other blocks; written in ascending J
+      for (int J = lane; J < nKB; J += 32) selrow[J] = is_cand(J) ? 1 : 0;
+      __syncwarp();
+      warp_top_r_dispatch<16>(
+          nKB, r - nc, lane, [&](int J) { return is_cand(J) ? 0u : score_key(srow[J]); },
+          [&](int J, int) { selrow[J] = 1; });
+      __syncwarp();
+      int base = 0;
+      const uint32_t lt_mask = (1u << lane) - 1u;
+      for (int J0 = 0; J0 < nKB; J0 += 32) {
+        const int J = J0 + lane;
+        const bool keep = J < nKB && selrow[J] != 0;
+        const uint32_t m = __ballot_sync(0xffffffffu, keep);
+        if (keep) out[base + __popc(m & lt_mask)] = J;
+        base += __popc(m);
+      }
     }
   }
 }

@@ -88,7 +88,7 @@ typedef struct hf_state {
 } hf_state;
 
 /* Workspace kinds for hf_workspace_size. */
-enum { HF_WS_SELECT = 1, HF_WS_ATTN = 2, HF_WS_ABSORB = 3 };
+enum { HF_WS_SELECT = 1, HF_WS_ATTN = 2, HF_WS_ABSORB = 3, HF_WS_SELECT_TWO_STAGE = 4 };
 
 /* Bytes of device workspace the call `which` needs (0 = none; NULL may be passed).
  * For HF_WS_ABSORB pass the number of evicted tokens as Nk (Nq, block, r ignored).
@@ -127,6 +127,32 @@ HF_API hf_status hf_absorb_evicted(hf_state* st, const hf_bf16* K_ev, const hf_b
 HF_API hf_status hf_select_blocks(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk, int d,
                                   int block, int r, int32_t* idx_out, float* scores_out, void* ws,
                                   size_t ws_bytes, void* stream);
+
+/* Two-stage top-r key-block selection: frames first, then blocks within the kept frames.
+ *   frames: runs of tokens_per_frame tokens of the window (the last may be partial),
+ *           W = ceil(Nk / tokens_per_frame); tokens_per_frame >= block
+ *   f[b][h][I][w] = mean(Q rows of block I) . mean(K rows of frame w)            (fp32)
+ *   frames_out[b][h][I][0..n_frames) = the n_frames frames of largest f, ties to the
+ *                                      lower w, ascending                      (int32)
+ *   candidate blocks: the key blocks with at least one token in a kept frame
+ *   idx_out[b][h][I][0..r) = the r candidates of largest score (as in hf_select_blocks),
+ *                            ties to the lower J, ascending; with fewer than r
+ *                            candidates, every candidate and then the best other
+ *                            blocks                                             (int32)
+ * Source: Light Forcing, German technical summary section 2.2 (tokens compressed by mean
+ * pooling at block and frame level; two-stage mask selection: a small set of frames by
+ * the frame-level compressed keys, then the blocks within them by the block-level ones).
+ * Q: [B][H][Nq][d], K: [B][H][Nk][d]. frames_out ([B][H][nQB][n_frames]) and scores_out
+ * ([B][H][nQB][nKB], fp32 block scores) are optional (NULL to skip). The output feeds
+ * hf_hybrid_attn_fwd like hf_select_blocks'. Nq == 0 is a no-op.
+ * ws: HF_WS_SELECT_TWO_STAGE bytes (hf_workspace_size with the same block and r).
+ * Errors: HF_ERR_INVALID_ARG (Nk < 1, r outside [1, nKB], n_frames outside [1, W],
+ * tokens_per_frame < block, NULL), HF_ERR_UNSUPPORTED (d, block, nKB > 4096),
+ * HF_ERR_ALIGNMENT, HF_ERR_WORKSPACE, HF_ERR_CUDA. */
+HF_API hf_status hf_select_blocks_two_stage(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk,
+                                            int d, int block, int r, int tokens_per_frame, int n_frames,
+                                            int32_t* idx_out, int32_t* frames_out, float* scores_out, void* ws,
+                                            size_t ws_bytes, void* stream);
 
 /* Upper bound, in bytes, of the select workspace that hf_select_blocks_noalloc can
  * serve: a call is accepted when hf_workspace_size(HF_WS_SELECT, ...) for its shapes

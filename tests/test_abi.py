@@ -134,3 +134,28 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "libhf.so"))
     with pytest.raises(ImportError):
         B.lib()
+
+
+def _sel2(**kw):
+    a = dict(Q=A, K=A, B=1, H=1, Nq=64, Nk=1000, d=64, block=32, r=4, T=100, nf=2, idx=A, frames=None, scores=None,
+             ws=A, ws_bytes=1 << 20)
+    a.update(kw)
+    return hf.lib().hf_select_blocks_two_stage(a["Q"], a["K"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], a["block"],
+                                               a["r"], a["T"], a["nf"], a["idx"], a["frames"], a["scores"], a["ws"],
+                                               a["ws_bytes"], None)
+
+
+def test_select_two_stage_validation():
+    assert _sel2(T=16) == B.HF_ERR_INVALID_ARG      # frames shorter than a block
+    assert _sel2(nf=0) == B.HF_ERR_INVALID_ARG
+    assert _sel2(nf=11) == B.HF_ERR_INVALID_ARG     # W = 10
+    assert _sel2(r=0) == B.HF_ERR_INVALID_ARG
+    assert _sel2(r=33) == B.HF_ERR_INVALID_ARG      # nKB = 32
+    assert _sel2(d=96) == B.HF_ERR_UNSUPPORTED
+    assert _sel2(Nk=4097 * 32, T=64) == B.HF_ERR_UNSUPPORTED  # nKB > 4096
+    assert _sel2(Q=None) == B.HF_ERR_INVALID_ARG
+    assert _sel2(frames=A + 4) == B.HF_ERR_ALIGNMENT
+    assert _sel2(ws_bytes=100) == B.HF_ERR_WORKSPACE
+    assert _sel2(Nq=0) == B.HF_OK
+    n = hf.hf_workspace_size(B.HF_WS_SELECT_TWO_STAGE, 1, 12, 4680, 32760, 128, 128, 64)
+    assert n == 12 * 37 * 128 * 4 + 12 * 256 * 128 * 4 * 4
