@@ -105,12 +105,12 @@ hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int 
       reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block, nQB,
       nKB, Qp, Kp);
   if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  // the opt-in covers static + dynamic shared memory above the 48 KB default; set on
+  // every launch so that no size of nKB depends on it having been set before
   const size_t smem = static_cast<size_t>(nKB) * hf::kSelQB * sizeof(float);
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(hf::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return HF_ERR_CUDA;
-  }
+  if (cudaFuncSetAttribute(hf::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return HF_ERR_CUDA;
   const long long groups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
   hf::score_select_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * groups), hf::kSelectThreads, smem,
                                st>>>(Qp, Kp, nQB, nKB, r, idx, scores);

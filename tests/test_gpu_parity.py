@@ -58,6 +58,7 @@ def _check_status():
     (1, 2, 33, 129, 128, 128, 2),      # 1-token key tail
     (1, 1, 64, 4096, 64, 32, 128),     # many key blocks
     (1, 2, 300, 2000, 128, 128, 16),   # r = nKB
+    (1, 1, 40, 131072, 128, 128, 64),  # 1024 key blocks: static + dynamic shared memory > 48 KB
 ])
 def test_select_matches_oracle(B, H, Nq, Nk, d, block, r):
     Q = _gen(1, B, H, Nq, d, w=0.5)
