@@ -92,7 +92,6 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bf
   const int bnd = parts ? min(hi, (lo / T + 1) * T) : hi;
 
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  float acc1[kParts ? 8 : 1] = {0.f};
   for (int base = lo + rr; base < hi; base += kRows * kUnroll) {
     uint4 v[kUnroll];
 #pragma unroll
@@ -101,11 +100,15 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bf
       v[u] = row < hi ? ld_stream_16(X + static_cast<size_t>(row) * D + c * kVec) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      acc_bf16x8(acc, v[u]);
-      if constexpr (kParts) {
-        if (base + u * kRows >= bnd) acc_bf16x8(acc1, v[u]);
-      }
+    for (int u = 0; u < kUnroll; ++u) acc_bf16x8(acc, v[u]);
+  }
+  // the second-frame sum, only in blocks that reach the next frame (CTA-uniform): a short
+  // second pass over those rows, just read and still in L2
+  float acc1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if constexpr (kParts) {
+    if (bnd < hi) {
+      for (int row = lo + rr; row < hi; row += kRows)
+        if (row >= bnd) acc_bf16x8(acc1, ld_stream_16(X + static_cast<size_t>(row) * D + c * kVec));
     }
   }
 #pragma unroll
