@@ -51,6 +51,8 @@ ATTN_TRAFFIC_BYTES = 161.3e6 + 12.8e6
 # frames kept per query block by the two-stage selection leg (8 of the window's 21 frames:
 # at least 12 blocks each, so the 64 kept blocks always come from the kept frames)
 TWO_STAGE_FRAMES = 8
+# keep ratios of the sparsity sweep leg (1 = dense window attention)
+SWEEP_KEEPS = (1.0, 0.5, 0.25, 0.125)
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -371,6 +373,29 @@ def run_gpu(args, wl) -> None:
     rc, word = hf.hf_query_status()
     if rc != hf.HF_OK:
         raise RuntimeError(f"device status after the two-stage leg: {hf.hf_status_string(rc)} ({word:#x})")
+    # ---- sparsity sweep: the attention alone at other keep ratios (same inputs and state)
+    log("sweep leg")
+    sweep = {}
+    for keep in SWEEP_KEEPS:
+        wk = wl.with_keep(keep)
+        idx_k = torch.empty(wl.B, wl.H, wl.nQB, wk.r, dtype=torch.int32, device=dev)
+        hf.hf_select_blocks(Q, K, wl.block, wk.r, idx_out=idx_k, ws=ws_sel)
+        ts = []
+        for k in range(12):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wk.r, idx_k, st, O=O)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if k >= 2:
+                ts.append(e0.elapsed_time(e1) * 1e-3)
+        t_k = statistics.mean(ts)
+        F_k = attn_flops(idx_k.cpu().numpy(), wk)
+        sweep[f"{keep:g}"] = {"r": wk.r, "us": t_k * 1e6, "tflops": F_k / t_k / 1e12}
+    rc, word = hf.hf_query_status()
+    if rc != hf.HF_OK:
+        raise RuntimeError(f"device status after the sweep leg: {hf.hf_status_string(rc)} ({word:#x})")
     log("end-to-end leg")
     # ---- end to end through the public API with host buffers (pinned), copies timed
     host = {k: v.cpu().pin_memory() for k, v in x.items()}
@@ -445,6 +470,7 @@ def run_gpu(args, wl) -> None:
                                               / peaks["hbm_gbs"]},
             "hbm_peak_gbs": peaks["hbm_gbs"],
         },
+        "sweep": {k: dict(v, frac=v["tflops"] / peaks["bf16_tflops"]) for k, v in sweep.items()},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
         "e2e": {"value": job_throughput(world, wl.B, wl.Nq, t_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,

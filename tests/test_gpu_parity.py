@@ -278,6 +278,45 @@ def test_streaming_300_steps():
     _check_status()
 
 
+def test_streaming_832x480_20_steps():
+    """20 chunk steps at the 832x480 shape, each evicting 3 fresh frames (4680 tokens per
+    head) into the state; at the end the state of two heads against a float64 batch
+    recompute, and one step's sampled query blocks against the oracle."""
+    wl = WORKLOADS["832x480"]
+    d = wl.d
+    S = torch.empty(wl.B, wl.H, d, d, device=DEV)
+    z = torch.empty(wl.B, wl.H, d, device=DEV)
+    st = hf.hf_state_init(S, z)
+    heads = (0, wl.H - 1)
+    ev_k, ev_v = [], []
+    for t in range(1, 21):
+        g = torch.Generator().manual_seed(10000 + t)
+        K_ev = frame_structured(g, wl.B, wl.H, wl.Ne_step, d, wl.tokens_per_frame, wl.w)
+        V_ev = frame_structured(g, wl.B, wl.H, wl.Ne_step, d, wl.tokens_per_frame, wl.w)
+        if t == 20:
+            # the last step's attention reads the state of the first 19 steps
+            x = draw_step_inputs(wl, seed=20000, n_evicted=1)
+            Qd, Kd, Vd = x["Q"].to(DEV), x["K"].to(DEV), x["V"].to(DEV)
+            idx = hf.hf_select_blocks(Qd, Kd, wl.block, wl.r)
+            O = hf.hf_hybrid_attn_fwd(Qd, Kd, Vd, wl.block, wl.r, idx, st)
+            torch.cuda.synchronize()
+            S19, z19 = f64(st.S), f64(st.z)
+            Q64, K64, V64 = f64(x["Q"]), f64(x["K"]), f64(x["V"])
+            Og = f64(O)
+            for (b, h, I) in _sample_tiles(wl, 3, seed=2):
+                lo, hi = I * wl.block, min((I + 1) * wl.block, wl.Nq)
+                want = oracle.hybrid_attention_tile(Q64, K64, V64, idx.cpu().numpy(), S19, z19, wl.block, b, h, I)
+                assert_output_close(Og[b, h, lo:hi], want, what=f"O tile {(b, h, I)} at step 20")
+        hf.hf_absorb_evicted(st, K_ev.to(DEV), V_ev.to(DEV))
+        ev_k.append(K_ev[:, list(heads)])
+        ev_v.append(V_ev[:, list(heads)])
+    torch.cuda.synchronize()
+    _check_status()
+    assert st.n_absorbed == 20 * wl.Ne_step
+    S_o, z_o = oracle.absorb_batch(f64(torch.cat(ev_k, 2)), f64(torch.cat(ev_v, 2)))
+    assert_state_close(f64(st.S[:, list(heads)]), f64(st.z[:, list(heads)]), S_o, z_o)
+
+
 def _sample_tiles(wl, n, seed=0):
     rng = np.random.default_rng(seed)
     tiles = {(0, h, int(rng.integers(0, wl.nQB))) for h in rng.integers(0, wl.H, size=n)}
