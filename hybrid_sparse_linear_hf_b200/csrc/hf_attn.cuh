@@ -17,8 +17,10 @@
 // 384 threads, three warpgroups; setmaxnreg moves registers from the first to the others:
 //   warp 0      TMA producer of the Q tile (once) and of the K tile of each kept block J
 //               into a ring of K slots (row coordinate J*block; rows past Nk are
-//               zero-filled); a K slot frees as soon as its QK^T is done.
-//   warp 1      TMEM owner (512 columns) + single-thread tcgen05 MMA issuer.
+//               zero-filled); warp 3 frees a K slot once its QK^T is done.
+//   warp 1      TMEM owner (512 columns) + single-thread tcgen05 MMA issuer: one wait
+//               (P ready) and one commit (the next S of that pipeline) per kept block, as
+//               the tensor core's shallow instruction queue idles whenever it does more.
 //   warp 2      TMA producer of the V tiles into a ring of V slots.
 //   warp 3      ring bookkeeping, off the softmax threads' path: in kept-block order it
 //               waits for S of block v (so QK(v), and PV(v-2) before it, are done), frees
