@@ -8,13 +8,15 @@ key blocks, state built from 60 evicted frames):
     hf_absorb_evicted     the chunk step's 3 evicted frames -> state (2 kernels)
 Metric: query tokens/s per chunk step (whole job, all GPUs), with the roofline fraction
 of the dominant kernel (hf_hybrid_attn_fwd, tensor-bound) against the measured bf16
-peak. Inputs are resident in HBM; L2 is flushed between timed steps (outside the
+peak. Legs reported beside the step: the 60-frame state build, the two-stage (frame,
+then block) selection, the attention at keep 1 / 0.5 / 0.25 / 0.125, and the step end to
+end with its inputs copied from pinned host memory and O copied back. Inputs are resident in HBM; L2 is flushed between timed steps (outside the
 timed events). Multi-GPU (torchrun): every rank runs its own chunk stream (weak
 scaling, no collective on the data path); time = max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
-``--impl reference`` times the fp64 CPU oracle instead (a bounded sample of heads of
+``--impl reference`` times the fp64 CPU oracle instead (per step a bounded sample of
 the same step, scaled to the whole step) on the host cores.
 """
 from __future__ import annotations

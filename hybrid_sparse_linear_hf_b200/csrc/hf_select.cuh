@@ -1,14 +1,15 @@
-// Block scoring and top-r selection (hf_select_blocks).
+// Block scoring and top-r selection (hf_select_blocks, hf_select_blocks_two_stage).
 //
 // Source: "Light Forcing: Accelerating Autoregressive Video Diffusion via Sparse
 // Attention", German technical summary, section 2.2 (query and key tokens are
 // compressed by mean pooling at block level; key blocks are selected per query
 // block); "Long-Horizon Streaming Video Generation via Hybrid Attention with
 // Decoupled Distillation", German technical summary, section 2 A (only the most
-// important, Top-K, blocks are computed).
+// important, Top-K, blocks are computed). Light Forcing section 2.2 also gives the
+// two-stage variant (frames by frame-pooled keys, then blocks within them).
 //
-// Two kernels, both on CUDA cores (the work is a streaming read of Q and K plus a
-// tiny score matrix, so tensor cores would not help):
+// All on CUDA cores (the work is a streaming read of Q and K plus a tiny score matrix,
+// so tensor cores would not help):
 //   pool_blocks_kernel   one CTA per (b,h,block) of Q or K: fp32 mean of the valid rows.
 //                        HBM-bound: reads Q and K once with 16-byte loads, 8 in flight
 //                        per thread.
@@ -18,6 +19,9 @@
 //                        reduction per bit), takes every block above it and the lowest-J
 //                        blocks equal to it, and writes the r blocks in ascending J.
 //                        NaN scores are ranked as -inf, so exactly r blocks are written.
+// Two-stage selection: pool_blocks_kernel<d, true> also writes each key block's sums in
+// its first and next frame, pool_frames_kernel adds them into frame means, and
+// score_select2_kernel keeps frames first, then blocks within them (see there).
 #pragma once
 
 #include "hf_ptx.cuh"
