@@ -89,6 +89,15 @@ def attn_flops(idx: np.ndarray, wl) -> float:
     return sparse + readout
 
 
+def attn_issued_flops(idx: np.ndarray, wl) -> float:
+    """FLOPs the attention kernel issues on the tensor cores: per kept block 128-row QK^T and
+    PV MMAs over the whole block (padding included), plus the three split-precision readout
+    MMAs (phi_hi S_hi, phi_hi S_lo, phi_lo S_hi) per 128-row query tile."""
+    kept = int(((idx >= 0) & (idx < wl.nKB)).sum())
+    tiles = wl.B * wl.H * wl.nQB
+    return 4.0 * 128 * wl.block * wl.d * kept + 3 * 2.0 * 128 * wl.d * wl.d * tiles
+
+
 def attn_bytes(wl) -> float:
     """Algorithmic bytes of one launch: Q and O once, the whole K/V window once, S and z."""
     return 2.0 * wl.B * wl.H * (2 * wl.Nq * wl.d + 2 * wl.Nk * wl.d) + 4.0 * wl.B * wl.H * (wl.d * wl.d + wl.d)
@@ -485,6 +494,7 @@ def run_gpu(args, wl) -> None:
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": achieved_tf / peaks["bf16_tflops"], "traffic": ATTN_TRAFFIC_BYTES,
                      "kernel": "hybrid_attn_kernel<128,128>", "flops_per_launch": F,
+                     "issued_flops_per_launch": attn_issued_flops(idx_host, wl),
                      "peak_source": f"{peaks['source']} dense bf16 (burst)"},
         "kernels": {
             "hf_hybrid_attn_fwd": {"us": fwd_mean * 1e6, "tflops": achieved_tf,

@@ -48,3 +48,4 @@ def test_two_rank_timing_and_inputs():
     assert s0 != s1, "ranks must stream different synthetic inputs"
     assert t0 == t1 == pytest.approx(0.002), "every rank reports the slowest rank's time"
     assert v0 == v1 == pytest.approx(world * 64 / 0.002)
+
