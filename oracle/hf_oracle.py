@@ -22,7 +22,9 @@ Sources (page title, then the section used):
            §2.2 Hierarchische Spärliche Attention (token compression by mean
            pooling at block and frame level; per-query-block selection; the
            two-stage mask selection: frames first by frame-level compressed keys,
-           then blocks within the selected frames).
+           then blocks within the selected frames); §2.1 Chunk-bewusstes
+           Wachstum (dense first chunk, sparsity s_i = s_base - alpha_i beta for
+           the later chunks, beta set by a FLOP budget).
 
 The pages give the structure (a compact KV state absorbing evicted tokens
 through a linear attention function; Top-K block-sparse attention inside the
@@ -56,7 +58,7 @@ __all__ = [
     "select_blocks", "frame_ranges", "pool_frames", "frame_scores", "candidate_blocks",
     "select_blocks_two_stage", "sparse_attention_tile", "sparse_attention", "linear_readout",
     "hybrid_attention", "hybrid_attention_tile", "absorb", "absorb_batch",
-    "dense_swa", "default_scale",
+    "dense_swa", "default_scale", "keep_schedule",
 ]
 
 
@@ -306,3 +308,42 @@ def dense_swa(Q, K, V, scale: float | None = None) -> np.ndarray:
     a = a - a.max(axis=-1, keepdims=True)
     p = np.exp(a)
     return (p @ V) / p.sum(axis=-1, keepdims=True)
+
+
+def keep_schedule(nKB, s_base: float, s_target: float):
+    """Chunk-aware growth: the sparsity of every chunk of a video and its kept key blocks.
+
+    [LF] §2.1: the first chunk attends densely; a later chunk i gets the sparsity ratio
+    s_i = s_base - alpha_i * beta, where alpha_i follows the noise scale 1/sqrt(T) and beta
+    is set so that the FLOPs of all chunks meet a target sparsity ratio, so that earlier
+    chunks keep more and later ones less.
+    Readings (the page gives no constants): T is the chunk's position i >= 1, so
+    alpha_i = 1/sqrt(i); a chunk's dense attention FLOPs are proportional to the key blocks of
+    its window, nKB[i] (every chunk has the same queries); the budget is
+        sum_i (1 - s_i) nKB[i] = (1 - s_target) sum_i nKB[i];
+    chunk i keeps r_i = clamp(ceil((1 - s_i) nKB[i]), 1, nKB[i]) blocks. A single chunk is
+    dense whatever the target. A schedule whose beta would be negative (sparsity falling
+    with i) or whose s_i would leave [0, 1) is rejected with ValueError.
+    Returns (r int64 [n], s float64 [n], beta).
+    """
+    nKB = [int(x) for x in nKB]
+    n = len(nKB)
+    if n < 1 or min(nKB) < 1:
+        raise ValueError("every chunk needs at least one key block")
+    if not (0.0 <= s_base < 1.0 and 0.0 <= s_target < 1.0):
+        raise ValueError("sparsity ratios lie in [0, 1)")
+    s = np.zeros(n)
+    beta = 0.0
+    if n > 1:
+        alpha = np.array([1.0 / math.sqrt(i) for i in range(1, n)])
+        later = np.array(nKB[1:], dtype=np.float64)
+        # nKB[0] + sum_{i>=1} (1 - s_base + alpha_i beta) nKB[i] = (1 - s_target) sum_i nKB[i]
+        budget = (1.0 - s_target) * float(sum(nKB))
+        beta = (budget - nKB[0] - (1.0 - s_base) * later.sum()) / float((alpha * later).sum())
+        if beta < 0.0:
+            raise ValueError("the budget needs sparsity falling with the chunk index (beta < 0)")
+        s[1:] = s_base - alpha * beta
+        if np.any(s < 0.0) or np.any(s >= 1.0):
+            raise ValueError("a chunk's sparsity leaves [0, 1)")
+    r = np.array([min(max(math.ceil((1.0 - s[i]) * nKB[i]), 1), nKB[i]) for i in range(n)], dtype=np.int64)
+    return r, s, beta

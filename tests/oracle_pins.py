@@ -344,6 +344,98 @@ def check_two_stage_bruteforce(o):
             assert idx[0, 0, I].tolist() == want, (trial, I, idx[0, 0, I].tolist(), want)
 
 
+# ---------------------------------------------------------------------------
+# chunk-aware growth (per-chunk keep schedule)
+# ---------------------------------------------------------------------------
+def check_schedule_golden(o):
+    for case in _golden()["keep_schedule"]["cases"]:
+        r, s, beta = o.keep_schedule(case["nKB"], case["s_base"], case["s_target"])
+        assert r.tolist() == case["r"], (r.tolist(), case["r"])
+        assert np.allclose(s, case["s"], atol=1e-6), (s, case["s"])
+        assert abs(beta - case["beta"]) < 1e-6, beta
+
+
+def _feasible_cases(seed, count):
+    """Random window sizes (a window filling up, then full), target and s_base with beta >= 0."""
+    rng = np.random.default_rng(seed)
+    out = []
+    while len(out) < count:
+        n = int(rng.integers(2, 14))
+        full = int(rng.integers(4, 300))
+        fill = int(rng.integers(1, 8))
+        nKB = [max(1, (full * min(i + 1, fill)) // fill) for i in range(n)]
+        t = float(rng.uniform(0.05, 0.9))
+        flat = 1.0 - ((1.0 - t) * sum(nKB) - nKB[0]) / sum(nKB[1:])  # s_base with beta = 0
+        if not (0.0 <= flat < 0.97):
+            continue
+        s_base = float(rng.uniform(flat, min(0.99, flat + 0.3)))
+        out.append((nKB, s_base, t, flat))
+    return out
+
+
+def check_schedule_budget_and_rounding(o):
+    for nKB, s_base, t, _ in _feasible_cases(31, 40):
+        try:
+            r, s, beta = o.keep_schedule(nKB, s_base, t)
+        except ValueError:
+            continue  # some s_i below 0: rejected, checked elsewhere
+        assert s[0] == 0.0 and r[0] == nKB[0], "the first chunk attends densely"
+        kept = sum((1.0 - s[i]) * nKB[i] for i in range(len(nKB)))
+        assert abs(kept - (1.0 - t) * sum(nKB)) <= 1e-9 * sum(nKB), "FLOP budget"
+        assert all(s[i] <= s[i + 1] + 1e-15 for i in range(1, len(nKB) - 1)), "sparsity grows with i"
+        for i, k in enumerate(nKB):
+            x = (1.0 - s[i]) * k
+            assert 1 <= r[i] <= k
+            assert r[i] >= min(x, k) - 1e-9 and (r[i] == 1 or r[i] - 1 < x + 1e-9), (i, x, r[i])
+
+
+def check_schedule_two_chunks(o):
+    """With one sparse chunk, it keeps exactly what the dense first chunk leaves of the budget."""
+    for a, b, t, s_base in ((3, 9, 0.4, 0.9), (37, 256, 0.75, 0.95), (1, 1, 0.25, 0.7), (5, 50, 0.6, 0.7)):
+        r, s, beta = o.keep_schedule([a, b], s_base, t)
+        s1 = 1.0 - ((1.0 - t) * (a + b) - a) / b
+        assert abs(s[1] - s1) < 1e-12 and abs(beta - (s_base - s1)) < 1e-12, (s, beta, s1)
+        assert r[1] == min(max(math.ceil((1.0 - s1) * b - 1e-12), 1), b)
+
+
+def check_schedule_noise_scale(o):
+    """Later chunks' sparsity gaps to s_base follow 1/sqrt(i): chunk 4 has half chunk 1's
+    gap, chunk 9 a third; at the flat s_base (beta = 0) every later chunk has s_base; beta
+    agrees with a bisection on the budget."""
+    nKB = [20] + [40] * 11
+    t = 0.6
+    flat = 1.0 - ((1.0 - t) * sum(nKB) - nKB[0]) / sum(nKB[1:])
+    _, s, beta = o.keep_schedule(nKB, flat + 0.2, t)
+    g = (flat + 0.2) - s
+    assert beta > 0 and abs(g[4] / g[1] - 0.5) < 1e-12 and abs(g[9] / g[1] - 1.0 / 3.0) < 1e-12, g
+    _, s, beta = o.keep_schedule(nKB, flat + 1e-9, t)  # just above: rounding decides beta's sign at flat
+    assert 0.0 <= beta < 1e-8 and np.allclose(s[1:], flat, atol=1e-8)
+    # beta by bisection on the budget residual, independent of the closed form
+    s_base = flat + 0.1
+    lo, hi = 0.0, 1.0
+    for _ in range(200):
+        mid = 0.5 * (lo + hi)
+        kept = nKB[0] + sum((1.0 - s_base + mid / math.sqrt(i)) * nKB[i] for i in range(1, len(nKB)))
+        lo, hi = (mid, hi) if kept < (1.0 - t) * sum(nKB) else (lo, mid)
+    _, _, beta = o.keep_schedule(nKB, s_base, t)
+    assert abs(beta - lo) < 1e-12, (beta, lo)
+
+
+def check_schedule_rejects(o):
+    def rejected(*a):
+        try:
+            o.keep_schedule(*a)
+        except ValueError:
+            return True
+        return False
+    assert rejected([10, 10], 0.2, 0.5), "s_base below the flat value needs beta < 0"
+    assert rejected([], 0.5, 0.5) and rejected([4, 0], 0.5, 0.5)
+    assert rejected([4, 4], 1.0, 0.5) and rejected([4, 4], 0.5, -0.1)
+    assert rejected([100, 1], 0.99, 0.9), "the budget leaves the later chunk nothing (s_1 >= 1)"
+    r, s, _ = o.keep_schedule([7], 0.5, 0.9)
+    assert r.tolist() == [7] and s.tolist() == [0.0], "a single chunk is dense"
+
+
 ALL_CHECKS = [
     check_phi_library, check_pool_by_hand, check_selection_golden, check_selection_bruteforce,
     check_selection_ties_constructed, check_selection_output_form, check_attention_golden,
@@ -352,5 +444,6 @@ ALL_CHECKS = [
     check_absorb_incremental_equals_batch, check_absorb_single_token,
     check_readout_closed_forms, check_hybrid_sum, check_two_stage_golden,
     check_two_stage_all_frames_is_one_stage, check_two_stage_frames_are_blocks,
-    check_two_stage_bruteforce,
+    check_two_stage_bruteforce, check_schedule_golden, check_schedule_budget_and_rounding,
+    check_schedule_two_chunks, check_schedule_noise_scale, check_schedule_rejects,
 ]

@@ -178,12 +178,62 @@ def _mut_two_stage_no_fill(m):
     m.select_blocks_two_stage = f
 
 
+def _mut_schedule_alpha_linear(m):
+    # alpha_i = 1/i instead of 1/sqrt(i)
+    import math as math_mod
+
+    class _Math:
+        def __getattr__(self, k):
+            return getattr(math_mod, k)
+
+        @staticmethod
+        def sqrt(x):
+            return float(x) if x >= 1 else math_mod.sqrt(x)
+    m.math = _Math()
+
+
+def _mut_schedule_first_chunk_sparse(m):
+    orig = m.keep_schedule
+
+    def f(nKB, s_base, s_target):
+        r, s, beta = orig(nKB, s_base, s_target)
+        s = s.copy()
+        s[0] = s_base - beta  # the formula applied to the first chunk too
+        r = r.copy()
+        r[0] = max(1, int(np.ceil((1.0 - s[0]) * nKB[0])))
+        return r, s, beta
+    m.keep_schedule = f
+
+
+def _mut_schedule_floor(m):
+    orig = m.keep_schedule
+
+    def f(nKB, s_base, s_target):
+        r, s, beta = orig(nKB, s_base, s_target)
+        r = np.array([min(max(int(np.floor((1.0 - s[i]) * nKB[i])), 1), nKB[i]) for i in range(len(nKB))])
+        return r, s, beta
+    m.keep_schedule = f
+
+
+def _mut_schedule_budget_on_chunks(m):
+    # the target read as a per-chunk sparsity for the later chunks only (dense chunk not counted)
+    orig = m.keep_schedule
+
+    def f(nKB, s_base, s_target):
+        total = float(sum(nKB))
+        t2 = 1.0 - (1.0 - s_target) * (total - nKB[0]) / total if len(nKB) > 1 else s_target
+        return orig(nKB, s_base, t2)
+    m.keep_schedule = f
+
+
 MUTANTS = [
     _mut_phi_no_plus_one, _mut_phi_exp, _mut_readout_no_eps, _mut_readout_transposed,
     _mut_readout_no_phi_q, _mut_select_ties_high, _mut_select_bottom, _mut_pool_sum,
     _mut_attention_no_scale, _mut_attention_sqrt_d, _mut_attention_all_keys,
     _mut_absorb_transposed, _mut_absorb_z_raw, _mut_hybrid_difference, _mut_two_stage_inside_only,
     _mut_two_stage_ignore_frames, _mut_pool_frames_sum, _mut_two_stage_frame_ties_high, _mut_two_stage_no_fill,
+    _mut_schedule_alpha_linear, _mut_schedule_first_chunk_sparse, _mut_schedule_floor,
+    _mut_schedule_budget_on_chunks,
 ]
 
 
