@@ -60,6 +60,9 @@ _SIGNATURES = {
     "hf_hybrid_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
                            [ctypes.c_void_p, ctypes.POINTER(HfStateC), ctypes.c_float, ctypes.c_void_p,
                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_keep_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_double,
+                                        ctypes.c_double, ctypes.POINTER(ctypes.c_int),
+                                        ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
     "hf_query_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
     "hf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "hf_version": (ctypes.c_char_p, []),
@@ -233,6 +236,22 @@ def hf_select_blocks_noalloc(Q: torch.Tensor, K: torch.Tensor, block: int, r: in
                                           if scores_out is not None else None, _stream(stream)),
            "hf_select_blocks_noalloc")
     return idx_out
+
+
+def hf_keep_schedule(nKB, s_base: float, s_target: float):
+    """Chunk-aware growth schedule (host only): for chunk windows of ``nKB[i]`` key blocks,
+    returns (r, s, beta): kept blocks per chunk (list of int, the ``r`` of that chunk's
+    select and attention calls), sparsity ratios (list of float) and beta. The first chunk
+    is dense; later chunks approach ``s_base`` as beta/sqrt(i) shrinks; beta makes the
+    kept FLOPs equal ``1 - s_target`` of the dense ones."""
+    n = len(nKB)
+    kb = (ctypes.c_int * max(n, 1))(*[int(x) for x in nKB])
+    r = (ctypes.c_int * max(n, 1))()
+    sv = (ctypes.c_double * max(n, 1))()
+    beta = ctypes.c_double(0.0)
+    _check(lib().hf_keep_schedule(n, kb, float(s_base), float(s_target), r, sv, ctypes.byref(beta)),
+           "hf_keep_schedule")
+    return list(r)[:n], list(sv)[:n], beta.value
 
 
 def hf_hybrid_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block: int, r: int,

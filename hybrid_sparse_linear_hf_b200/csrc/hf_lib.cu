@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "hf.h"
 #include "hf_absorb.cuh"
@@ -436,6 +437,36 @@ HF_API hf_status hf_hybrid_attn_fwd(const hf_bf16* Q, const hf_bf16* K, const hf
   HF_ATTN_CASE(64, 32)
 #undef HF_ATTN_CASE
   return HF_ERR_UNSUPPORTED;
+}
+
+HF_API hf_status hf_keep_schedule(int n_chunks, const int* nKB, double s_base, double s_target, int* r_out,
+                                  double* s_out, double* beta_out) {
+  if (n_chunks < 1 || !nKB || !r_out) return HF_ERR_INVALID_ARG;
+  if (!(s_base >= 0.0 && s_base < 1.0) || !(s_target >= 0.0 && s_target < 1.0)) return HF_ERR_INVALID_ARG;
+  double total = 0.0, later = 0.0, later_w = 0.0;  // all blocks; chunks >= 1; weighted by 1/sqrt(i)
+  for (int i = 0; i < n_chunks; ++i) {
+    if (nKB[i] < 1) return HF_ERR_INVALID_ARG;
+    total += nKB[i];
+    if (i > 0) {
+      later += nKB[i];
+      later_w += nKB[i] / std::sqrt(static_cast<double>(i));
+    }
+  }
+  // (1 - s_target) total = nKB[0] + (1 - s_base) later + beta later_w
+  const double beta = n_chunks > 1 ? ((1.0 - s_target) * total - nKB[0] - (1.0 - s_base) * later) / later_w : 0.0;
+  if (!(beta >= 0.0)) return HF_ERR_INVALID_ARG;
+  std::vector<double> s(n_chunks, 0.0);
+  for (int i = 1; i < n_chunks; ++i) {
+    s[i] = s_base - beta / std::sqrt(static_cast<double>(i));
+    if (!(s[i] >= 0.0 && s[i] < 1.0)) return HF_ERR_INVALID_ARG;
+  }
+  for (int i = 0; i < n_chunks; ++i) {
+    const double keep = std::ceil((1.0 - s[i]) * nKB[i]);
+    r_out[i] = keep < 1.0 ? 1 : (keep > nKB[i] ? nKB[i] : static_cast<int>(keep));
+    if (s_out) s_out[i] = s[i];
+  }
+  if (beta_out) *beta_out = beta;
+  return HF_OK;
 }
 
 HF_API hf_status hf_query_status(void* stream, uint32_t* detail_out) {

@@ -207,6 +207,27 @@ HF_API hf_status hf_hybrid_attn_fwd(const hf_bf16* Q, const hf_bf16* K, const hf
                                     const hf_state* st, float scale, hf_bf16* O, void* ws, size_t ws_bytes,
                                     void* stream);
 
+/* Per-chunk keep schedule of chunk-aware growth (host only; no device work): the
+ * sparsity ratio s[i] and the kept key blocks r[i] of every chunk i of a video, for
+ * hf_select_blocks / hf_hybrid_attn_fwd of that chunk.
+ *   s[0] = 0                                  (the first chunk attends densely)
+ *   s[i] = s_base - beta / sqrt(i), i >= 1    (sparsity grows towards s_base)
+ *   beta: sum_i (1 - s[i]) nKB[i] = (1 - s_target) sum_i nKB[i]   (the FLOP budget)
+ *   r[i] = clamp(ceil((1 - s[i]) nKB[i]), 1, nKB[i])
+ * Source: Light Forcing, German technical summary section 2.1 (dense first chunk;
+ * s_i = s_base - alpha_i beta with alpha_i following the noise scale 1/sqrt(T); beta set
+ * so that the total FLOPs meet a target sparsity ratio). Readings where the page gives
+ * no constants: alpha_i = 1/sqrt(i) with the chunk's position i as T; a chunk's FLOPs
+ * proportional to its window's key blocks nKB[i] (every chunk has the same queries).
+ * nKB: [n_chunks] host ints >= 1 (the window of chunk i, in blocks); r_out: [n_chunks]
+ * host ints (written on success only); s_out: optional [n_chunks] host doubles (NULL to
+ * skip); beta_out optional. n_chunks == 1 gives the dense first chunk whatever s_target.
+ * Errors (nothing written): HF_ERR_INVALID_ARG for n_chunks < 1, a NULL nKB or r_out,
+ * nKB[i] < 1, s_base or s_target outside [0, 1), a budget that would need beta < 0
+ * (sparsity falling with i: raise s_base) or an s[i] outside [0, 1). */
+HF_API hf_status hf_keep_schedule(int n_chunks, const int* nKB, double s_base, double s_target, int* r_out,
+                                  double* s_out, double* beta_out);
+
 /* Synchronise `stream`, then read and clear the device error word of the current
  * device. Returns HF_OK, HF_ERR_DEVICE_TIMEOUT, HF_ERR_DEVICE_BAD_INDEX or HF_ERR_CUDA
  * (an asynchronous CUDA error). If detail_out is not NULL it receives the raw word
