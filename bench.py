@@ -22,6 +22,7 @@ the same step, scaled to the whole step) on the host cores.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import faulthandler
 import json
 import math
@@ -55,6 +56,11 @@ ATTN_TRAFFIC_BYTES = 161.3e6 + 12.8e6
 TWO_STAGE_FRAMES = 8
 # keep ratios of the sparsity sweep leg (1 = dense window attention)
 SWEEP_KEEPS = (1.0, 0.5, 0.25, 0.125)
+# chunk-aware growth leg: a video's first chunks (the window filling up, then full) under
+# the keep schedule with these sparsity ratios, against the same mean sparsity per chunk
+SCHEDULE_CHUNKS = 12
+SCHEDULE_S_BASE = 0.85
+SCHEDULE_S_TARGET = 0.75
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -442,6 +448,45 @@ def run_gpu(args, wl) -> None:
     rc, word = hf.hf_query_status()
     if rc != hf.HF_OK:
         raise RuntimeError(f"device status after the sweep leg: {hf.hf_status_string(rc)} ({word:#x})")
+    # ---- chunk-aware growth: the attention of a video's first chunks under the keep
+    # schedule (chunk i's window holds the newest min(i + 1, full) chunks of keys)
+    log("keep schedule leg")
+    per_window = wl.window_frames // wl.chunk_frames
+    wls = [dataclasses.replace(wl, window_frames=min(i + 1, per_window) * wl.chunk_frames)
+           for i in range(SCHEDULE_CHUNKS)]
+    nKB_s = [w.nKB for w in wls]
+    r_s, s_s, beta_s = hf.hf_keep_schedule(nKB_s, SCHEDULE_S_BASE, SCHEDULE_S_TARGET)
+    r_u = [max(1, math.ceil((1.0 - SCHEDULE_S_TARGET) * n - 1e-9)) for n in nKB_s]
+    kv_win = {}
+    for w in wls:
+        if w.Nk not in kv_win:
+            kv_win[w.Nk] = (K[:, :, K.shape[2] - w.Nk:].contiguous(), V[:, :, V.shape[2] - w.Nk:].contiguous())
+
+    def time_chunk(w, r_c):
+        Kc, Vc = kv_win[w.Nk]
+        idx_c = torch.empty(wl.B, wl.H, wl.nQB, r_c, dtype=torch.int32, device=dev)
+        hf.hf_select_blocks(Q, Kc, wl.block, r_c, idx_out=idx_c, ws=ws_sel)
+        tc = []
+        for k in range(5):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            hf.hf_hybrid_attn_fwd(Q, Kc, Vc, wl.block, r_c, idx_c, st, O=O)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if k >= 2:
+                tc.append(e0.elapsed_time(e1) * 1e-3)
+        return statistics.mean(tc) * 1e6
+
+    us_s = [time_chunk(w, rc_) for w, rc_ in zip(wls, r_s)]
+    us_u = [time_chunk(w, rc_) for w, rc_ in zip(wls, r_u)]
+    del kv_win
+    rc, word = hf.hf_query_status()
+    if rc != hf.HF_OK:
+        raise RuntimeError(f"device status after the keep schedule leg: {hf.hf_status_string(rc)} ({word:#x})")
+    schedule = {"s_base": SCHEDULE_S_BASE, "s_target": SCHEDULE_S_TARGET, "beta": beta_s, "nKB": nKB_s,
+                "r": r_s, "attn_us": [round(u, 1) for u in us_s], "attn_us_total": sum(us_s),
+                "uniform_r": r_u, "uniform_attn_us_total": sum(us_u)}
     log("end-to-end leg")
     # ---- end to end through the public API with host buffers (pinned), copies timed
     host = {k: v.cpu().pin_memory() for k, v in x.items()}
@@ -518,6 +563,7 @@ def run_gpu(args, wl) -> None:
             "hbm_peak_gbs": peaks["hbm_gbs"],
         },
         "sweep": {k: dict(v, frac=v["tflops"] / peaks["bf16_tflops"]) for k, v in sweep.items()},
+        "keep_schedule": schedule,
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "clocks": clk.summary(),
         "e2e": {"value": job_throughput(world, wl.B, wl.Nq, t_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
