@@ -62,6 +62,8 @@ SWEEP_KEEPS = (1.0, 0.5, 0.25, 0.125)
 SCHEDULE_CHUNKS = 12
 SCHEDULE_S_BASE = 0.85
 SCHEDULE_S_TARGET = 0.75
+# pooled-key cache leg: tokens per granule sum (divides the 4680-key chunk and the block)
+KPOOL_GRANULE = 8
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -426,6 +428,32 @@ def run_gpu(args, wl) -> None:
     rc, word = hf.hf_query_status()
     if rc != hf.HF_OK:
         raise RuntimeError(f"device status after the two-stage leg: {hf.hf_status_string(rc)} ({word:#x})")
+    # ---- pooled-key cache: per step the chunk's keys enter the cache and the oldest chunk
+    # leaves (hf_kpool_push), then the selection pools its key blocks from the granule sums
+    log("pooled-key cache leg")
+    kp_sums = torch.empty(wl.B, wl.H, wl.Nk // KPOOL_GRANULE, wl.d, dtype=torch.float32, device=dev)
+    kp = hf.hf_kpool_init(kp_sums, KPOOL_GRANULE)
+    for c0 in range(0, wl.Nk, wl.Nq):
+        hf.hf_kpool_push(kp, K[:, :, c0:c0 + wl.Nq].contiguous())
+    K_in = K[:, :, wl.Nk - wl.Nq:].contiguous()  # stands in for the chunk's new keys
+    idx_c = torch.empty_like(idx)
+    t_push, t_selc = [], []
+    for k in range(n_sel2 + 3):
+        flush.zero_()
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        hf.hf_kpool_push(kp, K_in, n_evict=wl.Nq)
+        e1.record(stream)
+        hf.hf_select_blocks_cached(Q, kp, wl.block, wl.r, idx_out=idx_c, ws=ws_sel)
+        e2.record(stream)
+        torch.cuda.synchronize(dev)
+        if k >= 3:
+            t_push.append(e0.elapsed_time(e1) * 1e-3)
+            t_selc.append(e1.elapsed_time(e2) * 1e-3)
+    del kp_sums, K_in
+    rc, word = hf.hf_query_status()
+    if rc != hf.HF_OK:
+        raise RuntimeError(f"device status after the pooled-key cache leg: {hf.hf_status_string(rc)} ({word:#x})")
     # ---- sparsity sweep: the attention alone at other keep ratios (same inputs and state)
     log("sweep leg")
     sweep = {}
@@ -553,6 +581,10 @@ def run_gpu(args, wl) -> None:
                                            "gbs": select_bytes(wl) / statistics.mean(t_sel2) / 1e9,
                                            "hbm_frac": select_bytes(wl) / statistics.mean(t_sel2) / 1e9
                                            / peaks["hbm_gbs"]},
+            "hf_select_blocks_cached": {"us": statistics.mean(t_selc) * 1e6,
+                                        "push_us": statistics.mean(t_push) * 1e6, "granule": KPOOL_GRANULE,
+                                        "note": "per step: hf_kpool_push of the 4680 new keys (and eviction "
+                                                "of the oldest 4680), then the selection from the granule sums"},
             "hf_absorb_evicted_step": {"us": abs_mean * 1e6, "tokens": wl.Ne_step,
                                        "bytes": absorb_bytes(wl, wl.Ne_step),
                                        "gbs": absorb_bytes(wl, wl.Ne_step) / abs_mean / 1e9},

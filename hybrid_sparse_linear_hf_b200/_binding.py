@@ -37,6 +37,14 @@ class HfStateC(ctypes.Structure):
                 ("S", ctypes.c_void_p), ("z", ctypes.c_void_p), ("n_absorbed", ctypes.c_longlong)]
 
 
+class HfKpoolC(ctypes.Structure):
+    """Mirror of ``struct hf_kpool``."""
+
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int), ("granule", ctypes.c_int),
+                ("capacity", ctypes.c_int), ("n_gran", ctypes.c_int), ("head", ctypes.c_int),
+                ("sums", ctypes.c_void_p)]
+
+
 class HfError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -60,6 +68,11 @@ _SIGNATURES = {
     "hf_hybrid_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
                            [ctypes.c_void_p, ctypes.POINTER(HfStateC), ctypes.c_float, ctypes.c_void_p,
                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_kpool_init": (ctypes.c_int, [ctypes.POINTER(HfKpoolC)] + [ctypes.c_int] * 5 + [ctypes.c_void_p]),
+    "hf_kpool_push": (ctypes.c_int, [ctypes.POINTER(HfKpoolC), ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_void_p]),
+    "hf_select_blocks_cached": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(HfKpoolC)] + [ctypes.c_int] * 3 +
+                                [ctypes.c_void_p] * 3 + [ctypes.c_size_t, ctypes.c_void_p]),
     "hf_keep_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_double,
                                         ctypes.c_double, ctypes.POINTER(ctypes.c_int),
                                         ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
@@ -138,6 +151,19 @@ class HfState:
         return (self.c.B, self.c.H, self.c.d)
 
 
+class HfKpool:
+    """Python handle of ``hf_kpool``: keeps the granule sums [B,H,capacity,d] (fp32,
+    device) alive; ``n_tokens`` is the window length the pushes have built."""
+
+    def __init__(self, sums: torch.Tensor):
+        self.sums = sums
+        self.c = HfKpoolC()
+
+    @property
+    def n_tokens(self) -> int:
+        return int(self.c.n_gran) * int(self.c.granule)
+
+
 def hf_workspace_size(which: int, B: int, H: int, Nq: int, Nk: int, d: int, block: int, r: int) -> int:
     n = lib().hf_workspace_size(which, B, H, Nq, Nk, d, block, r)
     if n == _SIZE_T_MAX:
@@ -193,6 +219,48 @@ def hf_select_blocks(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, idx_o
                                   _dev(scores_out, torch.float32, "scores_out") if scores_out is not None else None,
                                   ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
            "hf_select_blocks")
+    return idx_out
+
+
+def hf_kpool_init(sums: torch.Tensor, granule: int) -> HfKpool:
+    """An empty pooled-key cache over ``sums`` [B,H,capacity,d] fp32 (device): the ring
+    of the window's sums of ``granule`` consecutive key tokens."""
+    if sums.dim() != 4:
+        raise ValueError("sums must be [B,H,capacity,d]")
+    B, H, cap, d = sums.shape
+    kp = HfKpool(sums)
+    _check(lib().hf_kpool_init(ctypes.byref(kp.c), B, H, d, granule, cap, _dev(sums, torch.float32, "sums")),
+           "hf_kpool_init")
+    return kp
+
+
+def hf_kpool_push(kp: HfKpool, K_new, n_evict: int = 0, stream=None) -> None:
+    """The window drops its ``n_evict`` oldest key tokens, then takes K_new [B,H,n,d] bf16
+    (or None for no new keys) as its newest."""
+    n = 0 if K_new is None else int(K_new.shape[2])
+    if K_new is not None and (K_new.dim() != 4 or tuple(K_new.shape[:2]) != (kp.c.B, kp.c.H)
+                              or K_new.shape[3] != kp.c.d):
+        raise ValueError("K_new must be [B,H,n,d] matching the cache")
+    _check(lib().hf_kpool_push(ctypes.byref(kp.c), _dev(K_new, torch.bfloat16, "K_new") if n > 0 else None, n,
+                               int(n_evict), _stream(stream)), "hf_kpool_push")
+
+
+def hf_select_blocks_cached(Q: torch.Tensor, kp: HfKpool, block: int, r: int, idx_out=None, scores_out=None,
+                            ws=None, stream=None) -> torch.Tensor:
+    """hf_select_blocks over the cached window (its ``kp.n_tokens`` keys)."""
+    B, H, Nq, d = Q.shape
+    Nk = kp.n_tokens
+    nQB = -(-Nq // block)
+    if idx_out is None:
+        idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
+    nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, max(Nk, 1), d, block, 1)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    _check(lib().hf_select_blocks_cached(_dev(Q, torch.bfloat16, "Q"), ctypes.byref(kp.c), Nq, block, r,
+                                         _dev(idx_out, torch.int32, "idx_out"),
+                                         _dev(scores_out, torch.float32, "scores_out")
+                                         if scores_out is not None else None,
+                                         ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
+           "hf_select_blocks_cached")
     return idx_out
 
 

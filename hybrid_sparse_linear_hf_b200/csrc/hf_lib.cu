@@ -95,6 +95,22 @@ size_t select_ws_bytes(int B, int H, int Nq, int Nk, int d, int block) {
          align256(static_cast<size_t>(bh) * ceil_div(Nk, block) * d * 4);
 }
 
+// scores and top-r from the pooled rows in the workspace
+template <int D>
+hf_status launch_score(const float* Qp, const float* Kp, int BH, int nQB, int nKB, int r, int32_t* idx,
+                       float* scores, cudaStream_t st) {
+  // the opt-in covers static + dynamic shared memory above the 48 KB default; set on
+  // every launch so that no size of nKB depends on it having been set before
+  const size_t smem = static_cast<size_t>(nKB) * hf::kSelQB * sizeof(float);
+  if (cudaFuncSetAttribute(hf::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return HF_ERR_CUDA;
+  const long long groups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
+  hf::score_select_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * groups), hf::kSelectThreads, smem,
+                               st>>>(Qp, Kp, nQB, nKB, r, idx, scores);
+  return launch_status();
+}
+
 template <int D>
 hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk, int block, int r,
                         int32_t* idx, float* scores, void* ws, cudaStream_t st) {
@@ -106,16 +122,26 @@ hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int 
       reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block, nQB,
       nKB, Qp, Kp);
   if (launch_status() != HF_OK) return HF_ERR_CUDA;
-  // the opt-in covers static + dynamic shared memory above the 48 KB default; set on
-  // every launch so that no size of nKB depends on it having been set before
-  const size_t smem = static_cast<size_t>(nKB) * hf::kSelQB * sizeof(float);
-  if (cudaFuncSetAttribute(hf::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return HF_ERR_CUDA;
-  const long long groups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
-  hf::score_select_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * groups), hf::kSelectThreads, smem,
-                               st>>>(Qp, Kp, nQB, nKB, r, idx, scores);
-  return launch_status();
+  return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st);
+}
+
+// selection over the pooled-key cache: Q pooled as above (no key blocks), key blocks from
+// the granule sums
+template <int D>
+hf_status launch_select_cached(const hf_bf16* Q, const hf_kpool* kp, int BH, int Nq, int Nk, int block, int r,
+                               int32_t* idx, float* scores, void* ws, cudaStream_t st) {
+  const int nQB = ceil_div(Nq, block), nKB = ceil_div(Nk, block);
+  float* Qp = static_cast<float*>(ws);
+  float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(BH) * nQB * D * 4));
+  hf::pool_blocks_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * nQB), hf::kPoolThreads, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(Q), nullptr, Nq, 0, block, nQB, 0, Qp, Kp);
+  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  constexpr int kWarpsPerCta = hf::kPoolThreads / 32;
+  const long long ctas = (static_cast<long long>(BH) * nKB + kWarpsPerCta - 1) / kWarpsPerCta;
+  hf::kpool_blocks_kernel<D><<<static_cast<unsigned>(ctas), hf::kPoolThreads, 0, st>>>(
+      kp->sums, kp->capacity, kp->head, kp->n_gran, kp->granule, block, nKB, BH, Kp);
+  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st);
 }
 
 // ---------------------------------------------------------------- two-stage select
@@ -378,6 +404,83 @@ HF_API hf_status hf_select_blocks(const hf_bf16* Q, const hf_bf16* K, int B, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_select<128>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s)
                   : launch_select<64>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s);
+}
+
+// ---------------------------------------------------------------- pooled-key cache
+HF_API hf_status hf_kpool_init(hf_kpool* kp, int B, int H, int d, int granule, int capacity, float* sums_dev) {
+  if (!kp || B < 1 || H < 1 || capacity < 1 || capacity > (1 << 30) || !sums_dev) return HF_ERR_INVALID_ARG;
+  if (granule < 1 || granule > 128 || (128 % granule) != 0) return HF_ERR_INVALID_ARG;
+  if (!supported_d(d)) return HF_ERR_UNSUPPORTED;
+  if (!aligned16(sums_dev)) return HF_ERR_ALIGNMENT;
+  if (static_cast<long long>(B) * H > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  kp->B = B;
+  kp->H = H;
+  kp->d = d;
+  kp->granule = granule;
+  kp->capacity = capacity;
+  kp->n_gran = 0;
+  kp->head = 0;
+  kp->sums = sums_dev;
+  return HF_OK;
+}
+
+HF_API hf_status hf_kpool_push(hf_kpool* kp, const hf_bf16* K_new, int n_tokens, int n_evict, void* stream) {
+  if (!kp || !kp->sums || kp->B < 1 || kp->H < 1 || kp->capacity < 1 || kp->granule < 1) return HF_ERR_INVALID_ARG;
+  if (!supported_d(kp->d)) return HF_ERR_UNSUPPORTED;
+  const int G = kp->granule, cap = kp->capacity;
+  if (n_tokens < 0 || n_evict < 0 || n_tokens % G != 0 || n_evict % G != 0) return HF_ERR_INVALID_ARG;
+  if (kp->n_gran < 0 || kp->n_gran > cap || kp->head < 0 || kp->head >= cap) return HF_ERR_INVALID_ARG;
+  const int ev = n_evict / G, n_new = n_tokens / G;
+  if (ev > kp->n_gran || kp->n_gran - ev + n_new > cap) return HF_ERR_INVALID_ARG;
+  if (n_new > 0 && !K_new) return HF_ERR_INVALID_ARG;
+  if (n_new > 0 && !aligned16(K_new)) return HF_ERR_ALIGNMENT;
+  const int head = (kp->head + ev) % cap, kept = kp->n_gran - ev;
+  if (n_new > 0) {
+    const long long BH = static_cast<long long>(kp->B) * kp->H;
+    constexpr int kGran128 = hf::kPoolThreads / (128 / 8), kGran64 = hf::kPoolThreads / (64 / 8);
+    const long long groups = (n_new + (kp->d == 128 ? kGran128 : kGran64) - 1) / (kp->d == 128 ? kGran128 : kGran64);
+    if (BH * groups > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+    const int base = (head + kept) % cap;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(K_new);
+    if (kp->d == 128)
+      hf::kpool_push_kernel<128><<<static_cast<unsigned>(BH * groups), hf::kPoolThreads, 0, s>>>(
+          K, n_tokens, G, n_new, base, cap, kp->sums);
+    else
+      hf::kpool_push_kernel<64><<<static_cast<unsigned>(BH * groups), hf::kPoolThreads, 0, s>>>(
+          K, n_tokens, G, n_new, base, cap, kp->sums);
+    if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  }
+  kp->head = head;
+  kp->n_gran = kept + n_new;
+  return HF_OK;
+}
+
+HF_API hf_status hf_select_blocks_cached(const hf_bf16* Q, const hf_kpool* kp, int Nq, int block, int r,
+                                         int32_t* idx_out, float* scores_out, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  if (!kp || !kp->sums || kp->B < 1 || kp->H < 1 || kp->granule < 1 || Nq < 0) return HF_ERR_INVALID_ARG;
+  if (kp->n_gran < 1 || kp->n_gran > kp->capacity || kp->head < 0 || kp->head >= kp->capacity)
+    return HF_ERR_INVALID_ARG;
+  if (!supported_d(kp->d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
+  if (block % kp->granule != 0) return HF_ERR_INVALID_ARG;
+  const long long nk = static_cast<long long>(kp->n_gran) * kp->granule;
+  if (nk > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  const int Nk = static_cast<int>(nk), B = kp->B, H = kp->H, d = kp->d;
+  const int nKB = ceil_div(Nk, block);
+  if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
+  if (nKB > hf::kMaxKeyBlocks) return HF_ERR_UNSUPPORTED;
+  if (Nq == 0) return HF_OK;
+  if (!Q || !idx_out) return HF_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(idx_out) || (scores_out && !aligned16(scores_out))) return HF_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < select_ws_bytes(B, H, Nq, Nk, d, block)) return HF_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128
+             ? launch_select_cached<128>(Q, kp, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s)
+             : launch_select_cached<64>(Q, kp, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s);
 }
 
 HF_API hf_status hf_select_blocks_two_stage(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk,

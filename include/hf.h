@@ -154,6 +154,46 @@ HF_API hf_status hf_select_blocks_two_stage(const hf_bf16* Q, const hf_bf16* K, 
                                             int32_t* idx_out, int32_t* frames_out, float* scores_out, void* ws,
                                             size_t ws_bytes, void* stream);
 
+/* Pooled-key cache of the sliding window: the window's keys as fp32 sums of `granule`
+ * consecutive tokens, in a ring of `capacity` sums per (b, h). A chunk step sums only the
+ * keys that enter the window (hf_kpool_push) and the selection pools its key blocks from
+ * the sums (hf_select_blocks_cached) instead of reading the window's K: with 8-token
+ * granules it reads a quarter of K's bytes. The window is the n_gran sums from ring slot
+ * head on, i.e. n_gran * granule key tokens. The library updates head and n_gran; the
+ * caller owns `sums` ([B][H][capacity][d] fp32, device). */
+typedef struct hf_kpool {
+  int B, H, d;
+  int granule;   /* tokens per sum; divides the block size and every push / evict count */
+  int capacity;  /* ring slots per (b, h) */
+  int n_gran;    /* sums in the window */
+  int head;      /* ring slot of the window's first sum */
+  float* sums;
+} hf_kpool;
+
+/* Empty cache. granule: 1, 2, 4, ... 128 (it must also divide the block size used with
+ * the cache); capacity >= 1; d in {64, 128}; sums 16-byte aligned. No device work.
+ * Errors: HF_ERR_INVALID_ARG, HF_ERR_UNSUPPORTED (d), HF_ERR_ALIGNMENT. */
+HF_API hf_status hf_kpool_init(hf_kpool* kp, int B, int H, int d, int granule, int capacity, float* sums_dev);
+
+/* The window moves: first the n_evict oldest key tokens leave it, then the n_tokens of
+ * K_new ([B][H][n_tokens][d] bf16, the newest keys, in order) enter it; the sums of their
+ * granules are written into the ring. n_tokens and n_evict are multiples of granule,
+ * n_evict at most the window, and the new window fits the capacity. Source: the sliding
+ * window of Hybrid Forcing (German technical summary sections 1 and 2 A: the window keeps
+ * the recent frames, the oldest leave it) with Light Forcing section 2.2's block mean
+ * pooling, computed from sums that stay valid while the window moves.
+ * Errors (kp unchanged): HF_ERR_INVALID_ARG, HF_ERR_ALIGNMENT, HF_ERR_CUDA. */
+HF_API hf_status hf_kpool_push(hf_kpool* kp, const hf_bf16* K_new, int n_tokens, int n_evict, void* stream);
+
+/* hf_select_blocks over the cached window: the same scores, blocks, order and outputs,
+ * for the window K of Nk = n_gran * granule tokens that the pushes put into kp (the key
+ * block means come from the granule sums, in fp32). block % granule == 0. ws:
+ * HF_WS_SELECT bytes for (Nq, Nk). Errors: those of hf_select_blocks, and
+ * HF_ERR_INVALID_ARG for an empty window or a block the granule does not divide. */
+HF_API hf_status hf_select_blocks_cached(const hf_bf16* Q, const hf_kpool* kp, int Nq, int block, int r,
+                                         int32_t* idx_out, float* scores_out, void* ws, size_t ws_bytes,
+                                         void* stream);
+
 /* Upper bound, in bytes, of the select workspace that hf_select_blocks_noalloc can
  * serve: a call is accepted when hf_workspace_size(HF_WS_SELECT, ...) for its shapes
  * is at most this (e.g. 12 heads x 4680 query x 32760 key tokens at d = 128, block

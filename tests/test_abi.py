@@ -159,3 +159,59 @@ def test_select_two_stage_validation():
     assert _sel2(Nq=0) == B.HF_OK
     n = hf.hf_workspace_size(B.HF_WS_SELECT_TWO_STAGE, 1, 12, 4680, 32760, 128, 128, 64)
     assert n == 12 * 37 * 128 * 4 + 12 * 256 * 128 * 4 * 4
+
+
+def _kp(**kw):
+    kp = B.HfKpoolC()
+    a = dict(B=1, H=2, d=64, G=8, cap=64, sums=A)
+    a.update(kw)
+    rc = hf.lib().hf_kpool_init(ctypes.byref(kp), a["B"], a["H"], a["d"], a["G"], a["cap"], a["sums"])
+    return rc, kp
+
+
+def test_kpool_validation():
+    assert _kp()[0] == B.HF_OK
+    rc, kp = _kp(G=16, cap=100)
+    assert rc == B.HF_OK and (kp.n_gran, kp.head, kp.granule, kp.capacity) == (0, 0, 16, 100)
+    assert _kp(G=3)[0] == B.HF_ERR_INVALID_ARG
+    assert _kp(G=256)[0] == B.HF_ERR_INVALID_ARG
+    assert _kp(cap=0)[0] == B.HF_ERR_INVALID_ARG
+    assert _kp(sums=None)[0] == B.HF_ERR_INVALID_ARG
+    assert _kp(d=32)[0] == B.HF_ERR_UNSUPPORTED
+    assert _kp(sums=A + 4)[0] == B.HF_ERR_ALIGNMENT
+    L = hf.lib()
+    _, kp = _kp()
+    # errors leave the cache unchanged; none of these reaches a launch
+    assert L.hf_kpool_push(ctypes.byref(kp), A, 12, 0, None) == B.HF_ERR_INVALID_ARG   # not whole granules
+    assert L.hf_kpool_push(ctypes.byref(kp), A, 0, 8, None) == B.HF_ERR_INVALID_ARG    # evicts more than the window
+    assert L.hf_kpool_push(ctypes.byref(kp), A, 65 * 8, 0, None) == B.HF_ERR_INVALID_ARG  # over capacity
+    assert L.hf_kpool_push(ctypes.byref(kp), None, 8, 0, None) == B.HF_ERR_INVALID_ARG
+    assert L.hf_kpool_push(ctypes.byref(kp), A + 2, 8, 0, None) == B.HF_ERR_ALIGNMENT
+    assert (kp.n_gran, kp.head) == (0, 0)
+    # evicting only is host bookkeeping: the ring head moves, wrapping at the capacity
+    kp.n_gran, kp.head = 40, 50
+    assert L.hf_kpool_push(ctypes.byref(kp), None, 0, 20 * 8, None) == B.HF_OK
+    assert (kp.n_gran, kp.head) == (20, (50 + 20) % 64)
+
+
+def test_select_cached_validation():
+    L = hf.lib()
+    _, kp = _kp()
+
+    def sel(kp_, **kw):
+        a = dict(Q=A, Nq=64, block=32, r=2, idx=A, scores=None, ws=A, ws_bytes=1 << 20)
+        a.update(kw)
+        return L.hf_select_blocks_cached(a["Q"], ctypes.byref(kp_), a["Nq"], a["block"], a["r"], a["idx"],
+                                         a["scores"], a["ws"], a["ws_bytes"], None)
+    assert sel(kp) == B.HF_ERR_INVALID_ARG            # empty window
+    kp.n_gran = 32                                    # 256 key tokens: 8 blocks of 32
+    assert sel(kp, Nq=0) == B.HF_OK
+    assert sel(kp, r=9) == B.HF_ERR_INVALID_ARG
+    assert sel(kp, block=48) == B.HF_ERR_UNSUPPORTED
+    _, kp16 = _kp(G=64)
+    kp16.n_gran = 4
+    assert sel(kp16, block=32) == B.HF_ERR_INVALID_ARG  # the granule does not divide the block
+    assert sel(kp, Q=A + 2) == B.HF_ERR_ALIGNMENT
+    assert sel(kp, ws_bytes=100) == B.HF_ERR_WORKSPACE
+    kp.head = 64
+    assert sel(kp) == B.HF_ERR_INVALID_ARG            # a corrupted head
