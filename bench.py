@@ -9,9 +9,10 @@ key blocks, state built from 60 evicted frames):
 Metric: query tokens/s per chunk step (whole job, all GPUs), with the roofline fraction
 of the dominant kernel (hf_hybrid_attn_fwd, tensor-bound) against the measured bf16
 peak. Legs reported beside the step: the 60-frame state build, the two-stage (frame,
-then block) selection, the attention at keep 1 / 0.5 / 0.25 / 0.125, a video's first 12
-chunks under the chunk-aware growth keep schedule, and the step end to end with its
-inputs copied from pinned host memory and O copied back. Inputs are
+then block) selection, the selection from the pooled-key cache (with the push of the
+chunk's keys), the attention at keep 1 / 0.5 / 0.25 / 0.125, a video's first 12 chunks
+under the chunk-aware growth keep schedule, and the step end to end with its inputs
+copied from pinned host memory and O copied back. Inputs are
 resident in HBM; L2 is flushed between timed steps (outside the timed events). Multi-GPU (torchrun): every rank runs its own chunk stream (weak
 scaling, no collective on the data path); time = max over ranks.
 
