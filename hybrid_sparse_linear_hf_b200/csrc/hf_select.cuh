@@ -1,4 +1,5 @@
-// Block scoring and top-r selection (hf_select_blocks, hf_select_blocks_two_stage).
+// Block scoring and top-r selection (hf_select_blocks, hf_select_blocks_two_stage,
+// hf_select_blocks_cached with hf_kpool_push).
 //
 // Source: "Light Forcing: Accelerating Autoregressive Video Diffusion via Sparse
 // Attention", German technical summary, section 2.2 (query and key tokens are
@@ -22,6 +23,8 @@
 // Two-stage selection: pool_blocks_kernel<d, true> also writes each key block's sums in
 // its first and next frame, pool_frames_kernel adds them into frame means, and
 // score_select2_kernel keeps frames first, then blocks within them (see there).
+// Pooled-key cache: kpool_push_kernel sums each granule of G new keys into a ring, and
+// kpool_blocks_kernel forms the window's key block means from those sums (see there).
 #pragma once
 
 #include "hf_ptx.cuh"
