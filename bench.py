@@ -209,13 +209,13 @@ def cpu_threads() -> int:
 
 
 # ----------------------------------------------------------------------------- oracle leg
-def oracle_sample(wl, x: dict, S0: torch.Tensor, z0: torch.Tensor, heads, ev_k, ev_v) -> float:
-    """Seconds the fp64 oracle takes for the whole step on the given heads (select,
-    hybrid attention, absorption of the step's evicted tokens)."""
+def oracle_sample(wl, x: dict, S0: torch.Tensor, z0: torch.Tensor, heads, ev_k, ev_v) -> dict:
+    """Seconds the fp64 oracle takes for the whole step on the given heads, per call:
+    {"select", "attention", "absorb"} (the absorption of the step's evicted tokens)."""
     import oracle
 
     f64 = lambda t: t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
-    total = 0.0
+    parts = {"select": 0.0, "attention": 0.0, "absorb": 0.0}
     for h in heads:
         Q = f64(x["Q"][:, h:h + 1])
         K = f64(x["K"][:, h:h + 1])
@@ -226,10 +226,15 @@ def oracle_sample(wl, x: dict, S0: torch.Tensor, z0: torch.Tensor, heads, ev_k, 
         Ve = f64(ev_v[:, h:h + 1])
         t0 = time.perf_counter()
         idx, _ = oracle.select_blocks(Q, K, wl.block, wl.r)
+        t1 = time.perf_counter()
         oracle.hybrid_attention(Q, K, V, idx, S, z, wl.block)
+        t2 = time.perf_counter()
         oracle.absorb(S, z, Ke, Ve)
-        total += time.perf_counter() - t0
-    return total
+        t3 = time.perf_counter()
+        parts["select"] += t1 - t0
+        parts["attention"] += t2 - t1
+        parts["absorb"] += t3 - t2
+    return parts
 
 
 REFERENCE_BUDGET_S = 150.0  # CPU seconds the whole reference run (warm-up + timed) aims at
@@ -237,8 +242,8 @@ REFERENCE_BUDGET_S = 150.0  # CPU seconds the whole reference run (warm-up + tim
 
 def oracle_step_sample(wl, x: dict, S0: torch.Tensor, z0: torch.Tensor, h: int, n_tiles: int, first_tile: int):
     """One bounded sample of the step on head h: the whole selection and absorption of the
-    head and the hybrid attention of n_tiles query blocks. Returns (seconds of selection +
-    absorption, seconds of the n_tiles attention tiles)."""
+    head and the hybrid attention of n_tiles query blocks. Returns the seconds of the
+    selection, of the absorption and of the n_tiles attention tiles."""
     import oracle
 
     f64 = lambda t: t.detach().cpu().to(torch.float64).numpy()  # noqa: E731
@@ -247,12 +252,13 @@ def oracle_step_sample(wl, x: dict, S0: torch.Tensor, z0: torch.Tensor, h: int, 
     Ke, Ve = f64(x["K_ev"][:, h:h + 1]), f64(x["V_ev"][:, h:h + 1])
     t0 = time.perf_counter()
     idx, _ = oracle.select_blocks(Q, K, wl.block, wl.r)
+    ta = time.perf_counter()
     oracle.absorb(S, z, Ke, Ve)
     t1 = time.perf_counter()
     for k in range(n_tiles):
         oracle.hybrid_attention_tile(Q, K, V, idx, S, z, wl.block, 0, 0, (first_tile + k) % wl.nQB)
     t2 = time.perf_counter()
-    return t1 - t0, t2 - t1
+    return ta - t0, t1 - ta, t2 - t1
 
 
 def run_reference(args, wl) -> None:
@@ -269,15 +275,19 @@ def run_reference(args, wl) -> None:
     S0 = torch.randn(wl.B, wl.H, wl.d, wl.d, generator=g).abs() * 50.0
     z0 = torch.rand(wl.B, wl.H, wl.d, generator=g) * 1e5
     # size the per-step sample from one probe (one query block) against the budget
-    t_fix, t_tile = oracle_step_sample(wl, x, S0, z0, 0, 1, 0)
+    t_sel, t_abs, t_tile = oracle_step_sample(wl, x, S0, z0, 0, 1, 0)
+    t_fix = t_sel + t_abs
     per_step = REFERENCE_BUDGET_S / max(1, args.steps + args.warmup)
     n_tiles = int(max(1, min(wl.nQB, (per_step - t_fix) / max(t_tile, 1e-9))))
     for i in range(args.warmup):
         oracle_step_sample(wl, x, S0, z0, i % wl.H, n_tiles, i * n_tiles)
-    times = []
+    times, parts = [], {"select": [], "attention": [], "absorb": []}
     for i in range(args.steps):
-        t_f, t_t = oracle_step_sample(wl, x, S0, z0, i % wl.H, n_tiles, i * n_tiles)
-        times.append((t_f + t_t / n_tiles * wl.nQB) * wl.H)
+        t_s, t_a, t_t = oracle_step_sample(wl, x, S0, z0, i % wl.H, n_tiles, i * n_tiles)
+        parts["select"].append(t_s * wl.H)
+        parts["absorb"].append(t_a * wl.H)
+        parts["attention"].append(t_t / n_tiles * wl.nQB * wl.H)
+        times.append(parts["select"][-1] + parts["absorb"][-1] + parts["attention"][-1])
     t_step = statistics.mean(times)
     value = wl.B * wl.Nq / t_step
     cores = cpu_threads()
@@ -289,7 +299,8 @@ def run_reference(args, wl) -> None:
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"fp64 numpy oracle per step: 1 of {wl.H} heads (its selection and the absorb "
                                    f"of {wl.Ne_step} evicted tokens, and the hybrid attention of {n_tiles} of its "
-                                   f"{wl.nQB} query blocks), scaled to all query blocks and heads"},
+                                   f"{wl.nQB} query blocks), scaled to all query blocks and heads",
+                         "ms_per_call": {k: statistics.mean(v) * 1e3 for k, v in parts.items()}},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -610,8 +621,12 @@ def run_gpu(args, wl) -> None:
         ev_k, ev_v = K_ev.cpu(), V_ev.cpu()
         xs = {k: x[k].cpu() for k in ("Q", "K", "V")}
         heads, spent = [], 0.0
+        per_call = {"select": 0.0, "attention": 0.0, "absorb": 0.0}
         for h in range(wl.H):
-            spent += oracle_sample(wl, xs, S.cpu(), z.cpu(), [h], ev_k, ev_v)
+            part = oracle_sample(wl, xs, S.cpu(), z.cpu(), [h], ev_k, ev_v)
+            for k in per_call:
+                per_call[k] += part[k]
+            spent += sum(part.values())
             heads.append(h)
             if spent >= 10.0:
                 break
@@ -619,7 +634,8 @@ def run_gpu(args, wl) -> None:
         line["cpu_baseline"] = {
             "value": wl.B * wl.Nq / t_cpu_step, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
             "sample": f"fp64 numpy oracle on {len(heads)} of {wl.H} heads (select + hybrid attention + absorb "
-                      f"of the step's {wl.Ne_step} evicted tokens), {spent:.1f} s, scaled to all heads"}
+                      f"of the step's {wl.Ne_step} evicted tokens), {spent:.1f} s, scaled to all heads",
+            "ms_per_call": {k: v / len(heads) * wl.H * 1e3 for k, v in per_call.items()}}
     print(json.dumps(line), flush=True)
 
 

@@ -18,3 +18,20 @@ def test_attention_flop_accounting():
     issued = bench.attn_issued_flops(idx, wl)
     assert issued == 4.0 * 128 * 128 * 128 * wl.r * 12 * 37 + 6.0 * 128 * 128 * 128 * 12 * 37
     assert issued > F
+
+
+def test_oracle_sample_times_every_call():
+    """The CPU baseline's oracle sample reports the selection, attention and absorption
+    separately (tiny workload, on the host)."""
+    import torch
+
+    from hybrid_sparse_linear_hf_b200.inputs import draw_step_inputs
+
+    wl = WORKLOADS["tiny"]
+    x = draw_step_inputs(wl, n_evicted=wl.Ne_step)
+    S0 = torch.zeros(wl.B, wl.H, wl.d, wl.d)
+    z0 = torch.zeros(wl.B, wl.H, wl.d)
+    parts = bench.oracle_sample(wl, x, S0, z0, [0], x["K_ev"], x["V_ev"])
+    assert set(parts) == {"select", "attention", "absorb"} and all(v > 0 for v in parts.values())
+    t_s, t_a, t_t = bench.oracle_step_sample(wl, x, S0, z0, 0, 2, 0)
+    assert t_s > 0 and t_a > 0 and t_t > 0
