@@ -160,7 +160,9 @@ HF_API hf_status hf_select_blocks_two_stage(const hf_bf16* Q, const hf_bf16* K, 
  * the sums (hf_select_blocks_cached) instead of reading the window's K: with 8-token
  * granules it reads a quarter of K's bytes. The window is the n_gran sums from ring slot
  * head on, i.e. n_gran * granule key tokens. The library updates head and n_gran; the
- * caller owns `sums` ([B][H][capacity][d] fp32, device). */
+ * caller owns `sums` ([B][H][capacity][d] fp32, device). A push writes ring slots that
+ * earlier calls may still read on the device: calls on one stream are ordered; calls on
+ * different streams must be ordered by the caller. */
 typedef struct hf_kpool {
   int B, H, d;
   int granule;   /* tokens per sum; divides the block size and every push / evict count */
