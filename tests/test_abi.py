@@ -215,3 +215,20 @@ def test_select_cached_validation():
     assert sel(kp, ws_bytes=100) == B.HF_ERR_WORKSPACE
     kp.head = 64
     assert sel(kp) == B.HF_ERR_INVALID_ARG            # a corrupted head
+
+
+def test_kpool_binding_checks_shapes_before_any_call():
+    """The Python binding rejects mismatched tensors on the host (no device needed)."""
+    import torch
+
+    kp = hf.HfKpool(torch.empty(0))
+    kp.c.B, kp.c.H, kp.c.d, kp.c.granule, kp.c.capacity = 1, 2, 64, 8, 16
+    with pytest.raises(ValueError):
+        hf.hf_kpool_push(kp, torch.empty(1, 3, 8, 64, dtype=torch.bfloat16))   # wrong head count
+    with pytest.raises(ValueError):
+        hf.hf_kpool_push(kp, torch.empty(1, 2, 8, 32, dtype=torch.bfloat16))   # wrong d
+    with pytest.raises(ValueError):
+        hf.hf_kpool_init(torch.empty(2, 16, 64), 8)                             # not [B,H,cap,d]
+    with pytest.raises(ValueError):
+        hf.hf_kpool_init(torch.empty(1, 2, 16, 64), 8)                          # a CPU tensor
+    assert kp.n_tokens == 0
