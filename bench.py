@@ -5,16 +5,21 @@ workload (B=1, H=12, d=128, 4680 queries, 32760-key window, block 128, top-64 of
 key blocks, state built from 60 evicted frames):
     hf_select_blocks      block mean pooling, scores, top-r          (2 kernels)
     hf_hybrid_attn_fwd    sparse attention + linear readout, summed  (1 kernel)
-    hf_absorb_evicted     the chunk step's 3 evicted frames -> state (2 kernels)
+    hf_absorb_evicted     the chunk step's 3 evicted frames -> state
 Metric: query tokens/s per chunk step (whole job, all GPUs), with the roofline fraction
 of the dominant kernel (hf_hybrid_attn_fwd, tensor-bound) against the measured bf16
 peak. Legs reported beside the step: the 60-frame state build, the two-stage (frame,
 then block) selection, the selection from the pooled-key cache (with the push of the
 chunk's keys), the attention at keep 1 / 0.5 / 0.25 / 0.125, a video's first 12 chunks
-under the chunk-aware growth keep schedule, and the step end to end with its inputs
-copied from pinned host memory and O copied back. Inputs are
-resident in HBM; L2 is flushed between timed steps (outside the timed events). Multi-GPU (torchrun): every rank runs its own chunk stream (weak
-scaling, no collective on the data path); time = max over ranks.
+under the chunk-aware growth keep schedule, the 1280x720-shaped step (attention,
+selection, 120-frame state build), and a streaming end-to-end step: the chunk's Q, K, V
+copied in from pinned host memory, the device-resident window shifted by the chunk, the
+evicted frames absorbed, O copied back.
+Inputs are resident in HBM. Between timed calls L2 is flushed: a 256 MiB buffer is
+written and then read, so that no dirty line of the flush is written back inside a timed
+kernel. Launches are enqueued without host synchronisation, so the host runs ahead and
+the CUDA events bracket device work only. Multi-GPU (torchrun): every rank runs its own
+chunk stream (weak scaling, no collective on the data path); time = max over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -26,9 +31,11 @@ from __future__ import annotations
 import argparse
 import dataclasses
 import faulthandler
+import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -46,13 +53,13 @@ from hybrid_sparse_linear_hf_b200.inputs import WORKLOADS, draw_step_inputs, fra
 METRIC = "hybrid attn query tokens/s per chunk step; % of bf16 tensor / HBM roofline"
 UNIT = "query tokens/s"
 WORKLOAD = "832x480"
+LARGE_WORKLOAD = "1280x720"
 L2_FLUSH_BYTES = 256 << 20
-LAUNCHES_PER_STEP = 5  # pool, score+select, hybrid attention, absorb partials, state reduce
-# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the current
-# hybrid_attn_kernel<128,128> on this workload, from one ncu capture of this script
-# (`ncu --set full --clock-control none -k regex:hybrid_attn -s 2 -c 1 ... bench.py
-# --steps 2 --warmup 3 --no-cpu-baseline`). Reset to None whenever the kernel changes.
-ATTN_TRAFFIC_BYTES = 161.3e6 + 12.8e6
+# The attention kernel's DRAM traffic per launch comes from its ncu summary in profiles/,
+# which records the hash of the kernel source it was taken on; a changed source makes
+# the recorded figure stale and the bench then reports no traffic.
+ATTN_PROFILE = os.path.join(ROOT, "profiles", "hybrid_attn_kernel_832x480.md")
+ATTN_SOURCES = [os.path.join(ROOT, "hybrid_sparse_linear_hf_b200", "csrc", f) for f in ("hf_attn.cuh", "hf_ptx.cuh")]
 # frames kept per query block by the two-stage selection leg (8 of the window's 21 frames:
 # at least 12 blocks each, so the 64 kept blocks always come from the kept frames)
 TWO_STAGE_FRAMES = 8
@@ -120,6 +127,38 @@ def select_bytes(wl) -> float:
 def absorb_bytes(wl, n_tokens) -> float:
     """K_ev and V_ev read once plus a read and a write of S and z."""
     return 2.0 * 2 * wl.B * wl.H * n_tokens * wl.d + 2 * 4.0 * wl.B * wl.H * (wl.d * wl.d + wl.d)
+
+
+def source_hash(paths) -> str:
+    """Hash of the code of the given C++/CUDA sources with comments and blank lines
+    removed, so that a change of comments only keeps a recorded measurement valid."""
+    h = hashlib.sha256()
+    for p in paths:
+        text = open(p).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in text.splitlines()]
+        h.update("\n".join(ln for ln in lines if ln.strip()).encode())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(md_path: str, sources) -> tuple:
+    """(DRAM bytes per launch or None, provenance) from an ncu summary that holds a line
+    ``| traffic (read + write) | X MB per launch |`` and ``kernel source hash: H``."""
+    cur = source_hash(sources)
+    try:
+        text = open(md_path).read()
+    except OSError:
+        return None, {"status": "no ncu summary", "kernel_source_hash": cur}
+    m_t = re.search(r"\|\s*traffic \(read \+ write\)\s*\|\s*([0-9.]+) MB per launch", text)
+    m_h = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", text)
+    prov = {"file": os.path.relpath(md_path, ROOT), "kernel_source_hash": cur,
+            "captured_on_hash": m_h.group(1) if m_h else None}
+    if not (m_t and m_h):
+        return None, dict(prov, status="summary lacks a traffic line or a source hash")
+    if m_h.group(1) != cur:
+        return None, dict(prov, status="stale: the kernel source changed since the ncu capture")
+    return float(m_t.group(1)) * 1e6, dict(prov, status="ncu dram__bytes_read.sum + dram__bytes_write.sum, "
+                                                       "one launch, same kernel source")
 
 
 def max_over_ranks(t_local: float, dist=None, device="cpu") -> float:
@@ -310,10 +349,94 @@ def config_dict(wl) -> dict:
     return {"workload": f"{wl.name} hybrid attention chunk step", "B": wl.B, "H": wl.H, "d": wl.d,
             "Nq": wl.Nq, "Nk": wl.Nk, "block": wl.block, "keep": wl.keep, "r": wl.r,
             "state_frames": wl.state_frames, "evict_frames_per_step": wl.evict_frames,
-            "l2": "flushed between timed steps (256 MiB write)", "parallelism": "independent streams per GPU"}
+            "l2": "flushed between timed calls (256 MiB written, then read back: no dirty line is left)",
+            "parallelism": "independent streams per GPU"}
 
 
 # ----------------------------------------------------------------------------- GPU leg
+class DeviceTimer:
+    """Times calls on one stream with CUDA events, an L2 flush before each call (a 256 MiB
+    write, then a read of it, so the flush's dirty lines are written back before the
+    timed call starts) and no host synchronisation between calls: the host enqueues
+    ahead of the device, so each event pair brackets device work only."""
+
+    def __init__(self, dev, stream):
+        self.dev, self.stream = dev, stream
+        self.buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush(self) -> None:
+        self.buf.fill_(1)
+        self.buf.view(torch.int64).sum()
+
+    def run(self, fn, n: int, warm: int = 2) -> list:
+        """Seconds of each of n calls of fn() (after `warm` untimed ones)."""
+        pairs = []
+        for k in range(warm + n):
+            self.flush()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            fn()
+            e1.record(self.stream)
+            if k >= warm:
+                pairs.append((e0, e1))
+        torch.cuda.synchronize(self.dev)
+        return [a.elapsed_time(b) * 1e-3 for a, b in pairs]
+
+
+def check_status(hf, where: str) -> None:
+    rc, word = hf.hf_query_status()
+    if rc != hf.HF_OK:
+        raise RuntimeError(f"device status after {where}: {hf.hf_status_string(rc)} ({word:#x})")
+
+
+def large_workload_leg(hf, dev, timer: DeviceTimer, peaks: dict, rank: int) -> dict:
+    """The 1280x720-shaped step (B=1, H=40, d=128, 10800 queries, 43200-key window, r=68,
+    state from 120 evicted frames): the state build, the selection and the attention,
+    each timed alone."""
+    wl = WORKLOADS[LARGE_WORKLOAD]
+    gen = torch.Generator(device=dev).manual_seed(wl.seed + 5000 + rank)
+    S = torch.empty(wl.B, wl.H, wl.d, wl.d, dtype=torch.float32, device=dev)
+    z = torch.empty(wl.B, wl.H, wl.d, dtype=torch.float32, device=dev)
+    st = hf.hf_state_init(S, z)
+    bK = frame_structured(gen, wl.B, wl.H, wl.Ne_state, wl.d, wl.tokens_per_frame, wl.w, device=dev)
+    bV = frame_structured(gen, wl.B, wl.H, wl.Ne_state, wl.d, wl.tokens_per_frame, wl.w, device=dev)
+    ws_b = torch.empty(hf.hf_workspace_size(hf.HF_WS_ABSORB, wl.B, wl.H, 0, wl.Ne_state, wl.d, 0, 0),
+                       dtype=torch.uint8, device=dev)
+    Sb, zb = torch.empty_like(S), torch.empty_like(z)
+    stb = hf.hf_state_init(Sb, zb)
+    t_build = timer.run(lambda: hf.hf_absorb_evicted(stb, bK, bV, ws=ws_b), n=3, warm=1)
+    hf.hf_absorb_evicted(st, bK, bV, ws=ws_b)
+    torch.cuda.synchronize(dev)
+    del bK, bV, ws_b, Sb, zb, stb
+    torch.cuda.empty_cache()
+    x = draw_step_inputs(wl, seed=rank_seed(wl.seed, rank), n_evicted=1, device=dev)
+    Q, K, V = x["Q"], x["K"], x["V"]
+    ws_s = torch.empty(hf.hf_workspace_size(hf.HF_WS_SELECT, wl.B, wl.H, wl.Nq, wl.Nk, wl.d, wl.block, wl.r),
+                       dtype=torch.uint8, device=dev)
+    idx = torch.empty(wl.B, wl.H, wl.nQB, wl.r, dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+    t_sel = timer.run(lambda: hf.hf_select_blocks(Q, K, wl.block, wl.r, idx_out=idx, ws=ws_s), n=5)
+    t_att = timer.run(lambda: hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wl.r, idx, st, O=O), n=5)
+    check_status(hf, "the 1280x720 leg")
+    F = attn_flops(idx.cpu().numpy(), wl)
+    ta, ts, tb = statistics.mean(t_att), statistics.mean(t_sel), statistics.mean(t_build)
+    out = {
+        "config": {"B": wl.B, "H": wl.H, "d": wl.d, "Nq": wl.Nq, "Nk": wl.Nk, "block": wl.block, "keep": wl.keep,
+                   "r": wl.r, "state_frames": wl.state_frames},
+        "hf_hybrid_attn_fwd": {"us": ta * 1e6, "flops_per_launch": F, "tflops": F / ta / 1e12,
+                               "frac": F / ta / 1e12 / peaks["bf16_tflops"]},
+        "hf_select_blocks": {"us": ts * 1e6, "bytes": select_bytes(wl),
+                             "hbm_frac": select_bytes(wl) / ts / 1e9 / peaks["hbm_gbs"]},
+        "hf_absorb_evicted_state_build": {"us": tb * 1e6, "tokens": wl.Ne_state,
+                                          "bytes": absorb_bytes(wl, wl.Ne_state),
+                                          "hbm_frac": absorb_bytes(wl, wl.Ne_state) / tb / 1e9 / peaks["hbm_gbs"]},
+        "step_query_tokens_per_s": wl.B * wl.Nq / (ta + ts),
+    }
+    del x, Q, K, V, O, idx, ws_s, S, z, st
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu(args, wl) -> None:
     import hybrid_sparse_linear_hf_b200 as hf
 
@@ -330,6 +453,8 @@ def run_gpu(args, wl) -> None:
     dev = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
+    timer = DeviceTimer(dev, stream)
+    peaks = load_peaks()
 
     log(f"rank {rank}/{world} on {dev}")
     # ---- inputs, drawn on the device (same recipe, device generator), resident in HBM
@@ -348,20 +473,9 @@ def run_gpu(args, wl) -> None:
     Sb = torch.empty_like(S)
     zb = torch.empty_like(z)
     stb = hf.hf_state_init(Sb, zb)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     torch.cuda.synchronize(dev)
     log("inputs drawn; timing the state build")
-    build_times = []
-    for i in range(4):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        hf.hf_absorb_evicted(stb, build_K, build_V, ws=ws_abs_build)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        if i > 0:
-            build_times.append(e0.elapsed_time(e1) * 1e-3)
-        log(f"state build {i}: {e0.elapsed_time(e1):.3f} ms")
+    build_times = timer.run(lambda: hf.hf_absorb_evicted(stb, build_K, build_V, ws=ws_abs_build), n=5, warm=2)
     hf.hf_absorb_evicted(st, build_K, build_V, ws=ws_abs_build)
     torch.cuda.synchronize(dev)
     del build_K, build_V, ws_abs_build, Sb, zb, stb
@@ -388,15 +502,13 @@ def run_gpu(args, wl) -> None:
 
     log("warm-up")
     for i in range(max(args.warmup, 3)):
-        flush.zero_()
+        timer.flush()
         step()
         if _VERBOSE:
             torch.cuda.synchronize(dev)
             log(f"warm-up step {i} done")
     torch.cuda.synchronize(dev)
-    rc, word = hf.hf_query_status()
-    if rc != hf.HF_OK:
-        raise RuntimeError(f"device status after warm-up: {hf.hf_status_string(rc)} ({word:#x})")
+    check_status(hf, "warm-up")
     idx_host = idx.cpu().numpy()
 
     events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
@@ -404,16 +516,16 @@ def run_gpu(args, wl) -> None:
         dist.barrier()
     torch.cuda.synchronize(dev)
     log("timed steps")
+    launches0 = hf.hf_launch_count()
     with ClockSampler(dev.index) as clk:
         for k in range(args.steps):
-            flush.zero_()
+            timer.flush()
             step(events[k])
         torch.cuda.synchronize(dev)
+    launches = hf.hf_launch_count() - launches0
     if dist:
         dist.barrier()
-    rc, word = hf.hf_query_status()
-    if rc != hf.HF_OK:
-        raise RuntimeError(f"device status after timing: {hf.hf_status_string(rc)} ({word:#x})")
+    check_status(hf, "timing")
     t_sel = [e[0].elapsed_time(e[1]) * 1e-3 for e in events]
     t_fwd = [e[1].elapsed_time(e[2]) * 1e-3 for e in events]
     t_abs = [e[2].elapsed_time(e[3]) * 1e-3 for e in events]
@@ -422,24 +534,14 @@ def run_gpu(args, wl) -> None:
 
     log(f"timed: {t_step_local * 1e3:.3f} ms/step; two-stage selection leg")
     # ---- two-stage (frame, then block) selection, timed alone beside the step
+    n_leg = max(3, min(args.steps, 50))
     ws_sel2 = torch.empty(hf.hf_workspace_size(hf.HF_WS_SELECT_TWO_STAGE, wl.B, wl.H, wl.Nq, wl.Nk, wl.d, wl.block,
                                                wl.r), dtype=torch.uint8, device=dev)
     idx2 = torch.empty_like(idx)
-    t_sel2 = []
-    n_sel2 = max(3, min(args.steps, 50))
-    for k in range(n_sel2 + 3):
-        flush.zero_()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        hf.hf_select_blocks_two_stage(Q, K, wl.block, wl.r, wl.tokens_per_frame, TWO_STAGE_FRAMES, idx_out=idx2,
-                                      ws=ws_sel2)
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        if k >= 3:
-            t_sel2.append(e0.elapsed_time(e1) * 1e-3)
-    rc, word = hf.hf_query_status()
-    if rc != hf.HF_OK:
-        raise RuntimeError(f"device status after the two-stage leg: {hf.hf_status_string(rc)} ({word:#x})")
+    t_sel2 = timer.run(lambda: hf.hf_select_blocks_two_stage(Q, K, wl.block, wl.r, wl.tokens_per_frame,
+                                                             TWO_STAGE_FRAMES, idx_out=idx2, ws=ws_sel2),
+                       n=n_leg, warm=3)
+    check_status(hf, "the two-stage leg")
     # ---- pooled-key cache: per step the chunk's keys enter the cache and the oldest chunk
     # leaves (hf_kpool_push), then the selection pools its key blocks from the granule sums
     log("pooled-key cache leg")
@@ -449,23 +551,11 @@ def run_gpu(args, wl) -> None:
         hf.hf_kpool_push(kp, K[:, :, c0:c0 + wl.Nq].contiguous())
     K_in = K[:, :, wl.Nk - wl.Nq:].contiguous()  # stands in for the chunk's new keys
     idx_c = torch.empty_like(idx)
-    t_push, t_selc = [], []
-    for k in range(n_sel2 + 3):
-        flush.zero_()
-        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        e0.record(stream)
-        hf.hf_kpool_push(kp, K_in, n_evict=wl.Nq)
-        e1.record(stream)
-        hf.hf_select_blocks_cached(Q, kp, wl.block, wl.r, idx_out=idx_c, ws=ws_sel)
-        e2.record(stream)
-        torch.cuda.synchronize(dev)
-        if k >= 3:
-            t_push.append(e0.elapsed_time(e1) * 1e-3)
-            t_selc.append(e1.elapsed_time(e2) * 1e-3)
+    t_push = timer.run(lambda: hf.hf_kpool_push(kp, K_in, n_evict=wl.Nq), n=n_leg, warm=3)
+    t_selc = timer.run(lambda: hf.hf_select_blocks_cached(Q, kp, wl.block, wl.r, idx_out=idx_c, ws=ws_sel),
+                       n=n_leg, warm=3)
     del kp_sums, K_in
-    rc, word = hf.hf_query_status()
-    if rc != hf.HF_OK:
-        raise RuntimeError(f"device status after the pooled-key cache leg: {hf.hf_status_string(rc)} ({word:#x})")
+    check_status(hf, "the pooled-key cache leg")
     # ---- sparsity sweep: the attention alone at other keep ratios (same inputs and state)
     log("sweep leg")
     sweep = {}
@@ -473,22 +563,11 @@ def run_gpu(args, wl) -> None:
         wk = wl.with_keep(keep)
         idx_k = torch.empty(wl.B, wl.H, wl.nQB, wk.r, dtype=torch.int32, device=dev)
         hf.hf_select_blocks(Q, K, wl.block, wk.r, idx_out=idx_k, ws=ws_sel)
-        ts = []
-        for k in range(12):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wk.r, idx_k, st, O=O)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            if k >= 2:
-                ts.append(e0.elapsed_time(e1) * 1e-3)
-        t_k = statistics.mean(ts)
+        t_k = statistics.mean(timer.run(lambda: hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wk.r, idx_k, st, O=O),
+                                        n=10))
         F_k = attn_flops(idx_k.cpu().numpy(), wk)
         sweep[f"{keep:g}"] = {"r": wk.r, "us": t_k * 1e6, "tflops": F_k / t_k / 1e12}
-    rc, word = hf.hf_query_status()
-    if rc != hf.HF_OK:
-        raise RuntimeError(f"device status after the sweep leg: {hf.hf_status_string(rc)} ({word:#x})")
+    check_status(hf, "the sweep leg")
     # ---- chunk-aware growth: the attention of a video's first chunks under the keep
     # schedule (chunk i's window holds the newest min(i + 1, full) chunks of keys)
     log("keep schedule leg")
@@ -507,78 +586,48 @@ def run_gpu(args, wl) -> None:
         Kc, Vc = kv_win[w.Nk]
         idx_c = torch.empty(wl.B, wl.H, wl.nQB, r_c, dtype=torch.int32, device=dev)
         hf.hf_select_blocks(Q, Kc, wl.block, r_c, idx_out=idx_c, ws=ws_sel)
-        tc = []
-        for k in range(5):
-            flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            hf.hf_hybrid_attn_fwd(Q, Kc, Vc, wl.block, r_c, idx_c, st, O=O)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-            if k >= 2:
-                tc.append(e0.elapsed_time(e1) * 1e-3)
-        return statistics.mean(tc) * 1e6
+        return statistics.mean(timer.run(lambda: hf.hf_hybrid_attn_fwd(Q, Kc, Vc, wl.block, r_c, idx_c, st, O=O),
+                                         n=3)) * 1e6
 
     us_s = [time_chunk(w, rc_) for w, rc_ in zip(wls, r_s)]
     us_u = [time_chunk(w, rc_) for w, rc_ in zip(wls, r_u)]
     del kv_win
-    rc, word = hf.hf_query_status()
-    if rc != hf.HF_OK:
-        raise RuntimeError(f"device status after the keep schedule leg: {hf.hf_status_string(rc)} ({word:#x})")
+    check_status(hf, "the keep schedule leg")
     schedule = {"s_base": SCHEDULE_S_BASE, "s_target": SCHEDULE_S_TARGET, "beta": beta_s, "nKB": nKB_s,
                 "r": r_s, "attn_us": [round(u, 1) for u in us_s], "attn_us_total": sum(us_s),
                 "uniform_r": r_u, "uniform_attn_us_total": sum(us_u)}
+
     log("end-to-end leg")
-    # ---- end to end through the public API with host buffers (pinned), copies timed
-    host = {k: v.cpu().pin_memory() for k, v in x.items()}
-    O_host = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = O_host.numel() * O_host.element_size()
-    n_e2e = max(3, min(args.steps, 20))
-    dQ, dK, dV, dKe, dVe = (torch.empty_like(x[k]) for k in ("Q", "K", "V", "K_ev", "V_ev"))
+    # ---- streaming end to end through the public API: per step the chunk's Q, K, V come
+    # from pinned host memory (on a copy stream, overlapping the previous step's compute),
+    # the device-resident window drops its oldest chunk (absorbed into the state) and takes
+    # the chunk's keys, then select + attention, and O goes back to pinned host memory.
+    e2e = streaming_e2e_leg(hf, wl, dev, stream, x, st, ws_sel, ws_abs, args, dist)
 
-    def e2e_step():
-        dQ.copy_(host["Q"], non_blocking=True)
-        dK.copy_(host["K"], non_blocking=True)
-        dV.copy_(host["V"], non_blocking=True)
-        dKe.copy_(host["K_ev"], non_blocking=True)
-        dVe.copy_(host["V_ev"], non_blocking=True)
-        hf.hf_select_blocks(dQ, dK, wl.block, wl.r, idx_out=idx, ws=ws_sel)
-        hf.hf_hybrid_attn_fwd(dQ, dK, dV, wl.block, wl.r, idx, st, O=O)
-        hf.hf_absorb_evicted(st, dKe, dVe, ws=ws_abs)
-        O_host.copy_(O, non_blocking=True)
-
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    if dist:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n_e2e):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    t_e2e = max_over_ranks(e0.elapsed_time(e1) * 1e-3 / n_e2e, dist, dev)
+    log("1280x720 leg")
+    del ws_sel, ws_abs, ws_sel2, idx2, idx_c
+    torch.cuda.empty_cache()
+    large = large_workload_leg(hf, dev, timer, peaks, rank) if not args.no_large else None
     if dist:
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return
 
-    peaks = load_peaks()
     F = attn_flops(idx_host, wl)
     fwd_mean = statistics.mean(t_fwd)
     achieved_tf = F / fwd_mean / 1e12
     sel_mean, abs_mean = statistics.mean(t_sel), statistics.mean(t_abs)
     build_mean = statistics.mean(build_times)
     value = job_throughput(world, wl.B, wl.Nq, t_step)
+    traffic, traffic_src = profile_traffic(ATTN_PROFILE, ATTN_SOURCES)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_dict(wl),
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                     "frac": achieved_tf / peaks["bf16_tflops"], "traffic": ATTN_TRAFFIC_BYTES,
+                     "frac": achieved_tf / peaks["bf16_tflops"], "traffic": traffic, "traffic_source": traffic_src,
                      "kernel": "hybrid_attn_kernel<128,128>", "flops_per_launch": F,
                      "issued_flops_per_launch": attn_issued_flops(idx_host, wl),
                      "peak_source": f"{peaks['source']} dense bf16 (burst)"},
@@ -609,11 +658,11 @@ def run_gpu(args, wl) -> None:
         },
         "sweep": {k: dict(v, frac=v["tflops"] / peaks["bf16_tflops"]) for k, v in sweep.items()},
         "keep_schedule": schedule,
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "large_workload": large,
+        "gpu_launches": launches,
+        "gpu_launches_source": "hf_launch_count() difference over the timed steps (the library's own launches)",
         "clocks": clk.summary(),
-        "e2e": {"value": job_throughput(world, wl.B, wl.Nq, t_e2e), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": n_e2e,
-                "note": "pinned host Q, K/V window, evicted K/V copied in and O copied out every step"},
+        "e2e": e2e,
     }
     log("cpu baseline")
     if world == 1 and not args.no_cpu_baseline:
@@ -639,6 +688,92 @@ def run_gpu(args, wl) -> None:
     print(json.dumps(line), flush=True)
 
 
+def streaming_e2e_leg(hf, wl, dev, stream, x, st, ws_sel, ws_abs, args, dist) -> dict:
+    """Streaming chunk steps end to end through the public API, timed on the device from
+    the first host-to-device copy to the last device-to-host copy. Per step: the chunk's
+    Q and its new K, V (Nq tokens each) are copied from pinned host memory on an upload
+    stream (double-buffered, so step k+1's copy overlaps step k's compute); the window
+    (device-resident, ping-pong buffers) drops its oldest Nq tokens, which are absorbed
+    into the state, and appends the chunk's keys and values; then the selection and the
+    hybrid attention of the chunk; O goes back to pinned host memory on a download
+    stream. Bytes: 3 x Nq x d bf16 per head in, Nq x d bf16 per head out."""
+    B, H, Nq, Nk, d = wl.B, wl.H, wl.Nq, wl.Nk, wl.d
+    shp = (B, H, Nq, d)
+    host_in = [torch.empty(shp, dtype=torch.bfloat16, pin_memory=True) for _ in range(3)]
+    host_in[0].copy_(x["Q"].cpu())
+    host_in[1].copy_(x["K"][:, :, Nk - Nq:].cpu())
+    host_in[2].copy_(x["V"][:, :, Nk - Nq:].cpu())
+    host_out = [torch.empty(shp, dtype=torch.bfloat16, pin_memory=True) for _ in range(2)]
+    dev_in = [[torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(3)] for _ in range(2)]
+    dev_out = [torch.empty(shp, dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    win_k = [x["K"].clone(), torch.empty_like(x["K"])]
+    win_v = [x["V"].clone(), torch.empty_like(x["V"])]
+    k_ev = torch.empty(shp, dtype=torch.bfloat16, device=dev)
+    v_ev = torch.empty(shp, dtype=torch.bfloat16, device=dev)
+    idx = torch.empty(B, H, wl.nQB, wl.r, dtype=torch.int32, device=dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    uploaded = [torch.cuda.Event() for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    downloaded = [torch.cuda.Event() for _ in range(2)]
+    state = {"k": 0, "cur": 0}
+
+    def e2e_step():
+        k, b = state["k"], state["k"] % 2
+        cur, nxt = state["cur"], 1 - state["cur"]
+        if k >= 2:
+            up.wait_event(computed[b])        # step k-2 has read this upload buffer
+        with torch.cuda.stream(up):
+            for i in range(3):
+                dev_in[b][i].copy_(host_in[i], non_blocking=True)
+            uploaded[b].record(up)
+        stream.wait_event(uploaded[b])
+        if k >= 2:
+            stream.wait_event(downloaded[b])  # O of step k-2 has left this output buffer
+        q, k_new, v_new = dev_in[b]
+        # the oldest chunk leaves the window and enters the state; the new chunk enters
+        k_ev.copy_(win_k[cur][:, :, :Nq])
+        v_ev.copy_(win_v[cur][:, :, :Nq])
+        win_k[nxt][:, :, :Nk - Nq].copy_(win_k[cur][:, :, Nq:])
+        win_v[nxt][:, :, :Nk - Nq].copy_(win_v[cur][:, :, Nq:])
+        win_k[nxt][:, :, Nk - Nq:].copy_(k_new)
+        win_v[nxt][:, :, Nk - Nq:].copy_(v_new)
+        hf.hf_absorb_evicted(st, k_ev, v_ev, ws=ws_abs)
+        hf.hf_select_blocks(q, win_k[nxt], wl.block, wl.r, idx_out=idx, ws=ws_sel)
+        hf.hf_hybrid_attn_fwd(q, win_k[nxt], win_v[nxt], wl.block, wl.r, idx, st, O=dev_out[b])
+        computed[b].record(stream)
+        down.wait_event(computed[b])
+        with torch.cuda.stream(down):
+            host_out[b].copy_(dev_out[b], non_blocking=True)
+            downloaded[b].record(down)
+        state["k"] += 1
+        state["cur"] = nxt
+
+    n_e2e = max(3, min(args.steps, 50))
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    up.wait_stream(stream)
+    down.wait_stream(stream)
+    e0.record(up)
+    for _ in range(n_e2e):
+        e2e_step()
+    stream.wait_stream(down)
+    stream.wait_stream(up)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t = max_over_ranks(e0.elapsed_time(e1) * 1e-3 / n_e2e, dist, dev)
+    world = dist.get_world_size() if dist else 1
+    nbytes = 2 * B * H * Nq * d
+    return {"value": job_throughput(world, B, Nq, t), "unit": UNIT, "h2d_bytes_per_step": 3 * nbytes,
+            "d2h_bytes_per_step": nbytes, "steps": n_e2e, "ms_per_step": t * 1e3,
+            "note": "streaming: per step the chunk's Q, K, V (4680 tokens) in from pinned host memory on an upload "
+                    "stream overlapping the previous step, window shift and absorption of the evicted chunk on "
+                    "the device, select + attention, O out to pinned host memory"}
+
+
 def main() -> None:
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -646,6 +781,7 @@ def main() -> None:
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["hf", "reference"], default="hf")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle CPU-baseline leg")
+    ap.add_argument("--no-large", action="store_true", help="skip the 1280x720 leg")
     ap.add_argument("--verbose", action="store_true", help="progress lines on stderr")
     ap.add_argument("--watchdog", type=float, default=0.0,
                     help="dump the Python stacks and exit if the run exceeds this many seconds")

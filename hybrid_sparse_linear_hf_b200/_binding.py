@@ -79,6 +79,7 @@ _SIGNATURES = {
     "hf_query_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_uint32)]),
     "hf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "hf_version": (ctypes.c_char_p, []),
+    "hf_launch_count": (ctypes.c_ulonglong, []),
     "hf_debug_inject_timeout": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_ulonglong]),
     "hf_debug_exp2": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                      ctypes.c_void_p]),
@@ -109,6 +110,11 @@ def hf_version() -> str:
     return lib().hf_version().decode()
 
 
+def hf_launch_count() -> int:
+    """Kernels the library has launched since it was loaded (host-side count)."""
+    return int(lib().hf_launch_count())
+
+
 def _check(rc: int, where: str) -> None:
     if rc != HF_OK:
         raise HfError(rc, where)
@@ -132,6 +138,27 @@ def _dev(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     return t.data_ptr()
+
+
+def _shape(t, shape, name: str) -> None:
+    """Host-side shape check of an optional tensor argument (before any device access)."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name} must have shape {tuple(int(x) for x in shape)}, got {tuple(t.shape)}")
+
+
+def _qkv_dims(Q: torch.Tensor, K: torch.Tensor, name_k: str = "K"):
+    """(B, H, Nq, Nk, d) of a query tensor [B,H,Nq,d] and a key tensor [B,H,Nk,d]."""
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 4:
+        raise ValueError("Q must be a 4-D tensor [B,H,Nq,d]")
+    B, H, Nq, d = Q.shape
+    if not isinstance(K, torch.Tensor) or K.dim() != 4 or tuple(K.shape[:2]) != (B, H) or K.shape[3] != d:
+        raise ValueError(f"{name_k} must be [B,H,Nk,d] with Q's B={B}, H={H} and d={d}, got "
+                         f"{tuple(K.shape) if isinstance(K, torch.Tensor) else type(K).__name__}")
+    return B, H, Nq, K.shape[2], d
 
 
 class HfState:
@@ -207,9 +234,10 @@ def hf_absorb_evicted(state: HfState, K_ev: torch.Tensor, V_ev: torch.Tensor, ws
 def hf_select_blocks(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, idx_out=None, scores_out=None,
                      ws=None, stream=None) -> torch.Tensor:
     """Top-r key blocks per query block: int32 [B,H,nQB,r] (ascending)."""
-    B, H, Nq, d = Q.shape
-    Nk = K.shape[2]
-    nQB = -(-Nq // block)
+    B, H, Nq, Nk, d = _qkv_dims(Q, K)
+    nQB, nKB = -(-Nq // block), -(-Nk // block)
+    _shape(idx_out, (B, H, nQB, r), "idx_out")
+    _shape(scores_out, (B, H, nQB, nKB), "scores_out")
     if idx_out is None:
         idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
     nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, Nk, d, block, r)
@@ -248,9 +276,15 @@ def hf_kpool_push(kp: HfKpool, K_new, n_evict: int = 0, stream=None) -> None:
 def hf_select_blocks_cached(Q: torch.Tensor, kp: HfKpool, block: int, r: int, idx_out=None, scores_out=None,
                             ws=None, stream=None) -> torch.Tensor:
     """hf_select_blocks over the cached window (its ``kp.n_tokens`` keys)."""
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 4:
+        raise ValueError("Q must be a 4-D tensor [B,H,Nq,d]")
     B, H, Nq, d = Q.shape
+    if (B, H, d) != (kp.c.B, kp.c.H, kp.c.d):
+        raise ValueError(f"Q's (B, H, d) = {(B, H, d)} must match the cache's {(kp.c.B, kp.c.H, kp.c.d)}")
     Nk = kp.n_tokens
-    nQB = -(-Nq // block)
+    nQB, nKB = -(-Nq // block), -(-Nk // block)
+    _shape(idx_out, (B, H, nQB, r), "idx_out")
+    _shape(scores_out, (B, H, nQB, nKB), "scores_out")
     if idx_out is None:
         idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
     nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, max(Nk, 1), d, block, 1)
@@ -269,9 +303,11 @@ def hf_select_blocks_two_stage(Q: torch.Tensor, K: torch.Tensor, block: int, r: 
                                stream=None) -> torch.Tensor:
     """Two-stage top-r key blocks per query block (frames, then blocks within them):
     int32 [B,H,nQB,r] (ascending). frames_out: optional int32 [B,H,nQB,n_frames]."""
-    B, H, Nq, d = Q.shape
-    Nk = K.shape[2]
-    nQB = -(-Nq // block)
+    B, H, Nq, Nk, d = _qkv_dims(Q, K)
+    nQB, nKB = -(-Nq // block), -(-Nk // block)
+    _shape(idx_out, (B, H, nQB, r), "idx_out")
+    _shape(frames_out, (B, H, nQB, n_frames), "frames_out")
+    _shape(scores_out, (B, H, nQB, nKB), "scores_out")
     if idx_out is None:
         idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
     nbytes = hf_workspace_size(HF_WS_SELECT_TWO_STAGE, B, H, Nq, Nk, d, block, r)
@@ -296,8 +332,12 @@ def hf_select_blocks_noalloc(Q: torch.Tensor, K: torch.Tensor, block: int, r: in
     ``idx_out`` [B,H,nQB,r] int32 is caller-provided, so nothing is allocated here either.
     The first call on a device does a one-off set-up (make it before any stream capture);
     calls on one device share the scratch, so calls that overlap in time race."""
-    B, H, Nq, d = Q.shape
-    Nk = K.shape[2]
+    B, H, Nq, Nk, d = _qkv_dims(Q, K)
+    nQB, nKB = -(-Nq // block), -(-Nk // block)
+    if idx_out is None:
+        raise ValueError("idx_out [B,H,nQB,r] int32 is required (nothing is allocated here)")
+    _shape(idx_out, (B, H, nQB, r), "idx_out")
+    _shape(scores_out, (B, H, nQB, nKB), "scores_out")
     _check(lib().hf_select_blocks_noalloc(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), B, H, Nq,
                                           Nk, d, block, r, _dev(idx_out, torch.int32, "idx_out"),
                                           _dev(scores_out, torch.float32, "scores_out")
@@ -325,8 +365,12 @@ def hf_keep_schedule(nKB, s_base: float, s_target: float):
 def hf_hybrid_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block: int, r: int,
                        idx: torch.Tensor, state: HfState, scale: float = 0.0, O=None, stream=None) -> torch.Tensor:
     """Hybrid attention output O [B,H,Nq,d] bf16 = sparse term + linear term."""
-    B, H, Nq, d = Q.shape
-    Nk = K.shape[2]
+    B, H, Nq, Nk, d = _qkv_dims(Q, K)
+    _shape(V, (B, H, Nk, d), "V")
+    _shape(idx, (B, H, -(-Nq // block), r), "idx")
+    _shape(O, (B, H, Nq, d), "O")
+    if state.shape != (B, H, d):
+        raise ValueError(f"the state's (B, H, d) = {state.shape} must match Q's {(B, H, d)}")
     if O is None:
         O = torch.empty_like(Q)
     _check(lib().hf_hybrid_attn_fwd(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"),

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -86,7 +87,15 @@ hf_status make_map(CUtensorMap* m, const void* base, int d, long long rows, long
   return r == CUDA_SUCCESS ? HF_OK : HF_ERR_CUDA;
 }
 
-hf_status launch_status() { return cudaGetLastError() == cudaSuccess ? HF_OK : HF_ERR_CUDA; }
+// Kernels this library instance has launched (reported by hf_launch_count).
+std::atomic<unsigned long long> g_launches{0};
+
+// Status of the launch just issued; a successful one is counted.
+hf_status launch_status() {
+  if (cudaGetLastError() != cudaSuccess) return HF_ERR_CUDA;
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  return HF_OK;
+}
 
 // ---------------------------------------------------------------- select
 size_t select_ws_bytes(int B, int H, int Nq, int Nk, int d, int block) {
@@ -290,21 +299,43 @@ static __device__ __align__(256) unsigned char g_select_scratch[HF_SELECT_NOALLO
 namespace {
 
 constexpr int kScratchMaxDevices = 64;
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kScratchMaxDevices] = {};
+// Per device: the context the address was looked up in, and the address. A symbol has
+// one copy per context, so a lookup made in another context (a non-primary context, or a
+// primary context created anew after cudaDeviceReset) is not reused.
+struct ScratchEntry {
+  CUcontext ctx = nullptr;
+  void* ptr = nullptr;
+};
+ScratchEntry g_scratch[kScratchMaxDevices];
 
-// Device address of g_select_scratch on the current device (set-up on first use).
+// Device address of g_select_scratch in the current context (set-up on first use there).
 hf_status select_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return HF_ERR_CUDA;
   if (dev < 0 || dev >= kScratchMaxDevices) return HF_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
+  static CtxGetCurrentFn ctx_get = nullptr;
+  if (!ctx_get) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return HF_ERR_CUDA;
+    ctx_get = reinterpret_cast<CtxGetCurrentFn>(fn);
+  }
+  // cudaGetDevice above made the device's primary context current when none was
+  CUcontext ctx = nullptr;
+  if (ctx_get(&ctx) != CUDA_SUCCESS || !ctx) return HF_ERR_CUDA;
+  ScratchEntry& e = g_scratch[dev];
+  if (!e.ptr || e.ctx != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || !p) return HF_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
+    e.ctx = ctx;
+    e.ptr = p;
   }
-  *out = g_scratch_ptr[dev];
+  *out = e.ptr;
   return HF_OK;
 }
 
@@ -605,12 +636,18 @@ HF_API hf_status hf_debug_inject_timeout(int kernel_id, int count, unsigned long
 HF_API hf_status hf_select_blocks_noalloc(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk,
                                           int d, int block, int r, int32_t* idx_out, float* scores_out,
                                           void* stream) {
-  // The same argument checks as hf_select_blocks, so that a rejected call never reaches
-  // the set-up; then the size check against the fixed scratch.
+  // Every argument check of hf_select_blocks, then the size check against the fixed
+  // scratch, all before the set-up: a rejected call makes no CUDA call at all.
   if (B < 1 || H < 1 || Nq < 0 || Nk < 1) return HF_ERR_INVALID_ARG;
   if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
-  if (r < 1 || r > ceil_div(Nk, block)) return HF_ERR_INVALID_ARG;
+  const int nKB = ceil_div(Nk, block);
+  if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
+  if (nKB > hf::kMaxKeyBlocks) return HF_ERR_UNSUPPORTED;
   if (Nq == 0) return HF_OK;
+  if (!Q || !K || !idx_out) return HF_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(idx_out) || (scores_out && !aligned16(scores_out)))
+    return HF_ERR_ALIGNMENT;
+  if (static_cast<long long>(B) * H * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
   const size_t need = select_ws_bytes(B, H, Nq, Nk, d, block);
   if (need > HF_SELECT_NOALLOC_SCRATCH_BYTES) return HF_ERR_WORKSPACE;
   void* scratch = nullptr;
@@ -619,5 +656,7 @@ HF_API hf_status hf_select_blocks_noalloc(const hf_bf16* Q, const hf_bf16* K, in
   return hf_select_blocks(Q, K, B, H, Nq, Nk, d, block, r, idx_out, scores_out, scratch,
                           HF_SELECT_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+HF_API unsigned long long hf_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 }  // extern "C"

@@ -184,6 +184,11 @@ HF_API hf_status hf_kpool_init(hf_kpool* kp, int B, int H, int d, int granule, i
  * window of Hybrid Forcing (German technical summary sections 1 and 2 A: the window keeps
  * the recent frames, the oldest leave it) with Light Forcing section 2.2's block mean
  * pooling, computed from sums that stay valid while the window moves.
+ * Ordering: kp->head and kp->n_gran move on the host when the push is issued, and the
+ * push's kernel overwrites the ring slots of the evicted keys. Every earlier
+ * hf_select_blocks_cached on the same ring must therefore be ordered before the push on
+ * the device: issue both on one stream, or make the push's stream wait on an event
+ * recorded after the select. The library does not detect a violation.
  * Errors (kp unchanged): HF_ERR_INVALID_ARG, HF_ERR_ALIGNMENT, HF_ERR_CUDA. */
 HF_API hf_status hf_kpool_push(hf_kpool* kp, const hf_bf16* K_new, int n_tokens, int n_evict, void* stream);
 
@@ -212,10 +217,15 @@ HF_API hf_status hf_select_blocks_cached(const hf_bf16* Q, const hf_kpool* kp, i
  * every device the library's kernels are loaded on, whether this call is used or not).
  *   - Shapes whose select workspace exceeds HF_SELECT_NOALLOC_SCRATCH_BYTES return
  *     HF_ERR_WORKSPACE before anything runs; use hf_select_blocks for those.
- *   - The first call on a device (that device current) does a one-off set-up: it looks
- *     up the scratch's device address, which may load the library's kernels on that
- *     device. Make that first call before any stream capture begins. A failed set-up
- *     returns HF_ERR_CUDA and is retried by the next call.
+ *   - The first call in a CUDA context (the device's primary context, or whichever
+ *     context is current) does a one-off set-up: it looks up the scratch's device
+ *     address in that context, which may load the library's kernels there. Make that
+ *     first call before any stream capture begins. The address is kept per device
+ *     together with the context it belongs to, and looked up again when the current
+ *     context differs (a symbol has one copy per context; after cudaDeviceReset the
+ *     primary context is a new one, so the first call after a reset is again a set-up
+ *     call). A failed set-up returns HF_ERR_CUDA and is retried by the next call.
+ *     Arguments the call rejects are rejected before the set-up, without any CUDA call.
  *   - Nothing in the scratch needs to start at zero: every byte a call reads was
  *     written earlier in that same call.
  *   - All calls on one device share the one scratch. Two calls whose kernels overlap
@@ -281,6 +291,11 @@ HF_API const char* hf_status_string(hf_status s);
 
 /* Library version string. */
 HF_API const char* hf_version(void);
+
+/* Number of kernels this library instance has launched since it was loaded (a host-side
+ * count of launches that returned without error, over all devices and streams). A
+ * caller reads it before and after a region to count the library's launches there. */
+HF_API unsigned long long hf_launch_count(void);
 
 /* TEST ONLY. Makes the next `count` launches of kernel `kernel_id` (1 = select,
  * 2 = absorb, 3 = attention) skip one internal barrier arrival, so that one wait runs

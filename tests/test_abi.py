@@ -232,3 +232,54 @@ def test_kpool_binding_checks_shapes_before_any_call():
     with pytest.raises(ValueError):
         hf.hf_kpool_init(torch.empty(1, 2, 16, 64), 8)                          # a CPU tensor
     assert kp.n_tokens == 0
+
+
+def test_binding_checks_every_tensor_shape_before_any_call():
+    """Every tensor the binding hands to the library is checked against the shapes that
+    Q (or the cache) implies, on the host, before a pointer is taken: a mismatched
+    buffer would otherwise be read or written past its end on the device."""
+    import torch
+
+    bf = torch.bfloat16
+    Q = torch.empty(1, 2, 100, 64, dtype=bf)
+    K = torch.empty(1, 2, 300, 64, dtype=bf)          # nQB = 4, nKB = 10 at block 32
+    i32 = lambda *s: torch.empty(*s, dtype=torch.int32)  # noqa: E731
+    with pytest.raises(ValueError, match="K must be"):
+        hf.hf_select_blocks(Q, torch.empty(1, 3, 300, 64, dtype=bf), 32, 2)
+    with pytest.raises(ValueError, match="K must be"):
+        hf.hf_select_blocks(Q, torch.empty(1, 2, 300, 128, dtype=bf), 32, 2)
+    with pytest.raises(ValueError, match="idx_out"):
+        hf.hf_select_blocks(Q, K, 32, 2, idx_out=i32(1, 2, 3, 2))
+    with pytest.raises(ValueError, match="scores_out"):
+        hf.hf_select_blocks(Q, K, 32, 2, idx_out=i32(1, 2, 4, 2), scores_out=torch.empty(1, 2, 4, 9))
+    with pytest.raises(ValueError, match="idx_out"):
+        hf.hf_select_blocks_two_stage(Q, K, 32, 2, 100, 2, idx_out=i32(1, 2, 4, 3))
+    with pytest.raises(ValueError, match="frames_out"):
+        hf.hf_select_blocks_two_stage(Q, K, 32, 2, 100, 2, frames_out=i32(1, 2, 4, 3))
+    with pytest.raises(ValueError, match="K must be"):
+        hf.hf_select_blocks_noalloc(Q, torch.empty(2, 2, 300, 64, dtype=bf), 32, 2, i32(1, 2, 4, 2))
+    with pytest.raises(ValueError, match="idx_out"):
+        hf.hf_select_blocks_noalloc(Q, K, 32, 2, i32(1, 2, 4, 3))
+    with pytest.raises(ValueError, match="scores_out"):
+        hf.hf_select_blocks_noalloc(Q, K, 32, 2, i32(1, 2, 4, 2), scores_out=torch.empty(1, 2, 4, 11))
+    # attention: V, idx, O and the state against Q and K
+    st = hf.HfState(torch.empty(0), torch.empty(0))
+    st.c.B, st.c.H, st.c.d = 1, 2, 64
+    V = torch.empty_like(K)
+    idx = i32(1, 2, 4, 2)
+    with pytest.raises(ValueError, match="V must"):
+        hf.hf_hybrid_attn_fwd(Q, K, torch.empty(1, 2, 299, 64, dtype=bf), 32, 2, idx, st)
+    with pytest.raises(ValueError, match="idx must"):
+        hf.hf_hybrid_attn_fwd(Q, K, V, 32, 2, i32(1, 2, 4, 3), st)
+    with pytest.raises(ValueError, match="O must"):
+        hf.hf_hybrid_attn_fwd(Q, K, V, 32, 2, idx, st, O=torch.empty(1, 2, 99, 64, dtype=bf))
+    st.c.H = 3
+    with pytest.raises(ValueError, match="state"):
+        hf.hf_hybrid_attn_fwd(Q, K, V, 32, 2, idx, st)
+    # the cached selection: Q against the cache
+    kp = hf.HfKpool(torch.empty(0))
+    kp.c.B, kp.c.H, kp.c.d, kp.c.granule, kp.c.capacity, kp.c.n_gran = 1, 2, 64, 8, 64, 32
+    with pytest.raises(ValueError, match="cache"):
+        hf.hf_select_blocks_cached(torch.empty(1, 2, 100, 128, dtype=bf), kp, 32, 2)
+    with pytest.raises(ValueError, match="idx_out"):
+        hf.hf_select_blocks_cached(Q, kp, 32, 2, idx_out=i32(1, 2, 4, 1))

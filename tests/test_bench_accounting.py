@@ -35,3 +35,28 @@ def test_oracle_sample_times_every_call():
     assert set(parts) == {"select", "attention", "absorb"} and all(v > 0 for v in parts.values())
     t_s, t_a, t_t = bench.oracle_step_sample(wl, x, S0, z0, 0, 2, 0)
     assert t_s > 0 and t_a > 0 and t_t > 0
+
+
+def test_traffic_comes_from_the_profile_of_the_same_kernel_source(tmp_path):
+    """roofline.traffic is the ncu figure of the profile only while the kernel source it
+    was captured on is unchanged (comments aside); otherwise it is reported as stale."""
+    src = tmp_path / "k.cuh"
+    src.write_text("// a comment\n__global__ void k() { int a = 1; }\n")
+    h = bench.source_hash([str(src)])
+    md = tmp_path / "prof.md"
+    md.write_text(f"kernel source hash: `{h}`\n\n| traffic (read + write) | 174.1 MB per launch |\n")
+    t, prov = bench.profile_traffic(str(md), [str(src)])
+    assert t == 174.1e6 and prov["captured_on_hash"] == h
+    src.write_text("// another comment\n\n__global__ void k() { int a = 1; }  // trailing\n")
+    assert bench.source_hash([str(src)]) == h          # comments and blank lines do not count
+    src.write_text("__global__ void k() { int a = 2; }\n")
+    t, prov = bench.profile_traffic(str(md), [str(src)])
+    assert t is None and prov["status"].startswith("stale")
+    t, prov = bench.profile_traffic(str(tmp_path / "missing.md"), [str(src)])
+    assert t is None
+
+
+def test_committed_attention_profile_parses():
+    t, prov = bench.profile_traffic(bench.ATTN_PROFILE, bench.ATTN_SOURCES)
+    assert prov["captured_on_hash"] is not None
+    assert t is None or 1e8 < t < 5e8

@@ -317,6 +317,21 @@ def test_streaming_832x480_20_steps():
     assert_state_close(f64(st.S[:, list(heads)]), f64(st.z[:, list(heads)]), S_o, z_o)
 
 
+def _check_every_tile(Og, Q64, K64, V64, idx, S64, z64, block, heads, what="O"):
+    """Every query block of the given heads against the oracle, tile by tile (each tile at
+    the output tolerances on its own)."""
+    Nq = Q64.shape[2]
+    n = 0
+    for b in range(Q64.shape[0]):
+        for h in heads:
+            sl = (slice(b, b + 1), slice(h, h + 1))
+            want = oracle.hybrid_attention(Q64[sl], K64[sl], V64[sl], idx[sl], S64[sl], z64[sl], block)
+            for I, (lo, hi) in enumerate(oracle.block_ranges(Nq, block)):
+                assert_output_close(Og[b, h, lo:hi], want[0, 0, lo:hi], what=f"{what} tile {(b, h, I)}")
+                n += 1
+    return n
+
+
 def _sample_tiles(wl, n, seed=0):
     rng = np.random.default_rng(seed)
     tiles = {(0, h, int(rng.integers(0, wl.nQB))) for h in rng.integers(0, wl.H, size=n)}
@@ -326,9 +341,9 @@ def _sample_tiles(wl, n, seed=0):
 
 
 @pytest.mark.parametrize("name", ["832x480"])
-def test_full_size_workload_sampled(name):
+def test_full_size_workload_every_tile(name):
     """The full 832x480-shaped step in the bench's launch configuration: every mask, the
-    whole state, and the outputs of sampled query blocks against the oracle."""
+    whole state, and the output of every one of the 444 query tiles against the oracle."""
     wl = WORKLOADS[name]
     x = draw_step_inputs(wl)
     Qd, Kd, Vd = x["Q"].to(DEV), x["K"].to(DEV), x["V"].to(DEV)
@@ -347,17 +362,16 @@ def test_full_size_workload_sampled(name):
     S_o, z_o = oracle.absorb_batch(f64(x["K_ev"]), f64(x["V_ev"]))
     assert_state_close(f64(st.S), f64(st.z), S_o, z_o)
     Og = f64(O)
-    for (b, h, I) in _sample_tiles(wl, 6):
-        lo, hi = I * wl.block, min((I + 1) * wl.block, wl.Nq)
-        want = oracle.hybrid_attention_tile(Q64, K64, V64, idx, S_o, z_o, wl.block, b, h, I)
-        assert_output_close(Og[b, h, lo:hi], want, what=f"O tile {(b, h, I)}")
+    n = _check_every_tile(Og, Q64, K64, V64, idx, f64(st.S), f64(st.z), wl.block, range(wl.H))
+    assert n == wl.B * wl.H * wl.nQB
 
 
-def test_1280x720_workload_sampled():
+def test_1280x720_workload_every_tile_of_four_heads():
     """The 1280x720-shaped step (40 heads, 10800 query x 43200 key tokens, block 128, r 68):
-    every mask and the outputs of sampled query blocks against the oracle. The state holds
-    2 evicted frames here (the attention reads S and z the same way whatever they absorbed;
-    the 120-frame build is checked on two heads below)."""
+    every mask, every query block of four heads (first, last and two between) and sampled
+    query blocks of the others against the oracle. The state holds 2 evicted frames here
+    (the attention reads S and z the same way whatever they absorbed; the 120-frame build
+    is checked on two heads below)."""
     wl = WORKLOADS["1280x720"]
     x = draw_step_inputs(wl, n_evicted=2 * wl.tokens_per_frame)
     Qd, Kd, Vd = x["Q"].to(DEV), x["K"].to(DEV), x["V"].to(DEV)
@@ -375,6 +389,9 @@ def test_1280x720_workload_sampled():
     S_o, z_o = oracle.absorb_batch(f64(x["K_ev"]), f64(x["V_ev"]))
     assert_state_close(f64(st.S), f64(st.z), S_o, z_o)
     Og = f64(O)
+    heads = (0, 13, 26, wl.H - 1)
+    n = _check_every_tile(Og, Q64, K64, V64, idx, f64(st.S), f64(st.z), wl.block, heads)
+    assert n == 4 * wl.nQB
     for (b, h, I) in _sample_tiles(wl, 6, seed=1):
         lo, hi = I * wl.block, min((I + 1) * wl.block, wl.Nq)
         want = oracle.hybrid_attention_tile(Q64, K64, V64, idx, S_o, z_o, wl.block, b, h, I)
@@ -425,7 +442,7 @@ def test_attention_online_rescale_mixed_rows():
 def test_bench_step_sequence_on_device_drawn_inputs():
     """The bench's loop (select -> hybrid attention -> absorb of the step's evicted
     frames, back to back without host syncs) on inputs drawn by the device generator,
-    checked on sampled tiles after several steps."""
+    every query tile of the last step checked against the oracle."""
     wl = WORKLOADS["832x480"]
     x = draw_step_inputs(wl, seed=123, n_evicted=wl.Ne_step, device=DEV)
     S = torch.empty(wl.B, wl.H, wl.d, wl.d, device=DEV)
@@ -447,7 +464,5 @@ def test_bench_step_sequence_on_device_drawn_inputs():
     Q64, K64, V64 = f64(x["Q"]), f64(x["K"]), f64(x["V"])
     idx_h = idx.cpu().numpy()
     Og = f64(O)
-    for (b, h, I) in _sample_tiles(wl, 4, seed=1):
-        lo, hi = I * wl.block, min((I + 1) * wl.block, wl.Nq)
-        want = oracle.hybrid_attention_tile(Q64, K64, V64, idx_h, f64(S_before), f64(z_before), wl.block, b, h, I)
-        assert_output_close(Og[b, h, lo:hi], want, what=f"O tile {(b, h, I)}")
+    n = _check_every_tile(Og, Q64, K64, V64, idx_h, f64(S_before), f64(z_before), wl.block, range(wl.H))
+    assert n == wl.B * wl.H * wl.nQB

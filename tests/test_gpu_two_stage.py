@@ -13,7 +13,7 @@ import torch
 import oracle
 import hybrid_sparse_linear_hf_b200 as hf
 from hybrid_sparse_linear_hf_b200.inputs import WORKLOADS, draw_step_inputs, frame_structured
-from tests.parity import SCORE_ABS, TIE_TOL, assert_masks_match, f64
+from tests.parity import SCORE_ABS, TIE_TOL, assert_masks_match, assert_output_close, f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -89,4 +89,12 @@ def test_two_stage_832x480_feeds_the_attention():
                               torch.from_numpy(idx).to(DEV), st)
     torch.cuda.synchronize()
     assert hf.hf_query_status()[0] == hf.HF_OK
-    assert torch.isfinite(O.float()).all()
+    # every query tile of the attention over the two-stage lists against the oracle
+    Q64, K64, V64 = f64(x["Q"]), f64(x["K"]), f64(x["V"])
+    S64, z64 = f64(st.S), f64(st.z)
+    Og = f64(O)
+    for h in range(wl.H):
+        sl = (slice(0, 1), slice(h, h + 1))
+        want = oracle.hybrid_attention(Q64[sl], K64[sl], V64[sl], idx[sl], S64[sl], z64[sl], wl.block)
+        for I, (lo, hi) in enumerate(oracle.block_ranges(wl.Nq, wl.block)):
+            assert_output_close(Og[0, h, lo:hi], want[0, 0, lo:hi], what=f"O tile {(0, h, I)}")

@@ -35,6 +35,13 @@ def test_noalloc_rejects_before_any_cuda_call():
     assert _noalloc_raw(Nk=0) == B.HF_ERR_INVALID_ARG
     assert _noalloc_raw(B=0) == B.HF_ERR_INVALID_ARG
     assert _noalloc_raw(Nq=0) == B.HF_OK  # empty query chunk: nothing to do, no set-up
+    # pointer, alignment and key-block limits are checked before the set-up too
+    assert _noalloc_raw(Q=None) == B.HF_ERR_INVALID_ARG
+    assert _noalloc_raw(idx=None) == B.HF_ERR_INVALID_ARG
+    assert _noalloc_raw(idx=A + 4) == B.HF_ERR_ALIGNMENT
+    assert _noalloc_raw(K=A + 2) == B.HF_ERR_ALIGNMENT
+    assert _noalloc_raw(scores=A + 8) == B.HF_ERR_ALIGNMENT
+    assert _noalloc_raw(Nk=8193 * 32, r=2) == B.HF_ERR_UNSUPPORTED  # more than 8192 key blocks
 
 
 def test_noalloc_size_limit():
