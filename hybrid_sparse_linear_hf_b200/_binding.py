@@ -68,6 +68,10 @@ _SIGNATURES = {
     "hf_hybrid_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
                            [ctypes.c_void_p, ctypes.POINTER(HfStateC), ctypes.c_float, ctypes.c_void_p,
                             ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_hybrid_attn_fwd_absorb": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
+                                  [ctypes.c_void_p, ctypes.POINTER(HfStateC), ctypes.c_float, ctypes.c_void_p,
+                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+                                   ctypes.c_size_t, ctypes.c_void_p]),
     "hf_kpool_init": (ctypes.c_int, [ctypes.POINTER(HfKpoolC)] + [ctypes.c_int] * 5 + [ctypes.c_void_p]),
     "hf_kpool_push": (ctypes.c_int, [ctypes.POINTER(HfKpoolC), ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_void_p]),
@@ -378,6 +382,33 @@ def hf_hybrid_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block:
                                     _dev(idx, torch.int32, "idx"), ctypes.byref(state.c), float(scale),
                                     _dev(O, torch.bfloat16, "O"), None, 0, _stream(stream)),
            "hf_hybrid_attn_fwd")
+    return O
+
+
+def hf_hybrid_attn_fwd_absorb(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block: int, r: int,
+                              idx: torch.Tensor, state: HfState, K_ev: torch.Tensor, V_ev: torch.Tensor,
+                              scale: float = 0.0, O=None, ws=None, stream=None) -> torch.Tensor:
+    """O [B,H,Nq,d] bf16 from the state as it stands, then the state absorbs K_ev, V_ev
+    [B,H,n,d] bf16 (one call: the absorption's partial sums overlap the attention's last
+    CTAs)."""
+    B, H, Nq, Nk, d = _qkv_dims(Q, K)
+    _shape(V, (B, H, Nk, d), "V")
+    _shape(idx, (B, H, -(-Nq // block), r), "idx")
+    _shape(O, (B, H, Nq, d), "O")
+    if state.shape != (B, H, d):
+        raise ValueError(f"the state's (B, H, d) = {state.shape} must match Q's {(B, H, d)}")
+    if K_ev.shape != V_ev.shape or K_ev.dim() != 4 or tuple(K_ev.shape[:2]) != (B, H) or K_ev.shape[3] != d:
+        raise ValueError("K_ev and V_ev must both be [B,H,n,d] matching Q")
+    n = K_ev.shape[2]
+    if O is None:
+        O = torch.empty_like(Q)
+    nbytes = hf_workspace_size(HF_WS_ABSORB, B, H, 0, n, d, 0, 0)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    _check(lib().hf_hybrid_attn_fwd_absorb(
+        _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V"), B, H, Nq, Nk, d,
+        block, r, _dev(idx, torch.int32, "idx"), ctypes.byref(state.c), float(scale), _dev(O, torch.bfloat16, "O"),
+        _dev(K_ev, torch.bfloat16, "K_ev") if n > 0 else None, _dev(V_ev, torch.bfloat16, "V_ev") if n > 0 else None,
+        n, ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)), "hf_hybrid_attn_fwd_absorb")
     return O
 
 

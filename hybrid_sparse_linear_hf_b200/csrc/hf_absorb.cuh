@@ -7,36 +7,41 @@
 // (a compact key-value state incrementally absorbs evicted tokens).
 //
 // Work split: the tokens of every (b,h) are cut into `nsplit` slices of whole
-// 64-token tiles; one CTA per (b,h,slice) accumulates its slice's phi(K)^T V in TMEM
-// and writes an fp32 partial; reduce_state_kernel adds the partials of a head to S
-// and z in slice order (deterministic).
+// 64-token tiles; one CTA per (b,h,slice) accumulates its slice's phi(K)^T V and writes
+// an fp32 partial; reduce_state_kernel adds the partials of a head to S and z in slice
+// order (deterministic).
 //
-// absorb_partial_kernel (576 threads, one CTA per SM):
-//   warp 0      TMA producer: K and V tiles [64 tokens][d] into a ring of stages taking
-//               the shared memory the A buffers leave (5 stages, 160 KB, at d = 128).
-//   warp 1      TMEM owner + MMA issuer: for each tile, D += A_hi x V and D += A_lo x V
-//               with M = 128 (d-index of S, zero-padded for d = 64), N = d, K = 64
-//               tokens; both operands MN-major (d contiguous). It waits only for the
-//               converters' "A written" barrier, which they arrive on after the tile's
-//               stage barrier (so the V tile has landed too).
+// absorb_partial_kernel (576 threads, one CTA per SM). The product is computed transposed,
+//   D[n][c] = sum_t V[t][n] * B[t][c],   B = [phi_hi | phi_lo]  (N = 2d columns),
+// so that one MMA of M = 128 (n, zero-padded rows for d = 64), N = 2d, K = 16 tokens covers
+// both halves of the split: S[k][n] = D[n][k] + D[n][d + k]. Both operands are MN-major
+// (the element index contiguous): A = V^T is the V tile as TMA wrote it, B is the
+// converted K tile.
+//   warp 0      TMA producer: the V and K tiles [64 tokens][d] of a tile into one ring
+//               stage laid out [V | K, then phi_hi over K | phi_lo], 64-column chunks of
+//               8 KB each, so the A chunks and the 2d/64 B chunks are 8 KB apart.
+//   warp 1      TMEM owner + MMA issuer: per tile 4 MMAs (K = 16 tokens each) into one of
+//               two TMEM accumulators of 2d columns. It waits only for the converters'
+//               "B written" barrier of the stage (they arrive after the stage barrier, so
+//               the V tile has landed too) and commits the stage back to the producer.
 //   warps 2..17 converters (four warps per SM sub-partition: the conversion is issue- and
-//               latency-bound, and it paces the whole kernel): phi(k) in fp32, split
-//               hi = bf16(phi), lo = bf16(phi - hi), z accumulated in fp32 registers. The
-//               A operand has the K tile's layout, so at d = 128 hi overwrites the K tile
-//               in place and lo goes to one of four lo buffers (a buffer is reused once
-//               the MMAs of four tiles back are done; one wait every second tile covers
-//               two tiles); at d = 64 (M = 128 needs 64 zero rows after the tile) hi and
-//               lo go to two separate zero-padded buffers. They also drain the
-//               accumulator: the tensor core's fp32 accumulation truncates, so a long
-//               chain of MMAs into one TMEM accumulator drifts (relative error grows with
-//               the chain length, ~2e-5 after 500 MMAs). The MMAs of every group of
-//               kAbsGroup tiles (32 MMAs) therefore go to one of two TMEM buffers, which
-//               the converters add into fp32 registers with round-to-nearest while the
-//               other buffer fills; the four warps that share a TMEM lane quarter take a
-//               quarter of the columns each. Epilogue: registers -> fp32 partial in the
-//               workspace.
-// Rows past the end of the token range are zero-filled by TMA; their phi is forced
-// to 0 (phi(0) = 1 would otherwise leak into z).
+//               MUFU-bound): phi(k) in fp32, split hi = bf16(phi), lo = bf16(phi - hi);
+//               hi overwrites the K chunk in place and lo goes to the stage's lo chunk; z
+//               is accumulated in fp32 registers. They also drain the accumulator: the
+//               tensor core's fp32 accumulation truncates, so a long chain of MMAs into one
+//               TMEM accumulator drifts (relative error grows with the chain length, ~2e-5
+//               after 500 MMAs). The MMAs of every group of kAbsGroup tiles (256 tokens)
+//               therefore go to one of two TMEM accumulators, which the converters add into
+//               fp32 registers with round-to-nearest while the other one fills; the four
+//               warps that share a TMEM lane quarter (rows n) take a quarter of the k
+//               columns each, hi and lo halves together. Epilogue: registers -> fp32 partial
+//               S[k][n] in the workspace.
+// Rows past the end of the token range are zero-filled by TMA; their phi is forced to 0
+// (phi(0) = 1 would otherwise leak into z).
+// Launch order: with `wait_first` the kernel waits for the previous grid of its stream
+// before its first load (its inputs may come from it); without, it reads K and V at once
+// (the caller guarantees they were complete before the previous grid started) and waits
+// only before it exits, so that the next grid of the stream sees the previous one done.
 #pragma once
 
 #include "hf_ptx.cuh"
@@ -45,30 +50,33 @@ namespace hf {
 
 constexpr uint32_t kKernAbsorb = 2;
 constexpr int kAbsTok = 64;        // tokens per tile
-constexpr int kAbsMaxStages = 8;   // K/V ring depth cap
+constexpr int kAbsMaxStages = 8;   // ring depth cap
 constexpr int kConvThreads = 512;  // converter warps 2..17
 constexpr int kAbsThreads = 64 + kConvThreads;
 constexpr int kAbsGroup = 4;       // tiles per TMEM accumulation chain
 
 template <int D>
 struct AbsorbCfg {
-  static constexpr int kChunks = D / 64;                  // 64-element column chunks of K/V
-  static constexpr int kChunkBytes = kAbsTok * 128;       // one chunk of a tile: 64 rows x 128 B
+  static constexpr int kChunks = D / 64;                  // 64-element column chunks of a tile
+  static constexpr int kChunkBytes = kAbsTok * 128;       // one chunk: 64 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes;      // K tile + V tile
-  static constexpr int kAOpBytes = 2 * kChunkBytes;       // A operand, M = 128 (2 chunks)
-  static constexpr bool kInPlace = D == 128;              // hi over the K tile
-  static constexpr int kABufBytes = kInPlace ? kAOpBytes : 2 * kAOpBytes;  // [lo] or [hi | lo]
-  static constexpr int kNA = kInPlace ? 4 : 2;            // A buffers
+  static constexpr int kStageBytes = 3 * kTileBytes;      // V | K (-> phi_hi) | phi_lo
+  static constexpr int kVOff = 0;
+  static constexpr int kKOff = kTileBytes;
+  static constexpr int kLoOff = 2 * kTileBytes;
+  static constexpr int kN = 2 * D;                        // MMA N: phi_hi and phi_lo columns
+  static constexpr uint32_t kAccCols = kN;                // TMEM columns per accumulator
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;     // two accumulators (256 or 512)
   static constexpr int kZredBytes = kConvThreads * 8 * 4;  // end-of-kernel z reduction (over the ring)
   static constexpr int kBudget = 232448 - 1024 - 1024;    // shared memory per CTA - alignment - static
-  static constexpr int kColsPerWarp = D / 4;              // drained accumulator columns per converter warp
-  static constexpr int kStagesFit = (kBudget - kNA * kABufBytes) / kStageBytes;
+  static constexpr int kStagesFit = kBudget / kStageBytes;
   static constexpr int kStages = kStagesFit < kAbsMaxStages ? kStagesFit : kAbsMaxStages;
   static_assert(kStages >= 2, "ring too small");
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kZredBytes <= kRingBytes, "z reduction must fit over the ring");
-  static constexpr int kDynSmem = 1024 + kRingBytes + kNA * kABufBytes;
+  static constexpr int kDynSmem = 1024 + kRingBytes;
+  static constexpr int kColsPerWarp = D / 4;              // k columns per converter warp in the drain
+  static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation is a power of two");
 };
 
 struct AbsorbParams {
@@ -77,6 +85,7 @@ struct AbsorbParams {
   int n_tokens;   // tokens per (b,h)
   int tiles_per_split;
   int nsplit;
+  int wait_first;  // 1: wait for the previous grid before the first load
   unsigned long long timeout_ns;
   int inject;     // test only: skip the first tile's load so a wait runs out
 };
@@ -86,15 +95,11 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     absorb_partial_kernel(const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                           AbsorbParams p) {
   using C = AbsorbCfg<D>;
-  constexpr int kAbsStages = C::kStages;
+  constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  uint8_t* abuf = smem + C::kRingBytes;  // [2][lo] (in place) or [2][hi | lo]
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
 
-  __shared__ uint64_t full_bar[kAbsStages], empty_bar[kAbsStages];
-  constexpr int NA = C::kNA;
-  __shared__ uint64_t afull_bar[NA], aempty_bar[NA];
+  __shared__ uint64_t full_bar[NS], empty_bar[NS], bfull_bar[NS];
   __shared__ uint64_t dfull_bar[2], dempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -108,13 +113,10 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
   volatile int* abort_flag = &abort_sh;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kAbsStages; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-    }
-    for (int a = 0; a < NA; ++a) {
-      mbar_init(&afull_bar[a], kConvThreads);
-      mbar_init(&aempty_bar[a], 1);
+      mbar_init(&bfull_bar[s], kConvThreads);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&dfull_bar[b], 1);
@@ -129,93 +131,77 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     tma_prefetch_desc(&mapV);
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, 256);
+    tmem_alloc(&tmem_base_sh, C::kTmemCols);
     tmem_relinquish();
-  }
-  if (!C::kInPlace && warp >= 2) {
-    // the upper 64 rows of the M = 128 A operand are zero padding for d = 64
-    for (int i = threadIdx.x - 64; i < NA * 2 * C::kChunkBytes / 16; i += kConvThreads) {
-      const int a = i / (2 * C::kChunkBytes / 16), rem = i % (2 * C::kChunkBytes / 16);
-      const int op = rem / (C::kChunkBytes / 16), u = rem % (C::kChunkBytes / 16);
-      reinterpret_cast<uint4*>(abuf + a * C::kABufBytes + op * C::kAOpBytes + C::kChunkBytes)[u] =
-          make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_d = tmem_base_sh;
+  // the next kernel of the stream (the slice reduction) may be scheduled now
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
+      if (p.wait_first) griddep_wait();
       int issued = 0;
       for (int i = 0; i < ntiles; ++i) {
-        const int s = i % kAbsStages, u = i / kAbsStages;
+        const int s = i % NS, u = i / NS;
         if (u >= 1 && !mbar_wait(&empty_bar[s], (u - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 1))
           break;
         if (*abort_flag) break;
         if (p.inject && i == 0) continue;  // test only: tile 0 never arrives
         uint8_t* st = ring + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&full_bar[s], C::kStageBytes);
+        mbar_arrive_expect_tx(&full_bar[s], 2 * C::kTileBytes);
         const int row = (tile0 + i) * kAbsTok;
 #pragma unroll
         for (int c = 0; c < C::kChunks; ++c) {
-          tma_load_3d(st + c * C::kChunkBytes, &mapK, &full_bar[s], c * 64, row, bh);
-          tma_load_3d(st + C::kTileBytes + c * C::kChunkBytes, &mapV, &full_bar[s], c * 64, row, bh);
+          tma_load_3d(st + C::kVOff + c * C::kChunkBytes, &mapV, &full_bar[s], c * 64, row, bh);
+          tma_load_3d(st + C::kKOff + c * C::kChunkBytes, &mapK, &full_bar[s], c * 64, row, bh);
         }
         issued = i + 1;
       }
       // drain: every issued copy must have landed before the CTA may exit
-      for (int i = max(0, issued - kAbsStages); i < issued; ++i) {
+      for (int i = max(0, issued - NS); i < issued; ++i) {
         if (p.inject && i == 0) continue;
-        mbar_wait_drain(&full_bar[i % kAbsStages], (i / kAbsStages) & 1, p.timeout_ns, (kKernAbsorb << 8) | 2);
+        mbar_wait_drain(&full_bar[i % NS], (i / NS) & 1, p.timeout_ns, (kKernAbsorb << 8) | 2);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
-      // descriptors built once; each MMA adds a constant offset to the start address
-      const uint64_t vdesc0 = sdesc_sw128(smem_u32(ring + C::kTileBytes), C::kChunkBytes, 1024);
-      const uint64_t kdesc0 = sdesc_sw128(smem_u32(ring), C::kChunkBytes, 1024);
-      const uint64_t adesc0 = sdesc_sw128(smem_u32(abuf), C::kChunkBytes, 1024);
+      // A = V^T (M = 128: the d columns of V, MN-major; for d = 64 the second M chunk is
+      // the next 8 KB of the stage, whose products land in TMEM rows that are never read),
+      // B = [phi_hi | phi_lo] (N = 2d, MN-major); chunks 8 KB apart, 8-row groups 1 KB apart
+      constexpr uint32_t idesc = idesc_bf16_f32(128, C::kN, true, true);
+      const uint64_t adesc0 = sdesc_sw128(smem_u32(ring + C::kVOff), C::kChunkBytes, 1024);
+      const uint64_t bdesc0 = sdesc_sw128(smem_u32(ring + C::kKOff), C::kChunkBytes, 1024);
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
-        const int s = i % kAbsStages, a = i % NA;
+        const int s = i % NS;
         const int g = i / kAbsGroup, b = g & 1;
         const bool first = (i % kAbsGroup) == 0;
         const bool last = (i % kAbsGroup) == kAbsGroup - 1 || i == ntiles - 1;
-        // A written implies the tile landed: the converters waited for the stage before arriving
-        ok = mbar_wait(&afull_bar[a], (i / NA) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 4);
+        ok = mbar_wait(&bfull_bar[s], (i / NS) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 4);
         if (ok && first && g >= 2)
           ok = mbar_wait(&dempty_bar[b], ((g >> 1) - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 9);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t bd = vdesc0 + static_cast<uint64_t>((s * C::kStageBytes) >> 4);
-        const uint64_t ab = adesc0 + static_cast<uint64_t>((a * C::kABufBytes) >> 4);
-        // A operands: hi (over the K tile of stage s, or the first half of buffer a), lo
-        const uint64_t a_hi = C::kInPlace ? kdesc0 + static_cast<uint64_t>((s * C::kStageBytes) >> 4) : ab;
-        const uint64_t a_lo = C::kInPlace ? ab : ab + static_cast<uint64_t>(C::kAOpBytes >> 4);
-        const uint32_t d_tmem = tmem_d + b * 128;
+        const uint64_t so = static_cast<uint64_t>((s * C::kStageBytes) >> 4);
+        const uint32_t d_tmem = tmem_d + b * C::kAccCols;
 #pragma unroll
-        for (int op = 0; op < 2; ++op) {
-#pragma unroll
-          for (int ks = 0; ks < kAbsTok / 16; ++ks)
-            umma_ss(d_tmem, (op == 0 ? a_hi : a_lo) + ks * 128, bd + ks * 128, idesc,
-                    (!first || op > 0 || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kAbsTok / 16; ++ks)  // 16 tokens = 16 rows of 128 B = 2048 B
+          umma_ss(d_tmem, adesc0 + so + ks * 128, bdesc0 + so + ks * 128, idesc, (!first || ks > 0) ? 1u : 0u);
         umma_commit(&empty_bar[s]);
-        if (NA == 2 || (i & 1)) umma_commit(&aempty_bar[a]);
         if (last) umma_commit(&dfull_bar[b]);
       }
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0, p.timeout_ns, (kKernAbsorb << 8) | 5);
     }
   } else {
-    // ---------------- converters + epilogue (256 threads) ----------------
-    const int t = threadIdx.x - 64;  // 0..255
+    // ---------------- converters + epilogue (512 threads) ----------------
+    const int t = threadIdx.x - 64;
     constexpr int kUnits = D / 8;    // 16-byte units per row
     constexpr int kPhases = kConvThreads / kUnits;
     constexpr int kRowsPerThread = kAbsTok / kPhases;
@@ -224,11 +210,12 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     const int chunk = ucol / 8;
     const uint32_t swz = static_cast<uint32_t>(((ucol % 8) ^ (phase & 7)) * 16);
     uint64_t zacc[4] = {0ull, 0ull, 0ull, 0ull};  // fp32 pairs: elements (2e, 2e+1) of the unit
-    // register accumulator: row m of phi(K)^T V (TMEM lane m), columns [col0, col0 + D/4);
-    // the four warps that share a TMEM lane quarter (warp % 4) take a quarter each
+    // register accumulator: row n of D (TMEM lane n), k columns [col0, col0 + NC) of both
+    // halves; the four warps that share a TMEM lane quarter (warp % 4) take a quarter each
     constexpr int NC = C::kColsPerWarp;
     const int quarter = warp & 3;
-    const int m = quarter * 32 + lane;
+    const int n_row = quarter * 32 + lane;
+    const bool drains = n_row < D;  // for d = 64 lanes 64..127 hold padding rows (warp-uniform)
     const int col0 = ((warp - 2) / 4) * NC;
     const uint32_t lane_base = tmem_d + (static_cast<uint32_t>(quarter * 32) << 16);
     float acc[NC];
@@ -244,13 +231,17 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
                       mbar_wait(&dfull_bar[b], (g >> 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 8)))
         return false;
       tc_fence_after();
-      {
-        uint32_t r[NC];
-        tmem_ld_cols<NC>(lane_base + b * 128 + col0, r);
-        tmem_wait_ld();
-        reg_fence<NC>(r);
+      if (drains) {
+        // the hi half, then the lo half (one half in registers at a time)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) acc[j] += __uint_as_float(r[j]);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t r[NC];
+          tmem_ld_cols<NC>(lane_base + b * C::kAccCols + half * D + col0, r);
+          tmem_wait_ld();
+          reg_fence<NC>(r);
+#pragma unroll
+          for (int j = 0; j < NC; ++j) acc[j] += __uint_as_float(r[j]);
+        }
       }
       tc_fence_before();
       mbar_arrive(&dempty_bar[b]);
@@ -274,28 +265,17 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       lo = pack_bf16x2(r0, r1);
     };
     for (int i = 0; i < ntiles && ok; ++i) {
-      const int s = i % kAbsStages, a = i % NA;
-      ok = mbar_wait(&full_bar[s], (i / kAbsStages) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 6);
-      // A buffer a is free once the MMAs of tile i - NA are done. With four buffers one wait
-      // every second tile suffices: at even i, MMA(i - 3) done covers tiles i and i + 1.
-      if (NA == 2) {
-        if (ok && i >= 2)
-          ok = mbar_wait(&aempty_bar[a], ((i >> 1) - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 7);
-      } else if (ok && i >= NA && (i & 1) == 0) {
-        const int t = i - NA + 1;
-        ok = mbar_wait(&aempty_bar[t % NA], (t / NA) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 7);
-      }
-      ok = __all_sync(0xffffffffu, ok);  // the warp stays converged for the collective drain
+      const int s = i % NS;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&full_bar[s], (i / NS) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 6));
       if (!ok) break;
-      uint8_t* ktile = ring + s * C::kStageBytes;
-      uint8_t* ahi = C::kInPlace ? ktile : abuf + a * C::kABufBytes;
-      uint8_t* alo = C::kInPlace ? abuf + a * C::kABufBytes : ahi + C::kAOpBytes;
+      uint8_t* stage = ring + s * C::kStageBytes;
       const int valid = min(kAbsTok, p.n_tokens - (tile0 + i) * kAbsTok);
 #pragma unroll
       for (int k = 0; k < kRowsPerThread; ++k) {
         const int row = phase + k * kPhases;
         const uint32_t off = chunk * C::kChunkBytes + row * 128 + swz;
-        const uint4 kv = *reinterpret_cast<const uint4*>(ktile + off);
+        const uint4 kv = *reinterpret_cast<const uint4*>(stage + C::kKOff + off);
         uint32_t hi[4], lo[4];
         if (valid == kAbsTok || row < valid) {
           convert_pair(kv.x, zacc[0], hi[0], lo[0]);
@@ -307,13 +287,13 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) hi[e] = lo[e] = 0u;
         }
-        *reinterpret_cast<uint4*>(ahi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(alo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(stage + C::kKOff + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(stage + C::kLoOff + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       fence_proxy_async_smem();
-      mbar_arrive(&afull_bar[a]);
+      mbar_arrive(&bfull_bar[s]);
       // once group g is fully converted, drain group g - 1 (one group of lag keeps the
-      // tensor core busy on the other buffer)
+      // tensor core busy on the other accumulator)
       const int g = i / kAbsGroup;
       const bool group_done = (i % kAbsGroup) == kAbsGroup - 1 || i == ntiles - 1;
       if (group_done && g >= 1) {
@@ -324,10 +304,10 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     if (ok) {
       for (int g = flushed; g < ngroups && ok; ++g) ok = flush_group(g);
     }
-    // z partial: reduce the kPhases row phases of each unit column (scratch over the ring,
-    // idle now: every tile has been converted and, once the last group was drained, every
-    // MMA is done)
+    // every MMA is done once the last group was drained (or the CTA gave up): the ring is
+    // idle and holds the z reduction
     float* zred = reinterpret_cast<float*>(ring);  // [kConvThreads][8]
+    named_bar_sync(1, kConvThreads);
 #pragma unroll
     for (int e = 0; e < 4; ++e) f32x2_split(zacc[e], zred[t * 8 + 2 * e], zred[t * 8 + 2 * e + 1]);
     named_bar_sync(1, kConvThreads);
@@ -337,12 +317,12 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       for (int ph = 0; ph < kPhases; ++ph) zs += zred[(ph * kUnits + uc) * 8 + e];
       p.part_z[(static_cast<size_t>(bh) * p.nsplit + split) * D + t] = zs;
     }
-    // S partial: row m, columns [col0, col0 + D/4) of this slice's phi(K)^T V
-    if (ok && m < D) {
-      float* dst = p.part_S + ((static_cast<size_t>(bh) * p.nsplit + split) * D + m) * D + col0;
+    // S partial: S[k][n] for n = this lane's row and k in [col0, col0 + NC) (for each k the
+    // warp's 32 lanes write 32 consecutive n: 128-byte stores)
+    if (ok && drains) {
+      float* dst = p.part_S + (static_cast<size_t>(bh) * p.nsplit + split) * D * D + n_row;
 #pragma unroll
-      for (int j = 0; j < NC; j += 4)
-        *reinterpret_cast<float4*>(dst + j) = make_float4(acc[j], acc[j + 1], acc[j + 2], acc[j + 3]);
+      for (int j = 0; j < NC; ++j) dst[static_cast<size_t>(col0 + j) * D] = acc[j];
     }
   }
 
@@ -351,8 +331,10 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_d, 256);
+    tmem_dealloc(tmem_d, C::kTmemCols);
   }
+  // the grid completes only after the previous one (see the file comment)
+  if (!p.wait_first) griddep_wait();
 }
 
 // S[bh] += sum_s part_S[bh][s], z[bh] += sum_s part_z[bh][s], slices in order.
@@ -362,6 +344,8 @@ __global__ void __launch_bounds__(256) reduce_state_kernel(float* __restrict__ S
                                                            const float* __restrict__ part_z, int nsplit) {
   constexpr int kVec4PerHead = D * D / 4;
   constexpr int kCtasPerHead = (kVec4PerHead + 255) / 256;
+  // the partials come from the previous grid; S and z may still be read by the one before
+  griddep_wait();
   const int bh = blockIdx.x / kCtasPerHead;
   const int e4 = (blockIdx.x % kCtasPerHead) * 256 + threadIdx.x;
   if (e4 < kVec4PerHead) {
@@ -374,7 +358,7 @@ __global__ void __launch_bounds__(256) reduce_state_kernel(float* __restrict__ S
       float4 v[kBatch];
 #pragma unroll
       for (int u = 0; u < kBatch; ++u)
-        if (s0 + u < nsplit) v[u] = __ldg(p4 + static_cast<size_t>(s0 + u) * kVec4PerHead);
+        if (s0 + u < nsplit) v[u] = __ldcg(p4 + static_cast<size_t>(s0 + u) * kVec4PerHead);
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         if (s0 + u < nsplit) {
@@ -389,7 +373,7 @@ __global__ void __launch_bounds__(256) reduce_state_kernel(float* __restrict__ S
   }
   if (blockIdx.x % kCtasPerHead == 0 && threadIdx.x < D) {
     float acc = z[static_cast<size_t>(bh) * D + threadIdx.x];
-    for (int s = 0; s < nsplit; ++s) acc += part_z[(static_cast<size_t>(bh) * nsplit + s) * D + threadIdx.x];
+    for (int s = 0; s < nsplit; ++s) acc += __ldcg(part_z + (static_cast<size_t>(bh) * nsplit + s) * D + threadIdx.x);
     z[static_cast<size_t>(bh) * D + threadIdx.x] = acc;
   }
 }

@@ -152,6 +152,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  // Q, K, V, idx, S and z may come from the previous grid of the stream; the next grid may
+  // be scheduled once every CTA of this one has started (it then fills the SMs that this
+  // grid's last CTAs leave)
+  griddep_wait();
+  griddep_launch_dependents();
 
   if (warp < 4) {
    // warpgroup 0: producers and MMA issuer give registers to the softmax warpgroups

@@ -97,6 +97,31 @@ hf_status launch_status() {
   return HF_OK;
 }
 
+// Launches `kernel` with programmatic stream serialisation: it may be scheduled before the
+// previous kernel of the stream has finished (once every CTA of that one has started);
+// each kernel of the library waits for its predecessor (griddep_wait) before it reads
+// anything that one may have written. The launch is counted on success.
+template <typename... KArgs, typename... Args>
+hf_status launch_pdl(void (*kernel)(KArgs...), long long grid, int block, size_t smem, cudaStream_t st,
+                     Args... args) {
+  if (grid < 1 || grid > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(block));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return HF_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 // ---------------------------------------------------------------- select
 size_t select_ws_bytes(int B, int H, int Nq, int Nk, int d, int block) {
   const long long bh = static_cast<long long>(B) * H;
@@ -115,9 +140,8 @@ hf_status launch_score(const float* Qp, const float* Kp, int BH, int nQB, int nK
                            static_cast<int>(smem)) != cudaSuccess)
     return HF_ERR_CUDA;
   const long long groups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
-  hf::score_select_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * groups), hf::kSelectThreads, smem,
-                               st>>>(Qp, Kp, nQB, nKB, r, idx, scores);
-  return launch_status();
+  return launch_pdl(hf::score_select_kernel<D>, static_cast<long long>(BH) * groups, hf::kSelectThreads, smem, st, Qp,
+                    Kp, nQB, nKB, r, idx, scores);
 }
 
 template <int D>
@@ -127,10 +151,10 @@ hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int 
   float* Qp = static_cast<float*>(ws);
   float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(BH) * nQB * D * 4));
   const long long grid1 = static_cast<long long>(BH) * (nQB + nKB);
-  hf::pool_blocks_kernel<D><<<static_cast<unsigned>(grid1), hf::kPoolThreads, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block, nQB,
-      nKB, Qp, Kp);
-  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  if (launch_pdl(hf::pool_blocks_kernel<D>, grid1, hf::kPoolThreads, 0, st, reinterpret_cast<const __nv_bfloat16*>(Q),
+                 reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block, nQB, nKB, Qp, Kp, 0,
+                 static_cast<float*>(nullptr)) != HF_OK)
+    return HF_ERR_CUDA;
   return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st);
 }
 
@@ -142,14 +166,15 @@ hf_status launch_select_cached(const hf_bf16* Q, const hf_kpool* kp, int BH, int
   const int nQB = ceil_div(Nq, block), nKB = ceil_div(Nk, block);
   float* Qp = static_cast<float*>(ws);
   float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(BH) * nQB * D * 4));
-  hf::pool_blocks_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * nQB), hf::kPoolThreads, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(Q), nullptr, Nq, 0, block, nQB, 0, Qp, Kp);
-  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  if (launch_pdl(hf::pool_blocks_kernel<D>, static_cast<long long>(BH) * nQB, hf::kPoolThreads, 0, st,
+                 reinterpret_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(nullptr), Nq, 0, block,
+                 nQB, 0, Qp, Kp, 0, static_cast<float*>(nullptr)) != HF_OK)
+    return HF_ERR_CUDA;
   constexpr int kWarpsPerCta = hf::kPoolThreads / 32;
   const long long ctas = (static_cast<long long>(BH) * nKB + kWarpsPerCta - 1) / kWarpsPerCta;
-  hf::kpool_blocks_kernel<D><<<static_cast<unsigned>(ctas), hf::kPoolThreads, 0, st>>>(
-      kp->sums, kp->capacity, kp->head, kp->n_gran, kp->granule, block, nKB, BH, Kp);
-  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  if (launch_pdl(hf::kpool_blocks_kernel<D>, ctas, hf::kPoolThreads, 0, st, static_cast<const float*>(kp->sums),
+                 kp->capacity, kp->head, kp->n_gran, kp->granule, block, nKB, BH, Kp) != HF_OK)
+    return HF_ERR_CUDA;
   return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st);
 }
 
@@ -176,21 +201,21 @@ hf_status launch_select2(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int
   base += align256(static_cast<size_t>(BH) * nKB * 2 * D * 4);
   float* Kf = reinterpret_cast<float*>(base);
   const long long grid1 = static_cast<long long>(BH) * (nQB + nKB);
-  hf::pool_blocks_kernel<D, true><<<static_cast<unsigned>(grid1), hf::kPoolThreads, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block, nQB,
-      nKB, Qp, Kp, T, Kpart);
-  if (launch_status() != HF_OK) return HF_ERR_CUDA;
-  hf::pool_frames_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * W), D, 0, st>>>(Kpart, Nk, block, T,
-                                                                                                nKB, W, Kf);
-  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  if (launch_pdl(hf::pool_blocks_kernel<D, true>, grid1, hf::kPoolThreads, 0, st,
+                 reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block,
+                 nQB, nKB, Qp, Kp, T, Kpart) != HF_OK)
+    return HF_ERR_CUDA;
+  if (launch_pdl(hf::pool_frames_kernel<D>, static_cast<long long>(BH) * W, D, 0, st, static_cast<const float*>(Kpart),
+                 Nk, block, T, nKB, W, Kf) != HF_OK)
+    return HF_ERR_CUDA;
   const size_t smem = static_cast<size_t>(hf::kSelQB) * (nKB + W) * (sizeof(float) + 1);
   if (cudaFuncSetAttribute(hf::score_select2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return HF_ERR_CUDA;
   const long long groups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
-  hf::score_select2_kernel<D><<<static_cast<unsigned>(static_cast<long long>(BH) * groups), hf::kSelectThreads, smem,
-                                st>>>(Qp, Kp, Kf, nQB, nKB, W, Nk, block, T, r, nf, idx, frames, scores);
-  return launch_status();
+  return launch_pdl(hf::score_select2_kernel<D>, static_cast<long long>(BH) * groups, hf::kSelectThreads, smem, st,
+                    static_cast<const float*>(Qp), static_cast<const float*>(Kp), static_cast<const float*>(Kf), nQB,
+                    nKB, W, Nk, block, T, r, nf, idx, frames, scores);
 }
 
 // ---------------------------------------------------------------- absorb
@@ -214,9 +239,13 @@ size_t absorb_ws_bytes(int B, int H, int n_tokens, int d) {
          align256(static_cast<size_t>(bh) * pl.nsplit * d * 4);
 }
 
+// wait_first: 1 when the absorbed tokens may come from the previous kernel of the stream;
+// 0 when the caller has ordered them before the previous kernel's start (the partial sums
+// may then run beside that kernel's last CTAs, and only the slice reduction, which writes
+// S and z, waits for it).
 template <int D>
 hf_status launch_absorb(hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, int n_tokens, void* ws,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, int wait_first) {
   using C = hf::AbsorbCfg<D>;
   const long long BH = static_cast<long long>(st->B) * st->H;
   const AbsorbPlan pl = absorb_plan(BH, n_tokens, kAbsorbTargetCtas);
@@ -230,17 +259,17 @@ hf_status launch_absorb(hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, 
   p.n_tokens = n_tokens;
   p.tiles_per_split = pl.tiles_per_split;
   p.nsplit = pl.nsplit;
+  p.wait_first = wait_first;
   take_injection(2, &p.inject, &p.timeout_ns);
   if (cudaFuncSetAttribute(hf::absorb_partial_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kDynSmem) != cudaSuccess)
     return HF_ERR_CUDA;
-  hf::absorb_partial_kernel<D>
-      <<<static_cast<unsigned>(BH * pl.nsplit), hf::kAbsThreads, C::kDynSmem, stream>>>(mk, mv, p);
-  if (launch_status() != HF_OK) return HF_ERR_CUDA;
+  if (launch_pdl(hf::absorb_partial_kernel<D>, BH * pl.nsplit, hf::kAbsThreads, C::kDynSmem, stream, mk, mv, p) !=
+      HF_OK)
+    return HF_ERR_CUDA;
   constexpr int kCtasPerHead = (D * D / 4 + 255) / 256;
-  hf::reduce_state_kernel<D><<<static_cast<unsigned>(BH * kCtasPerHead), 256, 0, stream>>>(st->S, st->z, p.part_S,
-                                                                                         p.part_z, pl.nsplit);
-  return launch_status();
+  return launch_pdl(hf::reduce_state_kernel<D>, BH * kCtasPerHead, 256, 0, stream, st->S, st->z,
+                    static_cast<const float*>(p.part_S), static_cast<const float*>(p.part_z), pl.nsplit);
 }
 
 // ---------------------------------------------------------------- attention
@@ -266,10 +295,8 @@ hf_status launch_attn(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int 
   if (cudaFuncSetAttribute(hf::hybrid_attn_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kDynSmem) != cudaSuccess)
     return HF_ERR_CUDA;
-  hf::hybrid_attn_kernel<D, BLK>
-      <<<static_cast<unsigned>(static_cast<long long>(BH) * nQB), hf::kAttnThreads, C::kDynSmem, stream>>>(
-          mq, mk, mv, mo, p);
-  return launch_status();
+  return launch_pdl(hf::hybrid_attn_kernel<D, BLK>, static_cast<long long>(BH) * nQB, hf::kAttnThreads, C::kDynSmem,
+                    stream, mq, mk, mv, mo, p);
 }
 
 __global__ void debug_exp2_kernel(const float* __restrict__ x, float* __restrict__ yp, float* __restrict__ ym,
@@ -341,6 +368,60 @@ hf_status select_scratch(void** out) {
 
 }  // namespace
 
+namespace {
+
+// Argument checks of hf_hybrid_attn_fwd (nothing is launched).
+hf_status check_attn_args(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H, int Nq, int Nk, int d,
+                          int block, int r, const int32_t* idx, const hf_state* st, float scale, const hf_bf16* O) {
+  if (B < 1 || H < 1 || Nq < 0 || Nk < 1 || !st) return HF_ERR_INVALID_ARG;
+  if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
+  const int nKB = ceil_div(Nk, block);
+  if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
+  if (st->B != B || st->H != H || st->d != d || !st->S || !st->z) return HF_ERR_INVALID_ARG;
+  if (!(scale == scale) || std::isinf(scale)) return HF_ERR_INVALID_ARG;
+  if (Nq == 0) return HF_OK;
+  if (!Q || !K || !V || !idx || !O) return HF_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx) || !aligned16(st->S) ||
+      !aligned16(st->z))
+    return HF_ERR_ALIGNMENT;
+  if (static_cast<long long>(B) * H * ceil_div(Nq, block) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  return HF_OK;
+}
+
+// Argument checks of hf_absorb_evicted for n_tokens >= 1 (nothing is launched).
+hf_status check_absorb_args(const hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, int n_tokens,
+                            const void* ws, size_t ws_bytes) {
+  if (!st || !st->S || !st->z || st->B < 1 || st->H < 1 || n_tokens < 0) return HF_ERR_INVALID_ARG;
+  if (!supported_d(st->d)) return HF_ERR_UNSUPPORTED;
+  if (n_tokens == 0) return HF_OK;
+  if (!K_ev || !V_ev) return HF_ERR_INVALID_ARG;
+  if (!aligned16(K_ev) || !aligned16(V_ev) || !aligned16(st->S) || !aligned16(st->z)) return HF_ERR_ALIGNMENT;
+  const size_t need = absorb_ws_bytes(st->B, st->H, n_tokens, st->d);
+  if (!ws || ws_bytes < need) return HF_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
+  return HF_OK;
+}
+
+// The attention launch for already-checked arguments with Nq >= 1.
+hf_status dispatch_attn(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H, int Nq, int Nk, int d,
+                        int block, int r, const int32_t* idx, const hf_state* st, float scale, hf_bf16* O,
+                        cudaStream_t s) {
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+  const int bh = B * H;
+#define HF_ATTN_CASE(DD, BB) \
+  if (d == DD && block == BB) return launch_attn<DD, BB>(Q, K, V, bh, Nq, Nk, r, idx, st, sc, O, s);
+  HF_ATTN_CASE(128, 128)
+  HF_ATTN_CASE(128, 64)
+  HF_ATTN_CASE(128, 32)
+  HF_ATTN_CASE(64, 128)
+  HF_ATTN_CASE(64, 64)
+  HF_ATTN_CASE(64, 32)
+#undef HF_ATTN_CASE
+  return HF_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+
 extern "C" {
 
 HF_API const char* hf_version(void) { return "hf-b200 0.1.0 (sm_100a)"; }
@@ -401,17 +482,11 @@ HF_API hf_status hf_state_init(hf_state* st, int B, int H, int d, float* S_dev, 
 
 HF_API hf_status hf_absorb_evicted(hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, int n_tokens, void* ws,
                                    size_t ws_bytes, void* stream) {
-  if (!st || !st->S || !st->z || st->B < 1 || st->H < 1 || n_tokens < 0) return HF_ERR_INVALID_ARG;
-  if (!supported_d(st->d)) return HF_ERR_UNSUPPORTED;
-  if (n_tokens == 0) return HF_OK;
-  if (!K_ev || !V_ev) return HF_ERR_INVALID_ARG;
-  if (!aligned16(K_ev) || !aligned16(V_ev) || !aligned16(st->S) || !aligned16(st->z)) return HF_ERR_ALIGNMENT;
-  const size_t need = absorb_ws_bytes(st->B, st->H, n_tokens, st->d);
-  if (!ws || ws_bytes < need) return HF_ERR_WORKSPACE;
-  if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
+  const hf_status chk = check_absorb_args(st, K_ev, V_ev, n_tokens, ws, ws_bytes);
+  if (chk != HF_OK || n_tokens == 0) return chk;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const hf_status rc = st->d == 128 ? launch_absorb<128>(st, K_ev, V_ev, n_tokens, ws, s)
-                                    : launch_absorb<64>(st, K_ev, V_ev, n_tokens, ws, s);
+  const hf_status rc = st->d == 128 ? launch_absorb<128>(st, K_ev, V_ev, n_tokens, ws, s, 1)
+                                    : launch_absorb<64>(st, K_ev, V_ev, n_tokens, ws, s, 1);
   if (rc == HF_OK) st->n_absorbed += n_tokens;
   return rc;
 }
@@ -474,13 +549,12 @@ HF_API hf_status hf_kpool_push(hf_kpool* kp, const hf_bf16* K_new, int n_tokens,
     const int base = (head + kept) % cap;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(K_new);
-    if (kp->d == 128)
-      hf::kpool_push_kernel<128><<<static_cast<unsigned>(BH * groups), hf::kPoolThreads, 0, s>>>(
-          K, n_tokens, G, n_new, base, cap, kp->sums);
-    else
-      hf::kpool_push_kernel<64><<<static_cast<unsigned>(BH * groups), hf::kPoolThreads, 0, s>>>(
-          K, n_tokens, G, n_new, base, cap, kp->sums);
-    if (launch_status() != HF_OK) return HF_ERR_CUDA;
+    const hf_status rc =
+        kp->d == 128 ? launch_pdl(hf::kpool_push_kernel<128>, BH * groups, hf::kPoolThreads, 0, s, K, n_tokens, G,
+                                  n_new, base, cap, kp->sums)
+                     : launch_pdl(hf::kpool_push_kernel<64>, BH * groups, hf::kPoolThreads, 0, s, K, n_tokens, G,
+                                  n_new, base, cap, kp->sums);
+    if (rc != HF_OK) return HF_ERR_CUDA;
   }
   kp->head = head;
   kp->n_gran = kept + n_new;
@@ -545,32 +619,31 @@ HF_API hf_status hf_hybrid_attn_fwd(const hf_bf16* Q, const hf_bf16* K, const hf
                                     float scale, hf_bf16* O, void* ws, size_t ws_bytes, void* stream) {
   (void)ws;
   (void)ws_bytes;
-  if (B < 1 || H < 1 || Nq < 0 || Nk < 1 || !st) return HF_ERR_INVALID_ARG;
-  if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
-  const int nKB = ceil_div(Nk, block);
-  if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
-  if (st->B != B || st->H != H || st->d != d || !st->S || !st->z) return HF_ERR_INVALID_ARG;
-  if (!(scale == scale) || std::isinf(scale)) return HF_ERR_INVALID_ARG;
-  if (Nq == 0) return HF_OK;
-  if (!Q || !K || !V || !idx || !O) return HF_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx) || !aligned16(st->S) ||
-      !aligned16(st->z))
-    return HF_ERR_ALIGNMENT;
-  const long long BH = static_cast<long long>(B) * H;
-  if (BH * ceil_div(Nq, block) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
-  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+  const hf_status rc = check_attn_args(Q, K, V, B, H, Nq, Nk, d, block, r, idx, st, scale, O);
+  if (rc != HF_OK || Nq == 0) return rc;
+  return dispatch_attn(Q, K, V, B, H, Nq, Nk, d, block, r, idx, st, scale, O, static_cast<cudaStream_t>(stream));
+}
+
+HF_API hf_status hf_hybrid_attn_fwd_absorb(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H,
+                                           int Nq, int Nk, int d, int block, int r, const int32_t* idx, hf_state* st,
+                                           float scale, hf_bf16* O, const hf_bf16* K_ev, const hf_bf16* V_ev,
+                                           int n_evicted, void* ws, size_t ws_bytes, void* stream) {
+  hf_status rc = check_attn_args(Q, K, V, B, H, Nq, Nk, d, block, r, idx, st, scale, O);
+  if (rc != HF_OK) return rc;
+  rc = check_absorb_args(st, K_ev, V_ev, n_evicted, ws, ws_bytes);
+  if (rc != HF_OK) return rc;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int bh = static_cast<int>(BH);
-#define HF_ATTN_CASE(DD, BB) \
-  if (d == DD && block == BB) return launch_attn<DD, BB>(Q, K, V, bh, Nq, Nk, r, idx, st, sc, O, s);
-  HF_ATTN_CASE(128, 128)
-  HF_ATTN_CASE(128, 64)
-  HF_ATTN_CASE(128, 32)
-  HF_ATTN_CASE(64, 128)
-  HF_ATTN_CASE(64, 64)
-  HF_ATTN_CASE(64, 32)
-#undef HF_ATTN_CASE
-  return HF_ERR_UNSUPPORTED;
+  int wait_first = 1;  // without an attention launch before it, the absorption waits as on its own
+  if (Nq > 0) {
+    rc = dispatch_attn(Q, K, V, B, H, Nq, Nk, d, block, r, idx, st, scale, O, s);
+    if (rc != HF_OK) return rc;
+    wait_first = 0;
+  }
+  if (n_evicted == 0) return HF_OK;
+  rc = d == 128 ? launch_absorb<128>(st, K_ev, V_ev, n_evicted, ws, s, wait_first)
+                : launch_absorb<64>(st, K_ev, V_ev, n_evicted, ws, s, wait_first);
+  if (rc == HF_OK) st->n_absorbed += n_evicted;
+  return rc;
 }
 
 HF_API hf_status hf_keep_schedule(int n_chunks, const int* nKB, double s_base, double s_target, int* r_out,

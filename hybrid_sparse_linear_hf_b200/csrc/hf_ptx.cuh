@@ -111,6 +111,23 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 }
 
 // ----------------------------------------------------------------------------
+// programmatic dependent launch (PDL)
+// ----------------------------------------------------------------------------
+// A kernel launched with programmatic stream serialisation may start before the
+// previous kernel of its stream has finished. griddep_wait() blocks the calling thread
+// until every prerequisite grid has completed and its memory is visible; every kernel of
+// this library calls it before it reads anything an earlier kernel may have written and
+// before it exits, so completion stays transitive along the stream. Without the launch
+// attribute both instructions do nothing.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next kernel of the stream be scheduled once every CTA of this grid has
+// executed this instruction or exited.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// ----------------------------------------------------------------------------
 // TMA (bulk tensor copies; never with cluster multicast)
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

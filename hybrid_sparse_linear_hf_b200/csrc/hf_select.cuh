@@ -25,6 +25,9 @@
 // score_select2_kernel keeps frames first, then blocks within them (see there).
 // Pooled-key cache: kpool_push_kernel sums each granule of G new keys into a ring, and
 // kpool_blocks_kernel forms the window's key block means from those sums (see there).
+// Every kernel is launched with programmatic stream serialisation: it waits for the
+// previous grid of its stream before its first read and then lets the next one be
+// scheduled (griddep_wait / griddep_launch_dependents in hf_ptx.cuh).
 #pragma once
 
 #include "hf_ptx.cuh"
@@ -72,6 +75,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bf
   constexpr int kUnroll = 8;                    // loads in flight per thread
   __shared__ float red[kRows * D];
   __shared__ float red1[kParts ? kRows * D : 1];
+  griddep_wait();
+  griddep_launch_dependents();
 
   const int per_bh = nQB + nKB;
   const int bh = blockIdx.x / per_bh;
@@ -148,6 +153,8 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bf
 template <int D>
 __global__ void __launch_bounds__(D) pool_frames_kernel(const float* __restrict__ Kpart, int Nk, int block, int T,
                                                         int nKB, int W, float* __restrict__ Kf) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int bh = blockIdx.x / W, w = blockIdx.x % W;
   const int f_lo = w * T, f_hi = min(f_lo + T, Nk);
   const int J_lo = f_lo / block, J_hi = (f_hi - 1) / block;
@@ -292,6 +299,8 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const floa
                                                                       float* __restrict__ scores_out) {
   extern __shared__ float s_sc[];  // [kSelQB][nKB] scores
   __shared__ __align__(16) float q_sh[kSelQB][D];
+  griddep_wait();
+  griddep_launch_dependents();
   const int groups = (nQB + kSelQB - 1) / kSelQB;
   const int bh = blockIdx.x / groups;
   const int I0 = (blockIdx.x % groups) * kSelQB;
@@ -333,6 +342,8 @@ __global__ void __launch_bounds__(kPoolThreads) kpool_push_kernel(const __nv_bfl
   constexpr int kTpr = D / kVec;                 // threads per granule
   constexpr int kGran = kPoolThreads / kTpr;     // granules per CTA
   constexpr int kUnroll = 8;
+  griddep_wait();
+  griddep_launch_dependents();
   const int groups = (n_new + kGran - 1) / kGran;
   const int bh = blockIdx.x / groups;
   const int g = (blockIdx.x % groups) * kGran + threadIdx.x / kTpr;
@@ -363,6 +374,8 @@ __global__ void __launch_bounds__(kPoolThreads) kpool_blocks_kernel(const float*
                                                                     int nKB, int BH, float* __restrict__ Kp) {
   constexpr int kC = D / 32;  // columns per lane: 4 or 2
   constexpr int kUnroll = 8;
+  griddep_wait();
+  griddep_launch_dependents();
   const long long wid = static_cast<long long>(blockIdx.x) * (kPoolThreads / 32) + threadIdx.x / 32;
   if (wid >= static_cast<long long>(BH) * nKB) return;
   const int lane = threadIdx.x % 32;
@@ -439,6 +452,8 @@ __global__ void __launch_bounds__(kSelectThreads) score_select2_kernel(
   uint8_t* kept = reinterpret_cast<uint8_t*>(f_sc + kSelQB * W);
   uint8_t* sel = kept + kSelQB * W;
   __shared__ __align__(16) float q_sh[kSelQB][D];
+  griddep_wait();
+  griddep_launch_dependents();
   const int groups = (nQB + kSelQB - 1) / kSelQB;
   const int bh = blockIdx.x / groups;
   const int I0 = (blockIdx.x % groups) * kSelQB;

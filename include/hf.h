@@ -42,7 +42,10 @@
  *     about one second) records HF_ERR_DEVICE_TIMEOUT in the device error word
  *     instead of hanging; hf_query_status reports it.
  *   - Calls on one stream are ordered; calls whose buffers overlap must not run
- *     concurrently on different streams.
+ *     concurrently on different streams. Kernels are launched with programmatic
+ *     stream serialisation: a kernel may be scheduled while the previous kernel of its
+ *     stream finishes its last CTAs, and waits for it on the device before reading
+ *     anything; stream order is kept for every caller-visible buffer.
  */
 #ifndef HF_H_
 #define HF_H_
@@ -258,6 +261,30 @@ HF_API hf_status hf_hybrid_attn_fwd(const hf_bf16* Q, const hf_bf16* K, const hf
                                     int Nq, int Nk, int d, int block, int r, const int32_t* idx,
                                     const hf_state* st, float scale, hf_bf16* O, void* ws, size_t ws_bytes,
                                     void* stream);
+
+/* One chunk step's attention and absorption in a single call:
+ *   O = hf_hybrid_attn_fwd(Q, K, V, idx, state as it stands), then
+ *   state += the n_evicted tokens (K_ev, V_ev: [B][H][n_evicted][d]) as hf_absorb_evicted.
+ * Source: Hybrid Forcing, German technical summary section 2 A (the output sums the
+ * sparse window term and the linear term of the compact state; frames leaving the window
+ * are aggregated into that state). The window of the next chunk no longer holds the
+ * evicted frames, so O reads the state before their absorption and the next call's O
+ * after it.
+ * The absorption's partial sums (which read only K_ev and V_ev) run on the SMs that the
+ * attention's last CTAs leave, while those CTAs finish; only the final slice reduction,
+ * which writes S and z, waits for the whole attention. Results are bit-identical to
+ * hf_hybrid_attn_fwd followed by hf_absorb_evicted on the same stream.
+ * K_ev, V_ev and ws must be complete when the call is issued (written by earlier work of
+ * `stream`) and must not overlap O. ws: HF_WS_ABSORB bytes for n_evicted tokens (NULL
+ * when n_evicted == 0). Nq == 0 runs the absorption alone; n_evicted == 0 the attention
+ * alone. st->n_absorbed += n_evicted on success.
+ * Errors: those of hf_hybrid_attn_fwd and hf_absorb_evicted, checked before anything is
+ * launched. */
+HF_API hf_status hf_hybrid_attn_fwd_absorb(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H,
+                                           int Nq, int Nk, int d, int block, int r, const int32_t* idx,
+                                           hf_state* st, float scale, hf_bf16* O, const hf_bf16* K_ev,
+                                           const hf_bf16* V_ev, int n_evicted, void* ws, size_t ws_bytes,
+                                           void* stream);
 
 /* Per-chunk keep schedule of chunk-aware growth (host only; no device work): the
  * sparsity ratio s[i] and the kept key blocks r[i] of every chunk i of a video, for

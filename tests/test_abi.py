@@ -283,3 +283,28 @@ def test_binding_checks_every_tensor_shape_before_any_call():
         hf.hf_select_blocks_cached(torch.empty(1, 2, 100, 128, dtype=bf), kp, 32, 2)
     with pytest.raises(ValueError, match="idx_out"):
         hf.hf_select_blocks_cached(Q, kp, 32, 2, idx_out=i32(1, 2, 4, 1))
+
+
+def test_fused_attention_absorb_validation():
+    """hf_hybrid_attn_fwd_absorb checks both halves' arguments before any launch."""
+    L = hf.lib()
+
+    def call(st=None, **kw):
+        a = dict(Q=A, K=A, V=A, B=1, H=1, Nq=64, Nk=256, d=64, block=32, r=2, idx=A, scale=0.0, O=A, Kev=A, Vev=A,
+                 n=100, ws=A, ws_bytes=1 << 30)
+        a.update(kw)
+        st = st or _state()
+        return L.hf_hybrid_attn_fwd_absorb(a["Q"], a["K"], a["V"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"],
+                                           a["block"], a["r"], a["idx"], ctypes.byref(st), a["scale"], a["O"],
+                                           a["Kev"], a["Vev"], a["n"], a["ws"], a["ws_bytes"], None)
+    assert call(r=9) == B.HF_ERR_INVALID_ARG            # attention argument
+    assert call(st=_state(H=2)) == B.HF_ERR_INVALID_ARG
+    assert call(O=A + 8) == B.HF_ERR_ALIGNMENT
+    assert call(Kev=None) == B.HF_ERR_INVALID_ARG       # absorption argument
+    assert call(Vev=A + 2) == B.HF_ERR_ALIGNMENT
+    assert call(n=-1) == B.HF_ERR_INVALID_ARG
+    assert call(ws=None) == B.HF_ERR_WORKSPACE
+    assert call(ws_bytes=16) == B.HF_ERR_WORKSPACE
+    st = _state()
+    assert call(st=st, Nq=0, n=0, Kev=None, Vev=None, ws=None) == B.HF_OK   # nothing to do
+    assert st.n_absorbed == 0

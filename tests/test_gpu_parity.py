@@ -466,3 +466,74 @@ def test_bench_step_sequence_on_device_drawn_inputs():
     Og = f64(O)
     n = _check_every_tile(Og, Q64, K64, V64, idx_h, f64(S_before), f64(z_before), wl.block, range(wl.H))
     assert n == wl.B * wl.H * wl.nQB
+
+
+# --------------------------------------------------------------------------- fused step
+@pytest.mark.parametrize("B,H,Nq,Nk,d,block,r,n_state,n_ev", [
+    (1, 1, 64, 256, 64, 32, 2, 192, 192),       # the tiny workload's shape
+    (1, 3, 300, 1000, 128, 128, 3, 500, 777),   # ragged tails, evicted tokens not a multiple of 64
+    (2, 2, 200, 700, 64, 64, 4, 64, 1),         # a single evicted token
+    (1, 12, 4680, 32760, 128, 128, 64, 1560, 4680),  # the 832x480 step
+])
+def test_fused_attention_absorb_equals_separate_calls(B, H, Nq, Nk, d, block, r, n_state, n_ev):
+    """hf_hybrid_attn_fwd_absorb gives bit-identically the O of hf_hybrid_attn_fwd (state
+    before the absorption) and the state of hf_absorb_evicted afterwards; both agree with
+    the oracle."""
+    g = torch.Generator().manual_seed(B * 1000 + Nq + n_ev)
+    Q, K, V, K0, V0, Ke, Ve = (frame_structured(g, B, H, n, d, 64, 0.5) for n in (Nq, Nk, Nk, n_state, n_state,
+                                                                                  n_ev, n_ev))
+    Qd, Kd, Vd, Ked, Ved = (t.to(DEV) for t in (Q, K, V, Ke, Ve))
+    st_a = _state_from(K0, V0, d)
+    st_b = _state_from(K0, V0, d)
+    S0, z0 = f64(st_a.S), f64(st_a.z)
+    idx = hf.hf_select_blocks(Qd, Kd, block, r)
+    O_a = hf.hf_hybrid_attn_fwd(Qd, Kd, Vd, block, r, idx, st_a)
+    hf.hf_absorb_evicted(st_a, Ked, Ved)
+    O_b = hf.hf_hybrid_attn_fwd_absorb(Qd, Kd, Vd, block, r, idx, st_b, Ked, Ved)
+    torch.cuda.synchronize()
+    _check_status()
+    assert torch.equal(O_a, O_b), "fused O differs from the separate attention call"
+    assert torch.equal(st_a.S, st_b.S) and torch.equal(st_a.z, st_b.z), "fused state differs"
+    assert st_b.n_absorbed == n_state + n_ev
+    S_o, z_o = oracle.absorb(S0, z0, f64(Ke), f64(Ve))
+    assert_state_close(f64(st_b.S), f64(st_b.z), S_o, z_o)
+    idx_h = idx.cpu().numpy()
+    heads = range(H) if H <= 3 else (0, H - 1)
+    _check_every_tile(f64(O_b), f64(Q), f64(K), f64(V), idx_h, S0, z0, block, heads, what="fused O")
+
+
+def test_streaming_832x480_fused_steps():
+    """20 chunk steps at the 832x480 shape through the fused call, back to back on one
+    stream (each step's absorption overlapping the attention's tail and the next step's
+    selection queued behind it): the final state against a float64 batch recompute on two
+    heads, and every query tile of the last step's output against the oracle run on the
+    state of the 19 steps before it."""
+    wl = WORKLOADS["832x480"]
+    d = wl.d
+    S = torch.empty(wl.B, wl.H, d, d, device=DEV)
+    z = torch.empty(wl.B, wl.H, d, device=DEV)
+    st = hf.hf_state_init(S, z)
+    heads = (0, wl.H - 1)
+    x = draw_step_inputs(wl, seed=20001, n_evicted=1)
+    Qd, Kd, Vd = x["Q"].to(DEV), x["K"].to(DEV), x["V"].to(DEV)
+    idx = hf.hf_select_blocks(Qd, Kd, wl.block, wl.r)
+    O = torch.empty_like(Qd)
+    ev_k, ev_v = [], []
+    snap = None
+    for t in range(1, 21):
+        g = torch.Generator().manual_seed(30000 + t)
+        K_ev = frame_structured(g, wl.B, wl.H, wl.Ne_step, d, wl.tokens_per_frame, wl.w)
+        V_ev = frame_structured(g, wl.B, wl.H, wl.Ne_step, d, wl.tokens_per_frame, wl.w)
+        if t == 20:
+            snap = (st.S.clone(), st.z.clone())
+        hf.hf_hybrid_attn_fwd_absorb(Qd, Kd, Vd, wl.block, wl.r, idx, st, K_ev.to(DEV), V_ev.to(DEV), O=O)
+        ev_k.append(K_ev[:, list(heads)])
+        ev_v.append(V_ev[:, list(heads)])
+    torch.cuda.synchronize()
+    _check_status()
+    assert st.n_absorbed == 20 * wl.Ne_step
+    S_o, z_o = oracle.absorb_batch(f64(torch.cat(ev_k, 2)), f64(torch.cat(ev_v, 2)))
+    assert_state_close(f64(st.S[:, list(heads)]), f64(st.z[:, list(heads)]), S_o, z_o)
+    n = _check_every_tile(f64(O), f64(x["Q"]), f64(x["K"]), f64(x["V"]), idx.cpu().numpy(), f64(snap[0]),
+                          f64(snap[1]), wl.block, range(wl.H), what="O at step 20")
+    assert n == wl.H * wl.nQB
