@@ -25,6 +25,9 @@ Sources (page title, then the section used):
            then blocks within the selected frames); §2.1 Chunk-bewusstes
            Wachstum (dense first chunk, sparsity s_i = s_base - alpha_i beta for
            the later chunks, beta set by a FLOP budget).
+  [HF-de] §2 C and [HF-pt] §2 B.2 (relative RoPE: the largest temporal RoPE
+           index is capped, in training and inference alike, and positions are
+           expressed as relative offsets).
 
 The pages give the structure (a compact KV state absorbing evicted tokens
 through a linear attention function; Top-K block-sparse attention inside the
@@ -58,7 +61,8 @@ __all__ = [
     "select_blocks", "frame_ranges", "pool_frames", "frame_scores", "candidate_blocks",
     "select_blocks_two_stage", "sparse_attention_tile", "sparse_attention", "linear_readout",
     "hybrid_attention", "hybrid_attention_tile", "absorb", "absorb_batch",
-    "dense_swa", "default_scale", "keep_schedule",
+    "dense_swa", "default_scale", "keep_schedule", "ROPE_BASE", "rope_positions", "rope_rotate", "rope_qk",
+    "select_blocks_rope", "hybrid_attention_rope", "hybrid_attention_rope_tile",
 ]
 
 
@@ -347,3 +351,86 @@ def keep_schedule(nKB, s_base: float, s_target: float):
             raise ValueError("a chunk's sparsity leaves [0, 1)")
     r = np.array([min(max(math.ceil((1.0 - s[i]) * nKB[i]), 1), nKB[i]) for i in range(n)], dtype=np.int64)
     return r, s, beta
+
+
+# ---------------------------------------------------------------------------
+# capped relative temporal RoPE ([HF-de] §2 C; [HF-pt] §2 B.2)
+# ---------------------------------------------------------------------------
+# Readings (the pages name the technique and nothing else): the temporal part of a
+# rotary embedding acts on the first d_t dimensions of a head, as consecutive pairs
+# (2i, 2i+1) turned by the angle p * base**(-2i/d_t) (the textbook RoPE frequencies,
+# base 10000); the spatial parts of a video RoPE do not depend on time and are left to
+# the model. A token's temporal index p counts from its frame's offset to the newest
+# frame of the window, delta, capped at P: p = P - min(delta, P), so the newest frame
+# sits at P and every frame P or more frames old at 0 (the index never exceeds P
+# however long the video). The rotation applies to q and k of the softmax branch, and
+# so to the tokens the block selection pools; the linear branch reads the raw q and k
+# (evicted frames are older than the window, i.e. at index 0 where the rotation is the
+# identity once P does not exceed the window).
+ROPE_BASE = 10000.0
+
+
+def rope_positions(n_tokens: int, tokens_per_frame: int, frame0: int, n_frames: int, cap: int) -> np.ndarray:
+    """Temporal index of each of n_tokens consecutive tokens whose first token lies in
+    window frame frame0 (frames of tokens_per_frame tokens; the window holds n_frames
+    frames, the newest being n_frames - 1): p = cap - min(delta, cap) with
+    delta = (n_frames - 1) - frame. int64 [n_tokens]."""
+    p = np.empty(n_tokens, dtype=np.int64)
+    for t in range(n_tokens):
+        frame = frame0 + t // tokens_per_frame
+        delta = (n_frames - 1) - frame
+        p[t] = cap - min(delta, cap)
+    return p
+
+
+def rope_rotate(X, positions, d_t: int, base: float = ROPE_BASE) -> np.ndarray:
+    """X [..., N, d] with the pairs (2i, 2i+1), i < d_t/2, of token n turned by the angle
+    positions[n] * base**(-2i/d_t); the other dimensions unchanged."""
+    X = _f64(X).copy()
+    pos = np.asarray(positions, dtype=np.float64)
+    for i in range(d_t // 2):
+        ang = pos * base ** (-2.0 * i / d_t)
+        c, s = np.cos(ang), np.sin(ang)
+        a = X[..., 2 * i].copy()
+        b = X[..., 2 * i + 1].copy()
+        X[..., 2 * i] = a * c - b * s
+        X[..., 2 * i + 1] = a * s + b * c
+    return X
+
+
+def rope_qk(Q, K, rope: dict):
+    """Q and K of a chunk step turned by their temporal indices. rope: d_t,
+    tokens_per_frame, cap, q_frame0 (window frame of Q's first token), base. K is the
+    window (its first token starts frame 0); the window holds ceil(Nk / tokens_per_frame)
+    frames."""
+    T = int(rope["tokens_per_frame"])
+    Nq, Nk = np.shape(Q)[2], np.shape(K)[2]
+    W = -(-Nk // T)
+    base = float(rope.get("base", ROPE_BASE))
+    pq = rope_positions(Nq, T, int(rope["q_frame0"]), W, int(rope["cap"]))
+    pk = rope_positions(Nk, T, 0, W, int(rope["cap"]))
+    return rope_rotate(Q, pq, int(rope["d_t"]), base), rope_rotate(K, pk, int(rope["d_t"]), base)
+
+
+def select_blocks_rope(Q, K, block: int, r: int, rope: dict):
+    """select_blocks on the turned Q and K (the selection pools the tokens the softmax
+    branch attends with)."""
+    Qr, Kr = rope_qk(Q, K, rope)
+    return select_blocks(Qr, Kr, block, r)
+
+
+def hybrid_attention_rope(Q, K, V, idx, S, z, block: int, rope: dict, scale: float | None = None) -> np.ndarray:
+    """Sparse term on the turned Q and K plus the linear term on the raw Q."""
+    Qr, Kr = rope_qk(Q, K, rope)
+    return sparse_attention(Qr, Kr, V, idx, block, scale) + linear_readout(Q, S, z)
+
+
+def hybrid_attention_rope_tile(Q, K, V, idx, S, z, block: int, rope: dict, b: int, h: int, I: int,
+                               scale: float | None = None) -> np.ndarray:
+    """Output rows of query block I of hybrid_attention_rope."""
+    Qr, Kr = rope_qk(np.asarray(Q)[b:b + 1, h:h + 1], np.asarray(K)[b:b + 1, h:h + 1], rope)
+    lo, hi = block_ranges(np.shape(Q)[2], block)[I]
+    o_s = sparse_attention_tile(Qr, Kr, np.asarray(V)[b:b + 1, h:h + 1], np.asarray(idx)[b:b + 1, h:h + 1],
+                                block, 0, 0, I, scale)
+    o_l = linear_readout(np.asarray(Q)[b, h, lo:hi], np.asarray(S)[b, h], np.asarray(z)[b, h])
+    return o_s + o_l

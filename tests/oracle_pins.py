@@ -436,6 +436,102 @@ def check_schedule_rejects(o):
     assert r.tolist() == [7] and s.tolist() == [0.0], "a single chunk is dense"
 
 
+# ---------------------------------------------------------------------------
+# capped relative temporal RoPE
+# ---------------------------------------------------------------------------
+def check_rope_positions_golden(o):
+    """Temporal indices of hand-worked cases (frames, offsets from the newest frame, cap)."""
+    for c in _golden()["rope"]["positions"]:
+        got = o.rope_positions(c["n_tokens"], c["tokens_per_frame"], c["frame0"], c["n_frames"], c["cap"])
+        assert got.tolist() == c["p"], (c, got.tolist())
+
+
+def check_rope_rotation_closed_form(o):
+    """One token, d = 6, d_t = 4, base 100, index 3: pair 0 turns by 3 rad, pair 1 by
+    3 * 100**(-1/2) = 0.3 rad (cos/sin from math), dims 4, 5 untouched."""
+    x = [1.0, 2.0, 3.0, 4.0, 5.0, 6.0]
+    got = o.rope_rotate(_as4([x]), [3], 4, base=100.0)[0, 0, 0]
+    c0, s0, c1, s1 = math.cos(3.0), math.sin(3.0), math.cos(0.3), math.sin(0.3)
+    want = [1 * c0 - 2 * s0, 1 * s0 + 2 * c0, 3 * c1 - 4 * s1, 3 * s1 + 4 * c1, 5.0, 6.0]
+    assert np.allclose(got, want, rtol=0, atol=1e-14), (got, want)
+
+
+def check_rope_complex_form(o):
+    """The same rotation written with complex numbers: pair (x[2i], x[2i+1]) is
+    x[2i] + 1j x[2i+1], multiplied by exp(1j p theta_i), theta_i = base**(-2i/d_t)."""
+    rng = np.random.default_rng(11)
+    X = rng.standard_normal((1, 2, 9, 12))
+    pos = rng.integers(0, 40, size=9)
+    d_t = 8
+    got = o.rope_rotate(X, pos, d_t)
+    zc = X[..., 0:d_t:2] + 1j * X[..., 1:d_t:2]
+    theta = 10000.0 ** (-np.arange(d_t // 2) * 2.0 / d_t)
+    zc = zc * np.exp(1j * pos[:, None] * theta[None, :])
+    want = X.copy()
+    want[..., 0:d_t:2] = zc.real
+    want[..., 1:d_t:2] = zc.imag
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
+def check_rope_norm_inverse_relative(o):
+    """A rotation keeps every token's norm, the index -p undoes the index p, and the
+    product of two turned vectors depends only on the difference of their indices."""
+    rng = np.random.default_rng(12)
+    X = rng.standard_normal((1, 1, 7, 16))
+    pos = rng.integers(0, 30, size=7)
+    Y = o.rope_rotate(X, pos, 10)
+    assert np.allclose(np.linalg.norm(Y, axis=-1), np.linalg.norm(X, axis=-1), rtol=1e-13)
+    assert np.allclose(o.rope_rotate(Y, -pos, 10), X, atol=1e-12)
+    q, k = X[0, 0, 0], X[0, 0, 1]
+    for pq, pk, sh in [(5, 2, 7), (0, 9, 3), (4, 4, 11)]:
+        a = o.rope_rotate(_as4([q]), [pq], 10)[0, 0, 0] @ o.rope_rotate(_as4([k]), [pk], 10)[0, 0, 0]
+        b = o.rope_rotate(_as4([q]), [pq + sh], 10)[0, 0, 0] @ o.rope_rotate(_as4([k]), [pk + sh], 10)[0, 0, 0]
+        assert abs(a - b) < 1e-12, (pq, pk, sh, a, b)
+
+
+def check_rope_cap_and_identity(o):
+    """Frames at least `cap` frames old sit at index 0 (unturned); with cap 0 or d_t 0
+    the turned step equals the plain one; the selection ranks blocks by the means of the
+    turned tokens."""
+    rng = np.random.default_rng(13)
+    T, W, C, d, block = 8, 5, 2, 8, 8
+    Q = rng.standard_normal((1, 1, C * T, d))
+    K = rng.standard_normal((1, 1, W * T, d))
+    V = rng.standard_normal((1, 1, W * T, d))
+    S = np.abs(rng.standard_normal((1, 1, d, d)))
+    z = np.abs(rng.standard_normal((1, 1, d)))
+    rope = {"d_t": 4, "tokens_per_frame": T, "cap": 2, "q_frame0": W - C}
+    Qr, Kr = o.rope_qk(Q, K, rope)
+    # by hand: the chunk's frames are window frames 3, 4 (offsets 1, 0: indices 1, 2); the
+    # window's frames 0..4 have offsets 4..0, indices 0, 0, 0, 1, 2
+    assert np.allclose(Qr, o.rope_rotate(Q, [1] * T + [2] * T, 4), atol=1e-14)
+    assert np.allclose(Kr, o.rope_rotate(K, [0] * (3 * T) + [1] * T + [2] * T, 4), atol=1e-14)
+    old = slice(0, (W - 2) * T)  # frames 0..2 are >= 2 frames older than the newest
+    assert np.array_equal(Kr[:, :, old], K[:, :, old])
+    assert not np.allclose(Kr[:, :, (W - 1) * T:], K[:, :, (W - 1) * T:])
+    idx = np.tile(np.arange(3, dtype=np.int32), (1, 1, 2, 1))
+    for ident in ({"d_t": 0}, {"cap": 0}):
+        r2 = dict(rope, **ident)
+        assert np.allclose(o.hybrid_attention_rope(Q, K, V, idx, S, z, block, r2),
+                           o.hybrid_attention(Q, K, V, idx, S, z, block), atol=1e-13)
+    # the sparse branch alone sees the turn; the linear branch reads the raw q
+    Qr, Kr = o.rope_qk(Q, K, rope)
+    got = o.hybrid_attention_rope(Q, K, V, idx, S, z, block, rope)
+    assert np.allclose(got - o.linear_readout(Q, S, z), o.sparse_attention(Qr, Kr, V, idx, block), atol=1e-13)
+    # turned keys of the first frame (index 0) and raw ones give the same readout of a
+    # state built from them (the linear branch of evicted frames)
+    S1, z1 = o.absorb_batch(K[:, :, :T], V[:, :, :T])
+    S2, z2 = o.absorb_batch(Kr[:, :, :T], V[:, :, :T])
+    assert np.array_equal(S1, S2) and np.array_equal(z1, z2)
+    # selection by brute force over the means of the turned tokens
+    s = Qr.reshape(1, 1, C * T // block, block, d).mean(3) @ np.swapaxes(
+        Kr.reshape(1, 1, W * T // block, block, d).mean(3), -1, -2)
+    idx_o, s_o = o.select_blocks_rope(Q, K, block, 2, rope)
+    assert np.allclose(s_o, s, atol=1e-12)
+    for I in range(2):
+        assert idx_o[0, 0, I].tolist() == sorted(_brute_force_topr(s[0, 0, I], 2))
+
+
 ALL_CHECKS = [
     check_phi_library, check_pool_by_hand, check_selection_golden, check_selection_bruteforce,
     check_selection_ties_constructed, check_selection_output_form, check_attention_golden,
@@ -446,4 +542,6 @@ ALL_CHECKS = [
     check_two_stage_all_frames_is_one_stage, check_two_stage_frames_are_blocks,
     check_two_stage_bruteforce, check_schedule_golden, check_schedule_budget_and_rounding,
     check_schedule_two_chunks, check_schedule_noise_scale, check_schedule_rejects,
+    check_rope_positions_golden, check_rope_rotation_closed_form, check_rope_complex_form,
+    check_rope_norm_inverse_relative, check_rope_cap_and_identity,
 ]

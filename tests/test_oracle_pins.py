@@ -226,6 +226,51 @@ def _mut_schedule_budget_on_chunks(m):
     m.keep_schedule = f
 
 
+def _mut_rope_sign(m):
+    orig = m.rope_rotate
+    m.rope_rotate = lambda X, positions, d_t, base=m.ROPE_BASE: orig(X, -np.asarray(positions), d_t, base)
+
+
+def _mut_rope_half_pairs(m):
+    def f(X, positions, d_t, base=m.ROPE_BASE):
+        X = np.asarray(X, dtype=np.float64).copy()
+        pos = np.asarray(positions, dtype=np.float64)
+        h = d_t // 2
+        for i in range(h):
+            ang = pos * base ** (-2.0 * i / d_t)
+            a, b = X[..., i].copy(), X[..., i + h].copy()
+            X[..., i] = a * np.cos(ang) - b * np.sin(ang)
+            X[..., i + h] = a * np.sin(ang) + b * np.cos(ang)
+        return X
+    m.rope_rotate = f
+
+
+def _mut_rope_uncapped(m):
+    def f(n_tokens, tokens_per_frame, frame0, n_frames, cap):
+        return np.array([frame0 + t // tokens_per_frame for t in range(n_tokens)], dtype=np.int64)
+    m.rope_positions = f
+
+
+def _mut_rope_frequency(m):
+    orig = m.rope_rotate
+
+    def f(X, positions, d_t, base=m.ROPE_BASE):
+        return orig(X, positions, 2 * d_t, base) if d_t else orig(X, positions, d_t, base)
+    m.rope_rotate = f
+
+
+def _mut_rope_turned_readout(m):
+    def f(Q, K, V, idx, S, z, block, rope, scale=None):
+        Qr, Kr = m.rope_qk(Q, K, rope)
+        return m.sparse_attention(Qr, Kr, V, idx, block, scale) + m.linear_readout(Qr, S, z)
+    m.hybrid_attention_rope = f
+
+
+def _mut_rope_query_frames(m):
+    orig = m.rope_qk
+    m.rope_qk = lambda Q, K, rope: orig(Q, K, dict(rope, q_frame0=0))
+
+
 MUTANTS = [
     _mut_phi_no_plus_one, _mut_phi_exp, _mut_readout_no_eps, _mut_readout_transposed,
     _mut_readout_no_phi_q, _mut_select_ties_high, _mut_select_bottom, _mut_pool_sum,
@@ -233,7 +278,8 @@ MUTANTS = [
     _mut_absorb_transposed, _mut_absorb_z_raw, _mut_hybrid_difference, _mut_two_stage_inside_only,
     _mut_two_stage_ignore_frames, _mut_pool_frames_sum, _mut_two_stage_frame_ties_high, _mut_two_stage_no_fill,
     _mut_schedule_alpha_linear, _mut_schedule_first_chunk_sparse, _mut_schedule_floor,
-    _mut_schedule_budget_on_chunks,
+    _mut_schedule_budget_on_chunks, _mut_rope_sign, _mut_rope_half_pairs, _mut_rope_uncapped,
+    _mut_rope_frequency, _mut_rope_turned_readout, _mut_rope_query_frames,
 ]
 
 
