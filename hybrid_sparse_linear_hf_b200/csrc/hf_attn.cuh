@@ -25,7 +25,8 @@
 //   warp 3      ring bookkeeping, off the softmax threads' path: in kept-block order it
 //               waits for S of block v (so QK(v), and PV(v-2) before it, are done), frees
 //               their K and V slots, waits for V(v) and K(v+2) to land, and adds its arrival
-//               to pipeline v%2's P-ready barrier (which also counts the 128 softmax threads).
+//               to pipeline v%2's P-ready barrier (which also counts one arrival per softmax
+//               warp of that pipeline).
 //   warps 4..7  pipeline A, warps 8..11 pipeline B: one thread per query row (TMEM lane
 //               quarter = warp % 4), the whole row of S per thread.
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+d), O_B [384,384+d). P (bf16
@@ -129,10 +130,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sfull_bar[b], 1);
-      mbar_init(&pfull_bar[b], 129);
+      mbar_init(&pfull_bar[b], 5);  // the pipeline's 4 warps + warp 3
     }
     mbar_init(&final_bar, 1);
-    mbar_init(&pro_bar, 256);
+    mbar_init(&pro_bar, 8);  // the 8 softmax warps
     mbar_init(&lin_bar, 1);
     mbar_init(&drain_bar, 1);
     abort_sh = 0;
@@ -415,9 +416,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st32(lane_addr + col_o + c, o);
         }
       }
+      // one arrival per warp, once every lane's P (and O rescale) stores are complete
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&pfull_bar[pipe]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pfull_bar[pipe]);
       ++i;
     }
 
@@ -483,7 +486,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       fence_proxy_async_smem();
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&pro_bar);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pro_bar);
     }
     // ---- merge of the two pipelines' softmax states and denominators (every row thread
     // reaches both named barriers, whatever happened before)

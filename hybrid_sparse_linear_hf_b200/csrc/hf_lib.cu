@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -122,6 +123,75 @@ hf_status launch_pdl(void (*kernel)(KArgs...), long long grid, int block, size_t
   return launch_status();
 }
 
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+// Checks of an hf_rope for a step with window Nk and blocks of `block` tokens.
+bool rope_ok(const hf_rope* rope, int d, int Nk, int block) {
+  if (!rope) return false;
+  if (rope->d_t < 0 || (rope->d_t & 1) || rope->d_t > d || rope->d_t > 64) return false;
+  if (rope->tokens_per_frame < block || rope->cap < 0 || rope->cap > 63) return false;
+  if (!(rope->base > 1.0f) || std::isinf(rope->base)) return false;
+  const int W = ceil_div(Nk, rope->tokens_per_frame);
+  return rope->q_frame0 >= 0 && rope->q_frame0 < W;
+}
+
+// Block pooling of Q (and K unless nKB == 0) by the persistent bulk-copy kernel; with a
+// rope (kRope), the means of the turned tokens.
+template <int D, bool kParts, bool kRope = false>
+hf_status launch_pool(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk, int block, int nQB, int nKB,
+                      float* Qp, float* Kp, int T, float* Kpart, cudaStream_t st, const hf_rope* rope = nullptr) {
+  hf::PoolArgs a;
+  if (kRope) {
+    T = rope->tokens_per_frame;
+    a.q_frame0 = rope->q_frame0;
+    a.n_frames = ceil_div(Nk, T);
+    a.rope_cap = rope->cap;
+    a.rope_dt = rope->d_t;
+    a.rope_log2base = std::log2(rope->base);
+  } else {
+    a.q_frame0 = a.n_frames = a.rope_cap = a.rope_dt = 0;
+    a.rope_log2base = 0.f;
+  }
+  a.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
+  a.K = reinterpret_cast<const __nv_bfloat16*>(K);
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.block = block;
+  a.nQB = nQB;
+  a.nKB = nKB;
+  a.BH = BH;
+  a.Qp = Qp;
+  a.Kp = Kp;
+  a.T = T;
+  a.Kpart = Kpart;
+  a.stage_bytes = block * D * 2;
+  // up to 192 KB of stages (six 32 KB stages at d = block = 128), at least two
+  constexpr int kStageBudget = 192 * 1024;
+  a.stages = std::min(hf::kPoolMaxStages, std::max(2, kStageBudget / a.stage_bytes));
+  take_injection(1, &a.inject, &a.timeout_ns);
+  const size_t smem = static_cast<size_t>(a.stages) * a.stage_bytes;
+  if (cudaFuncSetAttribute(hf::pool_bulk_kernel<D, kParts, kRope>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return HF_ERR_CUDA;
+  // CTAs per SM that fit beside one another (shared memory, threads), times the SMs
+  const size_t static_smem = 2 * sizeof(float) * hf::kPoolConsumers * 8 + 2 * 1024;
+  const long long per_sm = std::max<long long>(
+      1, std::min<long long>(2048 / hf::kPoolBulkThreads, (227 * 1024) / (smem + static_smem)));
+  const long long items = static_cast<long long>(BH) * (nQB + nKB);
+  const long long grid = std::min(items, per_sm * sm_count());
+  return launch_pdl(hf::pool_bulk_kernel<D, kParts, kRope>, grid, hf::kPoolBulkThreads, smem, st, a);
+}
+
 // ---------------------------------------------------------------- select
 size_t select_ws_bytes(int B, int H, int Nq, int Nk, int d, int block) {
   const long long bh = static_cast<long long>(B) * H;
@@ -146,15 +216,14 @@ hf_status launch_score(const float* Qp, const float* Kp, int BH, int nQB, int nK
 
 template <int D>
 hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk, int block, int r,
-                        int32_t* idx, float* scores, void* ws, cudaStream_t st) {
+                        int32_t* idx, float* scores, void* ws, cudaStream_t st, const hf_rope* rope = nullptr) {
   const int nQB = ceil_div(Nq, block), nKB = ceil_div(Nk, block);
   float* Qp = static_cast<float*>(ws);
   float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(BH) * nQB * D * 4));
-  const long long grid1 = static_cast<long long>(BH) * (nQB + nKB);
-  if (launch_pdl(hf::pool_blocks_kernel<D>, grid1, hf::kPoolThreads, 0, st, reinterpret_cast<const __nv_bfloat16*>(Q),
-                 reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block, nQB, nKB, Qp, Kp, 0,
-                 static_cast<float*>(nullptr)) != HF_OK)
-    return HF_ERR_CUDA;
+  const hf_status rc = rope ? launch_pool<D, false, true>(Q, K, BH, Nq, Nk, block, nQB, nKB, Qp, Kp, 0, nullptr, st,
+                                                            rope)
+                            : launch_pool<D, false>(Q, K, BH, Nq, Nk, block, nQB, nKB, Qp, Kp, 0, nullptr, st);
+  if (rc != HF_OK) return HF_ERR_CUDA;
   return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st);
 }
 
@@ -166,9 +235,7 @@ hf_status launch_select_cached(const hf_bf16* Q, const hf_kpool* kp, int BH, int
   const int nQB = ceil_div(Nq, block), nKB = ceil_div(Nk, block);
   float* Qp = static_cast<float*>(ws);
   float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(BH) * nQB * D * 4));
-  if (launch_pdl(hf::pool_blocks_kernel<D>, static_cast<long long>(BH) * nQB, hf::kPoolThreads, 0, st,
-                 reinterpret_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(nullptr), Nq, 0, block,
-                 nQB, 0, Qp, Kp, 0, static_cast<float*>(nullptr)) != HF_OK)
+  if (launch_pool<D, false>(Q, nullptr, BH, Nq, 0, block, nQB, 0, Qp, Kp, 0, nullptr, st) != HF_OK)
     return HF_ERR_CUDA;
   constexpr int kWarpsPerCta = hf::kPoolThreads / 32;
   const long long ctas = (static_cast<long long>(BH) * nKB + kWarpsPerCta - 1) / kWarpsPerCta;
@@ -200,11 +267,7 @@ hf_status launch_select2(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int
   float* Kpart = reinterpret_cast<float*>(base);
   base += align256(static_cast<size_t>(BH) * nKB * 2 * D * 4);
   float* Kf = reinterpret_cast<float*>(base);
-  const long long grid1 = static_cast<long long>(BH) * (nQB + nKB);
-  if (launch_pdl(hf::pool_blocks_kernel<D, true>, grid1, hf::kPoolThreads, 0, st,
-                 reinterpret_cast<const __nv_bfloat16*>(Q), reinterpret_cast<const __nv_bfloat16*>(K), Nq, Nk, block,
-                 nQB, nKB, Qp, Kp, T, Kpart) != HF_OK)
-    return HF_ERR_CUDA;
+  if (launch_pool<D, true>(Q, K, BH, Nq, Nk, block, nQB, nKB, Qp, Kp, T, Kpart, st) != HF_OK) return HF_ERR_CUDA;
   if (launch_pdl(hf::pool_frames_kernel<D>, static_cast<long long>(BH) * W, D, 0, st, static_cast<const float*>(Kpart),
                  Nk, block, T, nKB, W, Kf) != HF_OK)
     return HF_ERR_CUDA;
@@ -510,6 +573,29 @@ HF_API hf_status hf_select_blocks(const hf_bf16* Q, const hf_bf16* K, int B, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_select<128>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s)
                   : launch_select<64>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s);
+}
+
+HF_API hf_status hf_select_blocks_rope(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk, int d,
+                                       int block, int r, const hf_rope* rope, int32_t* idx_out, float* scores_out,
+                                       void* ws, size_t ws_bytes, void* stream) {
+  if (B < 1 || H < 1 || Nq < 0 || Nk < 1) return HF_ERR_INVALID_ARG;
+  if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
+  const int nKB = ceil_div(Nk, block);
+  if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
+  if (nKB > hf::kMaxKeyBlocks) return HF_ERR_UNSUPPORTED;
+  if (!rope_ok(rope, d, Nk, block)) return HF_ERR_INVALID_ARG;
+  if (Nq == 0) return HF_OK;
+  if (!Q || !K || !idx_out) return HF_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(idx_out) || (scores_out && !aligned16(scores_out)))
+    return HF_ERR_ALIGNMENT;
+  if (!ws || ws_bytes < select_ws_bytes(B, H, Nq, Nk, d, block)) return HF_ERR_WORKSPACE;
+  if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
+  const long long BH = static_cast<long long>(B) * H;
+  if (BH * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128
+             ? launch_select<128>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s, rope)
+             : launch_select<64>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s, rope);
 }
 
 // ---------------------------------------------------------------- pooled-key cache

@@ -11,16 +11,16 @@
 //
 // All on CUDA cores (the work is a streaming read of Q and K plus a tiny score matrix,
 // so tensor cores would not help):
-//   pool_blocks_kernel   one CTA per (b,h,block) of Q or K: fp32 mean of the valid rows.
-//                        HBM-bound: reads Q and K once with 16-byte loads, 8 in flight
-//                        per thread.
+//   pool_bulk_kernel     persistent, one CTA per SM: fp32 mean of the valid rows of every
+//                        block of Q and K. HBM-bound: each block's rows (contiguous) come
+//                        in by one bulk copy into a ring of up to 8 stages, 6 in flight.
 //   score_select_kernel  one CTA per (b,h, 4 query blocks): s_IJ = Qbar_I . Kbar_J, a
 //                        thread per key block; then one warp per query block finds the
 //                        r-th largest score by a bitwise search (per-lane counts, one warp
 //                        reduction per bit), takes every block above it and the lowest-J
 //                        blocks equal to it, and writes the r blocks in ascending J.
 //                        NaN scores are ranked as -inf, so exactly r blocks are written.
-// Two-stage selection: pool_blocks_kernel<d, true> also writes each key block's sums in
+// Two-stage selection: pool_bulk_kernel<d, true> also writes each key block's sums in
 // its first and next frame, pool_frames_kernel adds them into frame means, and
 // score_select2_kernel keeps frames first, then blocks within them (see there).
 // Pooled-key cache: kpool_push_kernel sums each granule of G new keys into a ring, and
@@ -57,92 +57,208 @@ __device__ __forceinline__ uint4 ld_stream_16(const void* p) {
   return v;
 }
 
-// Qp[bh][I][:] = mean of Q rows of block I; Kp[bh][J][:] likewise.
+constexpr uint32_t kKernSelect = 1;
+constexpr int kPoolConsumers = 256;                   // 8 consumer warps
+constexpr int kPoolBulkThreads = kPoolConsumers + 32;  // + the bulk-copy producer warp
+constexpr int kPoolMaxStages = 8;
+
+struct PoolArgs {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  int Nq, Nk, block, nQB, nKB, BH;
+  float* Qp;     // [BH][nQB][D]
+  float* Kp;     // [BH][nKB][D]
+  int T;         // frame length in tokens (kParts)
+  float* Kpart;  // [BH][nKB][2][D] (kParts)
+  int stages, stage_bytes;
+  unsigned long long timeout_ns;
+  int inject;    // test only: the first copy is never issued, so a wait runs out
+  // temporal RoPE (kRope): frames of T tokens; Q's first token lies in window frame
+  // q_frame0, K's in frame 0; the window holds n_frames frames; index cap, rotated
+  // dimensions [0, rope_dt), log2 of the frequency base
+  int q_frame0, n_frames, rope_cap, rope_dt;
+  float rope_log2base;
+};
+
+// Temporal RoPE index of window frame w: the newest frame (n_frames - 1) at cap, every
+// frame at least cap frames older at 0.
+__device__ __forceinline__ int rope_index(int w, int n_frames, int cap) {
+  return cap - min((n_frames - 1) - w, cap);
+}
+
+// (cos, sin) of the angle p * base^(-2i/d_t) of pair i (full-precision sincos).
+__device__ __forceinline__ void rope_cs(int p, int i, int d_t, float log2base, float& c, float& s) {
+  const float theta = exp2f(-static_cast<float>(2 * i) / static_cast<float>(d_t) * log2base);
+  sincosf(static_cast<float>(p) * theta, &s, &c);
+}
+
+// Qp[bh][I][:] = mean of the Q rows of block I; Kp[bh][J][:] likewise for K.
 // kParts (two-stage selection): also Kpart[bh][J][0|1][:] = the sums of the rows of key
 // block J that lie in its first frame (J*block / T) and in the next frame (zero when the
 // block does not reach it); frames are runs of T >= block tokens, so a block touches at
-// most two. The block means are computed exactly as without kParts.
-template <int D, bool kParts = false>
-__global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(const __nv_bfloat16* __restrict__ Q,
-                                                                   const __nv_bfloat16* __restrict__ K,
-                                                                   int Nq, int Nk, int block, int nQB, int nKB,
-                                                                   float* __restrict__ Qp,
-                                                                   float* __restrict__ Kp,
-                                                                   int T = 0, float* __restrict__ Kpart = nullptr) {
-  constexpr int kVec = 8;                       // bf16 per 16-byte load
-  constexpr int kTpr = D / kVec;                // threads per row
-  constexpr int kRows = kPoolThreads / kTpr;    // rows per pass
-  constexpr int kUnroll = 8;                    // loads in flight per thread
-  __shared__ float red[kRows * D];
-  __shared__ float red1[kParts ? kRows * D : 1];
+// most two.
+// kRope: the rows are summed per frame (a block spans at most two, T >= block), each
+// frame's sum is turned by that frame's temporal RoPE index (pairs (2i, 2i+1) of the
+// dimensions below d_t), and the mean is taken of the turned sums: the mean of the
+// turned tokens, as the rotation is linear and one per frame.
+// Persistent: CTA c takes the blocks c, c + gridDim.x, ... of the list [b,h][Q blocks | K
+// blocks]. A block's rows are contiguous in memory, so one bulk copy (up to block x d x 2
+// bytes) brings it into a ring stage; the producer warp keeps up to `stages` copies in
+// flight while the 8 consumer warps sum the stage they hold: thread (row phase rp, unit c)
+// adds 8 columns of the rows rp, rp + kPhases, ... in fp32, and the kPhases partial sums
+// of a column are added in row-phase order through shared memory (deterministic).
+template <int D, bool kParts = false, bool kRope = false>
+__global__ void __launch_bounds__(kPoolBulkThreads, 1) pool_bulk_kernel(PoolArgs a) {
+  constexpr int kUnits = D / 8;                   // 16-byte units per row
+  constexpr int kPhases = kPoolConsumers / kUnits;  // row phases
+  constexpr bool kSplit = kParts || kRope;        // per-frame sums
+  extern __shared__ __align__(128) uint8_t pool_smem[];
+  __shared__ uint64_t full_bar[kPoolMaxStages], empty_bar[kPoolMaxStages];
+  __shared__ float red[kPhases][D];
+  __shared__ float red1[kSplit ? kPhases : 1][kSplit ? D : 1];
+  __shared__ float tot[kRope ? 2 : 1][kRope ? D : 1];
+  __shared__ int abort_sh;
+  volatile int* abort_flag = &abort_sh;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int NS = a.stages;
+  const long long per_bh = static_cast<long long>(a.nQB) + a.nKB;
+  const long long total = static_cast<long long>(a.BH) * per_bh;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], kPoolConsumers / 32);
+    }
+    abort_sh = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
   griddep_wait();
   griddep_launch_dependents();
 
-  const int per_bh = nQB + nKB;
-  const int bh = blockIdx.x / per_bh;
-  int t = blockIdx.x % per_bh;
-  const bool is_key_block = t >= nQB;
-  const __nv_bfloat16* X;
-  int N;
-  float* out;
-  if (t < nQB) {
-    X = Q + static_cast<size_t>(bh) * Nq * D;
-    N = Nq;
-    out = Qp + (static_cast<size_t>(bh) * nQB + t) * D;
-  } else {
-    t -= nQB;
-    X = K + static_cast<size_t>(bh) * Nk * D;
-    N = Nk;
-    out = Kp + (static_cast<size_t>(bh) * nKB + t) * D;
-  }
-  const int lo = t * block;
-  const int hi = min(lo + block, N);
-  const int c = threadIdx.x % kTpr;
-  const int rr = threadIdx.x / kTpr;
-  // first row of the next frame, if this key block reaches it (kParts only)
-  const bool parts = kParts && is_key_block;
-  const int bnd = parts ? min(hi, (lo / T + 1) * T) : hi;
+  // rows [lo, hi) of item `item` and where they live
+  struct Item {
+    const __nv_bfloat16* src;
+    int lo, hi, bh, t;
+    bool key;
+  };
+  auto item_of = [&](long long item) {
+    Item it;
+    it.bh = static_cast<int>(item / per_bh);
+    int t = static_cast<int>(item % per_bh);
+    it.key = t >= a.nQB;
+    if (it.key) t -= a.nQB;
+    it.t = t;
+    const int N = it.key ? a.Nk : a.Nq;
+    it.lo = t * a.block;
+    it.hi = min(it.lo + a.block, N);
+    it.src = (it.key ? a.K : a.Q) + (static_cast<size_t>(it.bh) * N + it.lo) * D;
+    return it;
+  };
 
-  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  for (int base = lo + rr; base < hi; base += kRows * kUnroll) {
-    uint4 v[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int row = base + u * kRows;
-      v[u] = row < hi ? ld_stream_16(X + static_cast<size_t>(row) * D + c * kVec) : make_uint4(0, 0, 0, 0);
+  if (warp == kPoolConsumers / 32) {
+    // ---------------- bulk-copy producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      long long k = 0;
+      for (long long item = blockIdx.x; item < total; item += gridDim.x, ++k) {
+        const int s = static_cast<int>(k % NS), u = static_cast<int>(k / NS);
+        if (u >= 1 && !mbar_wait(&empty_bar[s], (u - 1) & 1, abort_flag, a.timeout_ns, (kKernSelect << 8) | 1))
+          break;
+        if (*abort_flag) break;
+        const Item it = item_of(item);
+        const uint32_t bytes = static_cast<uint32_t>(it.hi - it.lo) * D * 2;
+        issued = static_cast<int>(k) + 1;
+        if (a.inject && k == 0) continue;  // test only: stage 0 never fills
+        mbar_arrive_expect_tx(&full_bar[s], bytes);
+        bulk_load(pool_smem + static_cast<size_t>(s) * a.stage_bytes, it.src, bytes, &full_bar[s]);
+      }
+      // drain: every issued copy must have landed before the CTA may exit
+      for (int kk = max(0, issued - NS); kk < issued; ++kk) {
+        if (a.inject && kk == 0) continue;
+        mbar_wait_drain(&full_bar[kk % NS], (kk / NS) & 1, a.timeout_ns, (kKernSelect << 8) | 2);
+      }
     }
+  } else {
+    // ---------------- consumers ----------------
+    const int c = threadIdx.x % kUnits, rp = threadIdx.x / kUnits;
+    long long k = 0;
+    for (long long item = blockIdx.x; item < total; item += gridDim.x, ++k) {
+      const int s = static_cast<int>(k % NS);
+      const bool ok = mbar_wait(&full_bar[s], static_cast<uint32_t>(k / NS) & 1, abort_flag, a.timeout_ns,
+                                (kKernSelect << 8) | 3);
+      // every consumer has waited (or given up) and the previous item's shared-memory sums
+      // have been read; the decision to stop is the same for all of them
+      if (named_bar_any(1, kPoolConsumers, !ok || *abort_flag != 0)) break;
+      const Item it = item_of(item);
+      const int rows = it.hi - it.lo;
+      // first row of the next frame, relative to the block (kParts key blocks and every
+      // kRope block; else rows)
+      const int split = ((kParts && it.key) || kRope) ? min(rows, (it.lo / a.T + 1) * a.T - it.lo) : rows;
+      const uint8_t* stage = pool_smem + static_cast<size_t>(s) * a.stage_bytes;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float acc1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+      for (int r = rp; r < rows; r += kPhases) {
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + static_cast<size_t>(r) * (D * 2) + c * 16);
+        if (!kSplit || r < split)
+          acc_bf16x8(acc, v);
+        else
+          acc_bf16x8(acc1, v);
+      }
+      // the stage may be refilled once every consumer warp has read it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[s]);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) acc_bf16x8(acc, v[u]);
-  }
-  // the second-frame sum, only in blocks that reach the next frame (CTA-uniform): a short
-  // second pass over those rows, just read and still in L2
-  float acc1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if constexpr (kParts) {
-    if (bnd < hi) {
-      for (int row = lo + rr; row < hi; row += kRows)
-        if (row >= bnd) acc_bf16x8(acc1, ld_stream_16(X + static_cast<size_t>(row) * D + c * kVec));
-    }
-  }
+      for (int e = 0; e < 8; ++e) red[rp][c * 8 + e] = acc[e];
+      if constexpr (kSplit) {
 #pragma unroll
-  for (int k = 0; k < 8; ++k) red[rr * D + c * kVec + k] = acc[k];
-  if constexpr (kParts) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) red1[rr * D + c * kVec + k] = acc1[k];
-  }
-  __syncthreads();
-  if (threadIdx.x < D) {
-    float s = 0.f;
+        for (int e = 0; e < 8; ++e) red1[rp][c * 8 + e] = acc1[e];
+      }
+      named_bar_sync(1, kPoolConsumers);
+      float s0 = 0.f, s1 = 0.f;
+      if (threadIdx.x < D) {
 #pragma unroll 8
-    for (int q = 0; q < kRows; ++q) s += red[q * D + threadIdx.x];
-    out[threadIdx.x] = s / static_cast<float>(hi - lo);
-    if constexpr (kParts) {
-      if (parts) {
-        float s1 = 0.f;
+        for (int q = 0; q < kPhases; ++q) s0 += red[q][threadIdx.x];
+        if constexpr (kSplit) {
 #pragma unroll 8
-        for (int q = 0; q < kRows; ++q) s1 += red1[q * D + threadIdx.x];
-        float* pt = Kpart + ((static_cast<size_t>(bh) * nKB + t) * 2) * D;
-        pt[threadIdx.x] = s - s1;
-        pt[D + threadIdx.x] = s1;
+          for (int q = 0; q < kPhases; ++q) s1 += red1[q][threadIdx.x];
+        }
+      }
+      if constexpr (kRope) {
+        // turn the two frames' sums: pair (2i, 2i+1) needs its partner column
+        if (threadIdx.x < D) {
+          tot[0][threadIdx.x] = s0;
+          tot[1][threadIdx.x] = s1;
+        }
+        named_bar_sync(1, kPoolConsumers);
+        const int t = threadIdx.x;
+        if (t < a.rope_dt) {
+          const int i = t >> 1;
+          const int w0 = (it.key ? 0 : a.q_frame0) + it.lo / a.T;
+          float cs[2], sn[2];
+          rope_cs(rope_index(w0, a.n_frames, a.rope_cap), i, a.rope_dt, a.rope_log2base, cs[0], sn[0]);
+          rope_cs(rope_index(w0 + 1, a.n_frames, a.rope_cap), i, a.rope_dt, a.rope_log2base, cs[1], sn[1]);
+          float r[2];
+#pragma unroll
+          for (int f = 0; f < 2; ++f) {
+            const float x0 = tot[f][2 * i], x1 = tot[f][2 * i + 1];
+            r[f] = (t & 1) ? fmaf(x0, sn[f], x1 * cs[f]) : fmaf(x0, cs[f], -x1 * sn[f]);
+          }
+          s0 = r[0];
+          s1 = r[1];
+        }
+      }
+      if (threadIdx.x < D) {
+        float* out = it.key ? a.Kp + (static_cast<size_t>(it.bh) * a.nKB + it.t) * D
+                            : a.Qp + (static_cast<size_t>(it.bh) * a.nQB + it.t) * D;
+        out[threadIdx.x] = (s0 + s1) / static_cast<float>(rows);
+        if constexpr (kParts) {
+          if (it.key) {
+            float* pt = a.Kpart + ((static_cast<size_t>(it.bh) * a.nKB + it.t) * 2) * D;
+            pt[threadIdx.x] = s0;
+            pt[D + threadIdx.x] = s1;
+          }
+        }
       }
     }
   }
@@ -169,8 +285,10 @@ __global__ void __launch_bounds__(D) pool_frames_kernel(const float* __restrict_
 }
 
 // Scores of kSelQB query blocks of one head per CTA (each pooled K row is read once for
-// all of them), then one warp per query block selects its top r.
-constexpr int kSelQB = 4;
+// all of them), then one warp per query block selects its top r. One query block per CTA:
+// the kernel is bound by the latency of the pooled-K reads from L2, so it wants many
+// CTAs resident (one per query block fills the SMs several times over).
+constexpr int kSelQB = 1;
 
 // Order-preserving map of a float to an unsigned integer (NaN has been replaced by -inf).
 __device__ __forceinline__ uint32_t ordered_bits(float f) {

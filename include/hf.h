@@ -157,6 +157,45 @@ HF_API hf_status hf_select_blocks_two_stage(const hf_bf16* Q, const hf_bf16* K, 
                                             int32_t* idx_out, int32_t* frames_out, float* scores_out, void* ws,
                                             size_t ws_bytes, void* stream);
 
+/* Capped relative temporal RoPE of a chunk step. Source: Hybrid Forcing, German
+ * technical summary section 2 C and Portuguese technical summary section 2 B.2 (the
+ * largest temporal RoPE index is capped, in training and inference alike, and positions
+ * are expressed as relative offsets). Readings where the pages give no numbers:
+ *   - the temporal part acts on dimensions [0, d_t) of every head as consecutive pairs
+ *     (2i, 2i+1), turned by the angle p * base^(-2i/d_t) (textbook RoPE frequencies);
+ *   - a token's index p comes from its frame's offset delta to the newest frame of the
+ *     window: p = cap - min(delta, cap) (the newest frame at cap, every frame cap or more
+ *     frames old at 0);
+ *   - the window K holds ceil(Nk / tokens_per_frame) frames from frame 0; Q's first
+ *     token lies in window frame q_frame0 (the chunk is the window's newest frames);
+ *   - the rotation applies to q and k of the softmax branch and of the block selection;
+ *     the linear branch (readout and absorption) reads the raw q and k.
+ * Q and K are passed unrotated; the kernels turn them on the fly. */
+typedef struct hf_rope {
+  int d_t;               /* rotated dimensions: even, 0 <= d_t <= min(d, 64)             */
+  int tokens_per_frame;  /* >= block                                                    */
+  int cap;               /* index cap P: 0 <= cap <= 63                                 */
+  int q_frame0;          /* window frame of Q's first token, 0 <= q_frame0 < window frames */
+  float base;            /* frequency base (10000 in the textbook form); > 1            */
+} hf_rope;
+
+/* hf_select_blocks on the turned Q and K: the block means are those of the turned tokens
+ * (each block's per-frame sums turned by the frame's index). rope: see hf_rope.
+ * Errors: those of hf_select_blocks, and HF_ERR_INVALID_ARG for a NULL or invalid rope. */
+HF_API hf_status hf_select_blocks_rope(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk, int d,
+                                       int block, int r, const hf_rope* rope, int32_t* idx_out,
+                                       float* scores_out, void* ws, size_t ws_bytes, void* stream);
+
+/* hf_hybrid_attn_fwd with the softmax branch on the turned Q and K (the readout on the raw
+ * Q): O = softmax over the kept blocks of scale * (R q) . (R k), times V, plus
+ * phi(q)^T S / (phi(q) . z + 1e-6). The kernel turns the Q tile and every kept K tile in
+ * shared memory. ws: none. Errors: those of hf_hybrid_attn_fwd, and HF_ERR_INVALID_ARG
+ * for a NULL or invalid rope. */
+HF_API hf_status hf_hybrid_attn_fwd_rope(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H,
+                                         int Nq, int Nk, int d, int block, int r, const int32_t* idx,
+                                         const hf_state* st, float scale, const hf_rope* rope, hf_bf16* O, void* ws,
+                                         size_t ws_bytes, void* stream);
+
 /* Pooled-key cache of the sliding window: the window's keys as fp32 sums of `granule`
  * consecutive tokens, in a ring of `capacity` sums per (b, h). A chunk step sums only the
  * keys that enter the window (hf_kpool_push) and the selection pools its key blocks from

@@ -64,3 +64,22 @@ def test_attention_timeout_is_reported_and_recoverable(name, H):
     want = oracle.hybrid_attention(f64(x["Q"]), f64(x["K"]), f64(x["V"]), idx.cpu().numpy(), f64(st.S),
                                    f64(st.z), wl.block)
     assert_output_close(f64(O), want)
+
+
+def test_select_timeout_is_reported_and_recoverable():
+    """The block pooling's consumers give up on a ring stage that never fills."""
+    wl = WORKLOADS["832x480"]
+    x = draw_step_inputs(wl, n_evicted=1)
+    Q, K = x["Q"][:, :2].contiguous().to(DEV), x["K"][:, :2].contiguous().to(DEV)
+    ref = hf.hf_select_blocks(Q, K, wl.block, wl.r)
+    torch.cuda.synchronize()
+    assert hf.hf_query_status()[0] == hf.HF_OK
+    hf.hf_debug_inject_timeout(1, 1, LIMIT_NS)
+    hf.hf_select_blocks(Q, K, wl.block, wl.r)
+    rc, word = hf.hf_query_status()
+    assert rc == hf.HF_ERR_DEVICE_TIMEOUT, (rc, hex(word))
+    assert (word >> 8) & 0xFF == 1, hex(word)  # reported by the selection's pooling kernel
+    idx = hf.hf_select_blocks(Q, K, wl.block, wl.r)
+    torch.cuda.synchronize()
+    assert hf.hf_query_status()[0] == hf.HF_OK
+    assert torch.equal(idx, ref)
