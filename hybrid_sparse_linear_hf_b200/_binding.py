@@ -45,6 +45,18 @@ class HfKpoolC(ctypes.Structure):
                 ("sums", ctypes.c_void_p)]
 
 
+class HfRopeC(ctypes.Structure):
+    """Mirror of ``struct hf_rope``."""
+
+    _fields_ = [("d_t", ctypes.c_int), ("tokens_per_frame", ctypes.c_int), ("cap", ctypes.c_int),
+                ("q_frame0", ctypes.c_int), ("base", ctypes.c_float)]
+
+
+def hf_rope(d_t: int, tokens_per_frame: int, cap: int, q_frame0: int, base: float = 10000.0) -> HfRopeC:
+    """The temporal RoPE of a chunk step (see ``hf_rope`` in include/hf.h)."""
+    return HfRopeC(int(d_t), int(tokens_per_frame), int(cap), int(q_frame0), float(base))
+
+
 class HfError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -63,6 +75,12 @@ _SIGNATURES = {
                          [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "hf_select_blocks_two_stage": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 9 +
                                    [ctypes.c_void_p] * 4 + [ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_select_blocks_rope": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 +
+                              [ctypes.POINTER(HfRopeC), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                               ctypes.c_size_t, ctypes.c_void_p]),
+    "hf_hybrid_attn_fwd_rope": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
+                                [ctypes.c_void_p, ctypes.POINTER(HfStateC), ctypes.c_float, ctypes.POINTER(HfRopeC),
+                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "hf_select_blocks_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 +
                                  [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "hf_hybrid_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 3 + [ctypes.c_int] * 7 +
@@ -254,6 +272,28 @@ def hf_select_blocks(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, idx_o
     return idx_out
 
 
+def hf_select_blocks_rope(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, rope: HfRopeC, idx_out=None,
+                          scores_out=None, ws=None, stream=None) -> torch.Tensor:
+    """hf_select_blocks on Q and K turned by the temporal RoPE ``rope`` (``hf_rope(...)``)."""
+    B, H, Nq, Nk, d = _qkv_dims(Q, K)
+    nQB, nKB = -(-Nq // block), -(-Nk // block)
+    _shape(idx_out, (B, H, nQB, r), "idx_out")
+    _shape(scores_out, (B, H, nQB, nKB), "scores_out")
+    if not isinstance(rope, HfRopeC):
+        raise TypeError("rope must come from hf_rope(...)")
+    if idx_out is None:
+        idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
+    nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, Nk, d, block, r)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    _check(lib().hf_select_blocks_rope(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), B, H, Nq, Nk, d,
+                                       block, r, ctypes.byref(rope), _dev(idx_out, torch.int32, "idx_out"),
+                                       _dev(scores_out, torch.float32, "scores_out")
+                                       if scores_out is not None else None,
+                                       ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
+           "hf_select_blocks_rope")
+    return idx_out
+
+
 def hf_kpool_init(sums: torch.Tensor, granule: int) -> HfKpool:
     """An empty pooled-key cache over ``sums`` [B,H,capacity,d] fp32 (device): the ring
     of the window's sums of ``granule`` consecutive key tokens."""
@@ -382,6 +422,28 @@ def hf_hybrid_attn_fwd(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block:
                                     _dev(idx, torch.int32, "idx"), ctypes.byref(state.c), float(scale),
                                     _dev(O, torch.bfloat16, "O"), None, 0, _stream(stream)),
            "hf_hybrid_attn_fwd")
+    return O
+
+
+def hf_hybrid_attn_fwd_rope(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, block: int, r: int,
+                            idx: torch.Tensor, state: HfState, rope: HfRopeC, scale: float = 0.0, O=None,
+                            stream=None) -> torch.Tensor:
+    """hf_hybrid_attn_fwd with the softmax branch on Q and K turned by ``rope``."""
+    B, H, Nq, Nk, d = _qkv_dims(Q, K)
+    _shape(V, (B, H, Nk, d), "V")
+    _shape(idx, (B, H, -(-Nq // block), r), "idx")
+    _shape(O, (B, H, Nq, d), "O")
+    if state.shape != (B, H, d):
+        raise ValueError(f"the state's (B, H, d) = {state.shape} must match Q's {(B, H, d)}")
+    if not isinstance(rope, HfRopeC):
+        raise TypeError("rope must come from hf_rope(...)")
+    if O is None:
+        O = torch.empty_like(Q)
+    _check(lib().hf_hybrid_attn_fwd_rope(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"),
+                                         _dev(V, torch.bfloat16, "V"), B, H, Nq, Nk, d, block, r,
+                                         _dev(idx, torch.int32, "idx"), ctypes.byref(state.c), float(scale),
+                                         ctypes.byref(rope), _dev(O, torch.bfloat16, "O"), None, 0, _stream(stream)),
+           "hf_hybrid_attn_fwd_rope")
     return O
 
 

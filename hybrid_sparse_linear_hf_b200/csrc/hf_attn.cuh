@@ -38,6 +38,13 @@
 // when a block maximum exceeds the running max by more than 8, i.e. a factor 256; exact
 // since numerator and denominator share the max); the O rescale is warp-uniform because
 // TMEM access is warp-collective; 3 exp2 pairs in 8 run on the FMA pipe, the rest on MUFU.
+// Temporal RoPE variant (kRope, hf_hybrid_attn_fwd_rope; Hybrid Forcing, German technical
+// summary section 2 C): a fourth warpgroup (warps 12..15, one thread per row) builds a
+// table of (cos, sin) for every index 0..cap and pair, turns the Q tile's first 64
+// columns into a separate buffer (the MMAs read it in place of Q's chunk 0; the raw Q
+// stays for the readout) and every kept K tile in place once it has landed (dimensions
+// [0, d_t), pairs (2i, 2i+1), the index of the row's frame); the MMA issuer and warp 3
+// wait for "turned" in place of "landed". The rings lose one V slot to make room.
 // Linear term, after the last block: phi(q) in fp32 split into bf16 hi + lo (TMEM, over
 // S_B), the state S split into bf16 hi + lo (shared memory, over the idle rings),
 // D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi on the tensor cores (TMEM, over S_A),
@@ -51,28 +58,35 @@ namespace hf {
 
 constexpr uint32_t kKernAttn = 3;
 constexpr int kAttnThreads = 384;
+constexpr int kAttnThreadsRope = 512;  // + the RoPE warpgroup
 constexpr int kRegsSupport = 104;   // registers per thread, producer/MMA warpgroup
+constexpr int kRegsSupportRope = 56;  // producer/MMA and RoPE warpgroups, with the RoPE warpgroup
 constexpr int kRegsRows = 200;     // registers per thread, softmax warpgroups
 static_assert(128 * kRegsSupport + 256 * kRegsRows <= kAttnThreads * 168, "setmaxnreg split exceeds the launch");
+static_assert(2 * 128 * kRegsSupportRope + 256 * kRegsRows <= kAttnThreadsRope * 128,
+              "setmaxnreg split exceeds the launch");
 constexpr int kSmemLimit = 232448;  // max shared memory per CTA on sm_100
 constexpr int kAttnStaticSmem = 1024;  // upper bound of the kernel's static shared memory
 constexpr int kPolyOf8 = 3;         // pairs (of every 8) that take exp2 on the FMA pipe
 constexpr int kMaxSlots = 6;
 
-template <int D, int BLK>
+template <int D, int BLK, bool kRope = false>
 struct AttnCfg {
   static constexpr int kChunks = D / 64;
   static constexpr int kQBytes = 128 * D * 2;
+  static constexpr int kQRotBytes = kRope ? 128 * 128 : 0;   // the Q tile's first 64 columns, turned
+  static constexpr int kTabBytes = kRope ? 64 * 32 * 8 : 0;  // (cos, sin) of index 0..63 x pair 0..31
   static constexpr int kKVTileBytes = BLK * D * 2;
   static constexpr int kReadoutBytes = 2 * D * D * 2;  // S_hi + S_lo (bf16, d x d each)
   static constexpr int kXchBytes = 3 * 2 * 128 * 4;    // end-of-tile exchange [m | l | den][pipe][row]
-  static constexpr int kTiles = (kSmemLimit - kAttnStaticSmem - 1024 - kQBytes) / kKVTileBytes;
+  static constexpr int kTiles =
+      (kSmemLimit - kAttnStaticSmem - 1024 - kQBytes - kQRotBytes - kTabBytes) / kKVTileBytes;
   static constexpr int kKSlots = ((kTiles + 1) / 2) < kMaxSlots ? ((kTiles + 1) / 2) : kMaxSlots;
   static constexpr int kVSlots = (kTiles - kKSlots) < kMaxSlots ? (kTiles - kKSlots) : kMaxSlots;
   static_assert(kKSlots >= 2 && kVSlots >= 2, "ring too small");
   static_assert(kReadoutBytes + kXchBytes <= (kKSlots + kVSlots) * kKVTileBytes,
                 "readout operands and the exchange must fit in the rings");
-  static constexpr int kDynSmem = 1024 + kQBytes + (kKSlots + kVSlots) * kKVTileBytes;
+  static constexpr int kDynSmem = 1024 + kQBytes + kQRotBytes + kTabBytes + (kKSlots + kVSlots) * kKVTileBytes;
   static_assert(kDynSmem + kAttnStaticSmem <= kSmemLimit, "shared memory");
   static constexpr uint32_t kColS = 0;      // S_A at 0, S_B at 128
   static constexpr uint32_t kColO = 256;    // O_A at 256, O_B at 384
@@ -90,25 +104,32 @@ struct AttnParams {
   float scale_log2;    // softmax scale * log2(e)
   unsigned long long timeout_ns;
   int inject;          // test only: the first S-ready commit is skipped
+  // temporal RoPE (kRope): rotated dimensions [0, rope_dt), frames of rope_T tokens, Q's
+  // first token in window frame q_frame0, n_frames window frames, index cap
+  int rope_dt, rope_T, q_frame0, n_frames, rope_cap;
+  float rope_log2base;
 };
 
-template <int D, int BLK>
-__global__ void __launch_bounds__(kAttnThreads, 1)
+template <int D, int BLK, bool kRope = false>
+__global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
     hybrid_attn_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                        const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapO,
                        AttnParams p) {
-  using C = AttnCfg<D, BLK>;
+  using C = AttnCfg<D, BLK, kRope>;
   constexpr int NSK = C::kKSlots;
   constexpr int NSV = C::kVSlots;
   constexpr int HD = C::kHD;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;                             // Q tile; reused as the output staging tile
-  uint8_t* kring = smem + C::kQBytes;              // NSK K slots
+  uint8_t* qrot = sQ + C::kQBytes;                 // kRope: the Q tile's first chunk, turned
+  uint8_t* rtab = qrot + C::kQRotBytes;            // kRope: (cos, sin) table
+  uint8_t* kring = rtab + C::kTabBytes;            // NSK K slots
   uint8_t* vring = kring + NSK * C::kKVTileBytes;  // NSV V slots (S_hi/S_lo + exchange over both rings at the end)
 
   __shared__ uint64_t q_bar, kfull_bar[NSK], kempty_bar[NSK], vfull_bar[NSV], vempty_bar[NSV];
   __shared__ uint64_t sfull_bar[2], pfull_bar[2], final_bar, pro_bar, lin_bar, drain_bar;
+  __shared__ uint64_t qrot_bar, krot_bar[NSK];  // kRope: the Q tile / K slot has been turned
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
 
@@ -136,6 +157,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&pro_bar, 8);  // the 8 softmax warps
     mbar_init(&lin_bar, 1);
     mbar_init(&drain_bar, 1);
+    mbar_init(&qrot_bar, 4);  // the RoPE warpgroup's 4 warps
+    for (int s = 0; s < NSK; ++s) mbar_init(&krot_bar[s], 4);
     abort_sh = 0;
     fence_mbar_init();
   }
@@ -159,9 +182,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   griddep_wait();
   griddep_launch_dependents();
 
+  // With RoPE the Q tile's chunk 0 is read from qrot and a K slot only once turned.
+  uint64_t* q_ready = kRope ? &qrot_bar : &q_bar;
+  uint64_t* k_ready = kRope ? krot_bar : kfull_bar;
+
   if (warp < 4) {
    // warpgroup 0: producers and MMA issuer give registers to the softmax warpgroups
-   warpgroup_reg_dec<kRegsSupport>();
+   warpgroup_reg_dec<kRope ? kRegsSupportRope : kRegsSupport>();
    if (warp == 0 || warp == 2) {
     // ============================ TMA producers ============================
     if (lane == 0) {
@@ -214,6 +241,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       // to the 14-bit start-address field (shared-memory addresses stay below 256 KB, so the
       // field never carries). This keeps the single issuing thread ahead of the tensor core.
       const uint64_t qdesc = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t qrdesc = sdesc_sw128(smem_u32(qrot), 16, 1024);
       const uint64_t kdesc = sdesc_sw128(smem_u32(kring), 16, 1024);
       const uint64_t vdesc = sdesc_sw128(smem_u32(vring), BLK * 128, 1024);
       // The tensor core's instruction queue is shallow: whatever this thread does between
@@ -227,8 +255,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int ks = 0; ks < D / 16; ++ks) {
           constexpr int kQChunk = (128 * 128) >> 4;
           constexpr int kKChunk = (BLK * 128) >> 4;
-          umma_ss(d_tmem, qdesc + (ks / 4) * kQChunk + (ks % 4) * 2, kd + (ks / 4) * kKChunk + (ks % 4) * 2,
-                  idesc_qk, ks > 0 ? 1u : 0u);
+          const uint64_t qa = (kRope && ks < 4) ? qrdesc + (ks % 4) * 2 : qdesc + (ks / 4) * kQChunk + (ks % 4) * 2;
+          umma_ss(d_tmem, qa, kd + (ks / 4) * kKChunk + (ks % 4) * 2, idesc_qk, ks > 0 ? 1u : 0u);
         }
       };
       // O_p += P_p V for kept block v, p = v % 2 (P over the first columns of S_p)
@@ -241,9 +269,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int ks = 0; ks < BLK / 16; ++ks)
           umma_ts(o_tmem, p_tmem + ks * 8, vd + ks * 128, idesc_pv, (v > 1 || ks > 0) ? 1u : 0u);
       };
-      bool ok = mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 4);
+      bool ok = mbar_wait(q_ready, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 4);
       for (int v = 0; v < 2 && v < n && ok; ++v) {
-        if ((ok = mbar_wait(&kfull_bar[v], 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 6))) {
+        if ((ok = mbar_wait(&k_ready[v], 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 6))) {
           tc_fence_after();
           qk(v);
           if (!(p.inject && v == 0)) umma_commit(&sfull_bar[v]);
@@ -304,12 +332,82 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // the MMA issuer runs PV(v) and QK(v+2) on P-ready: their tiles must be there
         if (!mbar_wait(&vfull_bar[v % NSV], (v / NSV) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 14)) break;
         if (v + 2 < n &&
-            !mbar_wait(&kfull_bar[(v + 2) % NSK], ((v + 2) / NSK) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 15))
+            !mbar_wait(&k_ready[(v + 2) % NSK], ((v + 2) / NSK) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 15))
           break;
         mbar_arrive(&pfull_bar[pp]);
       }
     }
    }
+  } else if (warp >= 12) {
+    // ============== temporal RoPE warpgroup: turns the Q tile and every kept K tile ==============
+    warpgroup_reg_dec<kRegsSupportRope>();
+    if constexpr (kRope) {
+      const int rt = threadIdx.x - 384;  // a row of the Q tile, or of a K tile
+      const int npair = p.rope_dt / 2;
+      const int nunits = (p.rope_dt + 7) / 8;  // 16-byte units of chunk 0 that hold turned pairs
+      float2* tab = reinterpret_cast<float2*>(rtab);  // [index][pair]
+      for (int e = rt; e < (p.rope_cap + 1) * 32; e += 128) {
+        const int pi = e / 32, i = e % 32;
+        float c = 1.f, sn = 0.f;
+        if (i < npair) {
+          const float theta = exp2f(-static_cast<float>(2 * i) / static_cast<float>(p.rope_dt) * p.rope_log2base);
+          sincosf(static_cast<float>(pi) * theta, &sn, &c);
+        }
+        tab[e] = make_float2(c, sn);
+      }
+      named_bar_sync(2, 128);
+      // index of window frame w (newest at the cap); padding rows clamp into the table
+      auto index_of = [&](int w) { return min(max(p.rope_cap - min((p.n_frames - 1) - w, p.rope_cap), 0), p.rope_cap); };
+      // units [0, nunits) of one 128-byte row of a 128B-swizzled chunk turned from src to dst,
+      // units [nunits, nall) copied
+      auto turn_row = [&](const uint8_t* src, uint8_t* dst, int row, int pidx, int nall) {
+        const float2* trow = tab + pidx * 32;
+        for (int u = 0; u < nall; ++u) {
+          const uint32_t off = row * 128 + ((u ^ (row & 7)) * 16);
+          const uint4 w = *reinterpret_cast<const uint4*>(src + off);
+          uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          if (u < nunits) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int i = 4 * u + e;
+              if (i < npair) {
+                const float x0 = bf16_lo_to_f32(ww[e]), x1 = bf16_hi_to_f32(ww[e]);
+                const float2 cs = trow[i];
+                ww[e] = pack_bf16x2(fmaf(x0, cs.x, -x1 * cs.y), fmaf(x0, cs.y, x1 * cs.x));
+              }
+            }
+          }
+          *reinterpret_cast<uint4*>(dst + off) = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+        }
+      };
+      // the Q tile: chunk 0 into qrot (every unit, the first nunits turned)
+      bool ok = mbar_wait(&q_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 20);
+      if (ok) {
+        const int tok = I * BLK + rt;  // token of the chunk (rows past Nq hold TMA zeros)
+        turn_row(sQ, qrot, rt, index_of(p.q_frame0 + tok / p.rope_T), 8);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&qrot_bar);
+      }
+      // every kept K tile, in place, in kept-block order
+      int v = 0;
+      for (int jj = 0; jj < p.r && ok; ++jj) {
+        const int J = __ldg(idx_row + jj);
+        if (J < 0 || J >= p.nKB) continue;
+        const int s = v % NSK;
+        ok = mbar_wait(&kfull_bar[s], (v / NSK) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 21);
+        if (!ok) break;
+        const bool valid = rt < BLK && (J < p.nKB - 1 || rt < p.last_len);
+        if (valid) {
+          uint8_t* ktile = kring + s * C::kKVTileBytes;  // chunk 0: BLK rows x 128 B
+          turn_row(ktile, ktile, rt, index_of((J * BLK + rt) / p.rope_T), nunits);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&krot_bar[s]);
+        ++v;
+      }
+    }
   } else {
     warpgroup_reg_inc<kRegsRows>();
     // ======================= softmax pipelines, readout, epilogue =======================

@@ -22,7 +22,6 @@
 
 namespace {
 
-using hf::AttnCfg;
 
 constexpr unsigned long long kDefaultTimeoutNs = 1000000000ull;  // 1 s per wait
 // CTAs the absorption spreads a call over (one per SM of a B200). A constant, so the
@@ -135,14 +134,15 @@ int sm_count() {
   return n;
 }
 
-// Checks of an hf_rope for a step with window Nk and blocks of `block` tokens.
-bool rope_ok(const hf_rope* rope, int d, int Nk, int block) {
+// Checks of an hf_rope for a step with Nq queries, a window of Nk keys and blocks of
+// `block` tokens: the chunk must lie inside the window's frames.
+bool rope_ok(const hf_rope* rope, int d, int Nq, int Nk, int block) {
   if (!rope) return false;
   if (rope->d_t < 0 || (rope->d_t & 1) || rope->d_t > d || rope->d_t > 64) return false;
   if (rope->tokens_per_frame < block || rope->cap < 0 || rope->cap > 63) return false;
   if (!(rope->base > 1.0f) || std::isinf(rope->base)) return false;
   const int W = ceil_div(Nk, rope->tokens_per_frame);
-  return rope->q_frame0 >= 0 && rope->q_frame0 < W;
+  return rope->q_frame0 >= 0 && static_cast<long long>(rope->q_frame0) + ceil_div(Nq, rope->tokens_per_frame) <= W;
 }
 
 // Block pooling of Q (and K unless nKB == 0) by the persistent bulk-copy kernel; with a
@@ -336,10 +336,11 @@ hf_status launch_absorb(hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, 
 }
 
 // ---------------------------------------------------------------- attention
-template <int D, int BLK>
+template <int D, int BLK, bool kRope = false>
 hf_status launch_attn(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int BH, int Nq, int Nk, int r,
-                      const int32_t* idx, const hf_state* st, float scale, hf_bf16* O, cudaStream_t stream) {
-  using C = AttnCfg<D, BLK>;
+                      const int32_t* idx, const hf_state* st, float scale, hf_bf16* O, cudaStream_t stream,
+                      const hf_rope* rope = nullptr) {
+  using C = hf::AttnCfg<D, BLK, kRope>;
   const int nQB = ceil_div(Nq, BLK), nKB = ceil_div(Nk, BLK);
   CUtensorMap mq, mk, mv, mo;
   if (make_map(&mq, Q, D, Nq, BH, 128) != HF_OK || make_map(&mk, K, D, Nk, BH, BLK) != HF_OK ||
@@ -355,11 +356,21 @@ hf_status launch_attn(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int 
   p.last_len = Nk - (nKB - 1) * BLK;
   p.scale_log2 = scale * 1.4426950408889634f;
   take_injection(3, &p.inject, &p.timeout_ns);
-  if (cudaFuncSetAttribute(hf::hybrid_attn_kernel<D, BLK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  p.rope_dt = p.rope_T = p.q_frame0 = p.n_frames = p.rope_cap = 0;
+  p.rope_log2base = 0.f;
+  if (kRope) {
+    p.rope_dt = rope->d_t;
+    p.rope_T = rope->tokens_per_frame;
+    p.q_frame0 = rope->q_frame0;
+    p.n_frames = ceil_div(Nk, rope->tokens_per_frame);
+    p.rope_cap = rope->cap;
+    p.rope_log2base = std::log2(rope->base);
+  }
+  if (cudaFuncSetAttribute(hf::hybrid_attn_kernel<D, BLK, kRope>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kDynSmem) != cudaSuccess)
     return HF_ERR_CUDA;
-  return launch_pdl(hf::hybrid_attn_kernel<D, BLK>, static_cast<long long>(BH) * nQB, hf::kAttnThreads, C::kDynSmem,
-                    stream, mq, mk, mv, mo, p);
+  return launch_pdl(hf::hybrid_attn_kernel<D, BLK, kRope>, static_cast<long long>(BH) * nQB,
+                    kRope ? hf::kAttnThreadsRope : hf::kAttnThreads, C::kDynSmem, stream, mq, mk, mv, mo, p);
 }
 
 __global__ void debug_exp2_kernel(const float* __restrict__ x, float* __restrict__ yp, float* __restrict__ ym,
@@ -465,14 +476,17 @@ hf_status check_absorb_args(const hf_state* st, const hf_bf16* K_ev, const hf_bf
   return HF_OK;
 }
 
-// The attention launch for already-checked arguments with Nq >= 1.
+// The attention launch for already-checked arguments with Nq >= 1 (rope: the temporal
+// RoPE variant, or NULL).
 hf_status dispatch_attn(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H, int Nq, int Nk, int d,
                         int block, int r, const int32_t* idx, const hf_state* st, float scale, hf_bf16* O,
-                        cudaStream_t s) {
+                        cudaStream_t s, const hf_rope* rope = nullptr) {
   const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
   const int bh = B * H;
-#define HF_ATTN_CASE(DD, BB) \
-  if (d == DD && block == BB) return launch_attn<DD, BB>(Q, K, V, bh, Nq, Nk, r, idx, st, sc, O, s);
+#define HF_ATTN_CASE(DD, BB)                                                                               \
+  if (d == DD && block == BB)                                                                              \
+    return rope ? launch_attn<DD, BB, true>(Q, K, V, bh, Nq, Nk, r, idx, st, sc, O, s, rope)                \
+                : launch_attn<DD, BB>(Q, K, V, bh, Nq, Nk, r, idx, st, sc, O, s);
   HF_ATTN_CASE(128, 128)
   HF_ATTN_CASE(128, 64)
   HF_ATTN_CASE(128, 32)
@@ -583,7 +597,7 @@ HF_API hf_status hf_select_blocks_rope(const hf_bf16* Q, const hf_bf16* K, int B
   const int nKB = ceil_div(Nk, block);
   if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
   if (nKB > hf::kMaxKeyBlocks) return HF_ERR_UNSUPPORTED;
-  if (!rope_ok(rope, d, Nk, block)) return HF_ERR_INVALID_ARG;
+  if (!rope_ok(rope, d, Nq, Nk, block)) return HF_ERR_INVALID_ARG;
   if (Nq == 0) return HF_OK;
   if (!Q || !K || !idx_out) return HF_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(idx_out) || (scores_out && !aligned16(scores_out)))
@@ -708,6 +722,20 @@ HF_API hf_status hf_hybrid_attn_fwd(const hf_bf16* Q, const hf_bf16* K, const hf
   const hf_status rc = check_attn_args(Q, K, V, B, H, Nq, Nk, d, block, r, idx, st, scale, O);
   if (rc != HF_OK || Nq == 0) return rc;
   return dispatch_attn(Q, K, V, B, H, Nq, Nk, d, block, r, idx, st, scale, O, static_cast<cudaStream_t>(stream));
+}
+
+HF_API hf_status hf_hybrid_attn_fwd_rope(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H,
+                                         int Nq, int Nk, int d, int block, int r, const int32_t* idx,
+                                         const hf_state* st, float scale, const hf_rope* rope, hf_bf16* O, void* ws,
+                                         size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  const hf_status rc = check_attn_args(Q, K, V, B, H, Nq, Nk, d, block, r, idx, st, scale, O);
+  if (rc != HF_OK) return rc;
+  if (!rope_ok(rope, d, Nq, Nk, block)) return HF_ERR_INVALID_ARG;
+  if (Nq == 0) return HF_OK;
+  return dispatch_attn(Q, K, V, B, H, Nq, Nk, d, block, r, idx, st, scale, O, static_cast<cudaStream_t>(stream),
+                       rope);
 }
 
 HF_API hf_status hf_hybrid_attn_fwd_absorb(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int B, int H,

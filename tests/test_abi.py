@@ -308,3 +308,35 @@ def test_fused_attention_absorb_validation():
     st = _state()
     assert call(st=st, Nq=0, n=0, Kev=None, Vev=None, ws=None) == B.HF_OK   # nothing to do
     assert st.n_absorbed == 0
+
+
+def test_rope_validation():
+    """The RoPE entry points reject an invalid or missing rope before any launch."""
+    L = hf.lib()
+
+    def sel(rope, **kw):
+        a = dict(Q=A, K=A, B=1, H=1, Nq=64, Nk=256, d=64, block=32, r=2, idx=A, ws=A, ws_bytes=1 << 20)
+        a.update(kw)
+        return L.hf_select_blocks_rope(a["Q"], a["K"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], a["block"], a["r"],
+                                       ctypes.byref(rope) if rope is not None else None, a["idx"], None, a["ws"],
+                                       a["ws_bytes"], None)
+
+    def fwd(rope, **kw):
+        a = dict(Q=A, K=A, V=A, B=1, H=1, Nq=64, Nk=256, d=64, block=32, r=2, idx=A, O=A)
+        a.update(kw)
+        st = _state()
+        return L.hf_hybrid_attn_fwd_rope(a["Q"], a["K"], a["V"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"],
+                                         a["block"], a["r"], a["idx"], ctypes.byref(st), 0.0,
+                                         ctypes.byref(rope) if rope is not None else None, a["O"], None, 0, None)
+
+    good = hf.hf_rope(16, 64, 3, 3)   # window 256 keys = 4 frames of 64; a 1-frame chunk at frame 3
+    for call in (sel, fwd):
+        assert call(good, Nq=0) == B.HF_OK
+        assert call(None) == B.HF_ERR_INVALID_ARG
+        assert call(hf.hf_rope(15, 64, 3, 3)) == B.HF_ERR_INVALID_ARG    # odd d_t
+        assert call(hf.hf_rope(66, 64, 3, 3)) == B.HF_ERR_INVALID_ARG    # d_t > d
+        assert call(hf.hf_rope(16, 16, 3, 3)) == B.HF_ERR_INVALID_ARG    # frames shorter than a block
+        assert call(hf.hf_rope(16, 64, 64, 3)) == B.HF_ERR_INVALID_ARG   # cap > 63
+        assert call(hf.hf_rope(16, 64, 3, 4)) == B.HF_ERR_INVALID_ARG    # the chunk past the window
+        assert call(hf.hf_rope(16, 64, 3, 3, base=1.0)) == B.HF_ERR_INVALID_ARG
+        assert call(hf.hf_rope(16, 64, 3, 3), r=9) == B.HF_ERR_INVALID_ARG
