@@ -3,15 +3,17 @@
 One step = one pass of the whole hot path over one chunk of the 832x480-shaped
 workload (B=1, H=12, d=128, 4680 queries, 32760-key window, block 128, top-64 of 256
 key blocks, state built from 60 evicted frames):
-    hf_select_blocks      block mean pooling, scores, top-r          (2 kernels)
-    hf_hybrid_attn_fwd    sparse attention + linear readout, summed  (1 kernel)
-    hf_absorb_evicted     the chunk step's 3 evicted frames -> state
+    hf_select_blocks           block mean pooling, scores, top-r                (2 kernels)
+    hf_hybrid_attn_fwd_absorb  sparse attention + linear readout, summed, then the
+                               chunk step's 3 evicted frames -> state           (3 kernels)
 Metric: query tokens/s per chunk step (whole job, all GPUs), with the roofline fraction
 of the dominant kernel (hf_hybrid_attn_fwd, tensor-bound) against the measured bf16
-peak. Legs reported beside the step: the 60-frame state build, the two-stage (frame,
+peak (timed alone in its own leg, as are the selection and the absorption). Legs
+reported beside the step: the 60-frame state build, the two-stage (frame,
 then block) selection, the selection from the pooled-key cache (with the push of the
 chunk's keys), the attention at keep 1 / 0.5 / 0.25 / 0.125, a video's first 12 chunks
-under the chunk-aware growth keep schedule, the 1280x720-shaped step (attention,
+under the chunk-aware growth keep schedule, the selection and attention with the capped
+relative temporal RoPE, the 1280x720-shaped step (attention,
 selection, 120-frame state build), and a streaming end-to-end step: the chunk's Q, K, V
 copied in from pinned host memory, the device-resident window shifted by the chunk, the
 evicted frames absorbed, O copied back.
@@ -72,6 +74,10 @@ SCHEDULE_S_BASE = 0.85
 SCHEDULE_S_TARGET = 0.75
 # pooled-key cache leg: tokens per granule sum (divides the 4680-key chunk and the block)
 KPOOL_GRANULE = 8
+# temporal RoPE leg: 44 of the 128 dimensions turned (a 3-D video RoPE's temporal share,
+# 128 - 2 x 42), the index capped at 8 frames (a 9-frame window)
+ROPE_DT = 44
+ROPE_CAP = 8
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -488,17 +494,15 @@ def run_gpu(args, wl) -> None:
     O = torch.empty_like(Q)
 
     def step(ev=None):
+        # select, then the attention and the absorption of the step's evicted frames in one
+        # call (the absorption's partial sums run beside the attention's last CTAs); events
+        # only around the whole step, so that no event sits between dependent launches
         if ev:
             ev[0].record(stream)
         hf.hf_select_blocks(Q, K, wl.block, wl.r, idx_out=idx, ws=ws_sel)
+        hf.hf_hybrid_attn_fwd_absorb(Q, K, V, wl.block, wl.r, idx, st, K_ev, V_ev, O=O, ws=ws_abs)
         if ev:
             ev[1].record(stream)
-        hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wl.r, idx, st, O=O)
-        if ev:
-            ev[2].record(stream)
-        hf.hf_absorb_evicted(st, K_ev, V_ev, ws=ws_abs)
-        if ev:
-            ev[3].record(stream)
 
     log("warm-up")
     for i in range(max(args.warmup, 3)):
@@ -511,7 +515,7 @@ def run_gpu(args, wl) -> None:
     check_status(hf, "warm-up")
     idx_host = idx.cpu().numpy()
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
@@ -526,15 +530,33 @@ def run_gpu(args, wl) -> None:
     if dist:
         dist.barrier()
     check_status(hf, "timing")
-    t_sel = [e[0].elapsed_time(e[1]) * 1e-3 for e in events]
-    t_fwd = [e[1].elapsed_time(e[2]) * 1e-3 for e in events]
-    t_abs = [e[2].elapsed_time(e[3]) * 1e-3 for e in events]
-    t_step_local = sum(e[0].elapsed_time(e[3]) for e in events) * 1e-3 / args.steps
+    t_step_local = sum(e[0].elapsed_time(e[1]) for e in events) * 1e-3 / args.steps
     t_step = max_over_ranks(t_step_local, dist, dev)
+
+    # ---- each call of the step timed alone (the attention's time gives the roofline)
+    log("per-call legs")
+    n_leg = max(3, min(args.steps, 50))
+    t_sel = timer.run(lambda: hf.hf_select_blocks(Q, K, wl.block, wl.r, idx_out=idx, ws=ws_sel), n=n_leg, warm=3)
+    attn_launches0 = hf.hf_launch_count()
+    t_fwd = timer.run(lambda: hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wl.r, idx, st, O=O), n=n_leg, warm=3)
+    attn_launches = hf.hf_launch_count() - attn_launches0
+    t_abs = timer.run(lambda: hf.hf_absorb_evicted(st, K_ev, V_ev, ws=ws_abs), n=n_leg, warm=3)
+    t_fused = timer.run(lambda: hf.hf_hybrid_attn_fwd_absorb(Q, K, V, wl.block, wl.r, idx, st, K_ev, V_ev, O=O,
+                                                             ws=ws_abs), n=n_leg, warm=3)
+    check_status(hf, "the per-call legs")
+    # ---- capped relative temporal RoPE: the selection and the attention on turned Q, K
+    log("rope leg")
+    rope = hf.hf_rope(ROPE_DT, wl.tokens_per_frame, ROPE_CAP, wl.window_frames - wl.chunk_frames)
+    idx_rope = torch.empty_like(idx)
+    t_sel_rope = timer.run(lambda: hf.hf_select_blocks_rope(Q, K, wl.block, wl.r, rope, idx_out=idx_rope,
+                                                            ws=ws_sel), n=n_leg, warm=3)
+    t_fwd_rope = timer.run(lambda: hf.hf_hybrid_attn_fwd_rope(Q, K, V, wl.block, wl.r, idx_rope, st, rope, O=O),
+                           n=n_leg, warm=3)
+    check_status(hf, "the rope leg")
+    F_rope = attn_flops(idx_rope.cpu().numpy(), wl)
 
     log(f"timed: {t_step_local * 1e3:.3f} ms/step; two-stage selection leg")
     # ---- two-stage (frame, then block) selection, timed alone beside the step
-    n_leg = max(3, min(args.steps, 50))
     ws_sel2 = torch.empty(hf.hf_workspace_size(hf.HF_WS_SELECT_TWO_STAGE, wl.B, wl.H, wl.Nq, wl.Nk, wl.d, wl.block,
                                                wl.r), dtype=torch.uint8, device=dev)
     idx2 = torch.empty_like(idx)
@@ -649,6 +671,17 @@ def run_gpu(args, wl) -> None:
             "hf_absorb_evicted_step": {"us": abs_mean * 1e6, "tokens": wl.Ne_step,
                                        "bytes": absorb_bytes(wl, wl.Ne_step),
                                        "gbs": absorb_bytes(wl, wl.Ne_step) / abs_mean / 1e9},
+            "hf_hybrid_attn_fwd_absorb": {"us": statistics.mean(t_fused) * 1e6,
+                                          "saved_us": (fwd_mean + abs_mean - statistics.mean(t_fused)) * 1e6,
+                                          "note": "attention + the step's absorption in one call, against the two "
+                                                  "calls timed alone"},
+            "rope": {"d_t": ROPE_DT, "cap": ROPE_CAP, "q_frame0": wl.window_frames - wl.chunk_frames,
+                     "hf_select_blocks_rope_us": statistics.mean(t_sel_rope) * 1e6,
+                     "hf_hybrid_attn_fwd_rope_us": statistics.mean(t_fwd_rope) * 1e6,
+                     "attn_tflops": F_rope / statistics.mean(t_fwd_rope) / 1e12,
+                     "attn_frac": F_rope / statistics.mean(t_fwd_rope) / 1e12 / peaks["bf16_tflops"],
+                     "attn_cost_vs_plain": statistics.mean(t_fwd_rope) / fwd_mean - 1.0,
+                     "select_cost_vs_plain": statistics.mean(t_sel_rope) / sel_mean - 1.0},
             "hf_absorb_evicted_state_build": {"us": build_mean * 1e6, "tokens": wl.Ne_state,
                                               "bytes": absorb_bytes(wl, wl.Ne_state),
                                               "gbs": absorb_bytes(wl, wl.Ne_state) / build_mean / 1e9,
@@ -661,6 +694,7 @@ def run_gpu(args, wl) -> None:
         "large_workload": large,
         "gpu_launches": launches,
         "gpu_launches_source": "hf_launch_count() difference over the timed steps (the library's own launches)",
+        "attn_launches_per_call": attn_launches / (n_leg + 3),
         "clocks": clk.summary(),
         "e2e": e2e,
     }
@@ -693,10 +727,11 @@ def streaming_e2e_leg(hf, wl, dev, stream, x, st, ws_sel, ws_abs, args, dist) ->
     the first host-to-device copy to the last device-to-host copy. Per step: the chunk's
     Q and its new K, V (Nq tokens each) are copied from pinned host memory on an upload
     stream (double-buffered, so step k+1's copy overlaps step k's compute); the window
-    (device-resident, ping-pong buffers) drops its oldest Nq tokens, which are absorbed
-    into the state, and appends the chunk's keys and values; then the selection and the
-    hybrid attention of the chunk; O goes back to pinned host memory on a download
-    stream. Bytes: 3 x Nq x d bf16 per head in, Nq x d bf16 per head out."""
+    (device-resident, ping-pong buffers) drops its oldest Nq tokens (absorbed into the
+    state at the end of the previous step) and appends the chunk's keys and values; then
+    the selection and, in one call, the chunk's hybrid attention and the absorption of the
+    window's oldest chunk, which leaves it at the next step; O goes back to pinned host
+    memory on a download stream. Bytes: 3 x Nq x d bf16 per head in, Nq x d bf16 per head out."""
     B, H, Nq, Nk, d = wl.B, wl.H, wl.Nq, wl.Nk, wl.d
     shp = (B, H, Nq, d)
     host_in = [torch.empty(shp, dtype=torch.bfloat16, pin_memory=True) for _ in range(3)]
@@ -730,16 +765,18 @@ def streaming_e2e_leg(hf, wl, dev, stream, x, st, ws_sel, ws_abs, args, dist) ->
         if k >= 2:
             stream.wait_event(downloaded[b])  # O of step k-2 has left this output buffer
         q, k_new, v_new = dev_in[b]
-        # the oldest chunk leaves the window and enters the state; the new chunk enters
-        k_ev.copy_(win_k[cur][:, :, :Nq])
-        v_ev.copy_(win_v[cur][:, :, :Nq])
+        # the window drops its oldest chunk (absorbed at the end of the previous step) and
+        # takes the new one
         win_k[nxt][:, :, :Nk - Nq].copy_(win_k[cur][:, :, Nq:])
         win_v[nxt][:, :, :Nk - Nq].copy_(win_v[cur][:, :, Nq:])
         win_k[nxt][:, :, Nk - Nq:].copy_(k_new)
         win_v[nxt][:, :, Nk - Nq:].copy_(v_new)
-        hf.hf_absorb_evicted(st, k_ev, v_ev, ws=ws_abs)
+        # the chunk that leaves the window next: absorbed right after this step's attention
+        k_ev.copy_(win_k[nxt][:, :, :Nq])
+        v_ev.copy_(win_v[nxt][:, :, :Nq])
         hf.hf_select_blocks(q, win_k[nxt], wl.block, wl.r, idx_out=idx, ws=ws_sel)
-        hf.hf_hybrid_attn_fwd(q, win_k[nxt], win_v[nxt], wl.block, wl.r, idx, st, O=dev_out[b])
+        hf.hf_hybrid_attn_fwd_absorb(q, win_k[nxt], win_v[nxt], wl.block, wl.r, idx, st, k_ev, v_ev,
+                                     O=dev_out[b], ws=ws_abs)
         computed[b].record(stream)
         down.wait_event(computed[b])
         with torch.cuda.stream(down):
@@ -770,8 +807,8 @@ def streaming_e2e_leg(hf, wl, dev, stream, x, st, ws_sel, ws_abs, args, dist) ->
     return {"value": job_throughput(world, B, Nq, t), "unit": UNIT, "h2d_bytes_per_step": 3 * nbytes,
             "d2h_bytes_per_step": nbytes, "steps": n_e2e, "ms_per_step": t * 1e3,
             "note": "streaming: per step the chunk's Q, K, V (4680 tokens) in from pinned host memory on an upload "
-                    "stream overlapping the previous step, window shift and absorption of the evicted chunk on "
-                    "the device, select + attention, O out to pinned host memory"}
+                    "stream overlapping the previous step, window shift on the device, select, attention + "
+                    "absorption of the chunk leaving the window (one call), O out to pinned host memory"}
 
 
 def main() -> None:
