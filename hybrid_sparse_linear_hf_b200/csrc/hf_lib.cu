@@ -203,6 +203,16 @@ size_t select_ws_bytes(int B, int H, int Nq, int Nk, int d, int block) {
 template <int D>
 hf_status launch_score(const float* Qp, const float* Kp, int BH, int nQB, int nKB, int r, int32_t* idx,
                        float* scores, cudaStream_t st) {
+  const long long ngroups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
+  if (static_cast<long long>(nKB) * D * 4 <= hf::kStagedKBytes) {
+    // the head's pooled K rows staged in shared memory by bulk copies
+    const size_t smem = static_cast<size_t>(nKB) * D * 4 + static_cast<size_t>(nKB) * hf::kSelQB * sizeof(float);
+    if (cudaFuncSetAttribute(hf::score_select_staged_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return HF_ERR_CUDA;
+    return launch_pdl(hf::score_select_staged_kernel<D>, static_cast<long long>(BH) * ngroups, hf::kSelectThreads,
+                      smem, st, Qp, Kp, nQB, nKB, r, idx, scores, kDefaultTimeoutNs);
+  }
   // the opt-in covers static + dynamic shared memory above the 48 KB default; set on
   // every launch so that no size of nKB depends on it having been set before
   const size_t smem = static_cast<size_t>(nKB) * hf::kSelQB * sizeof(float);

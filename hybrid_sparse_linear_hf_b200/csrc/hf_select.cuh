@@ -285,10 +285,8 @@ __global__ void __launch_bounds__(D) pool_frames_kernel(const float* __restrict_
 }
 
 // Scores of kSelQB query blocks of one head per CTA (each pooled K row is read once for
-// all of them), then one warp per query block selects its top r. One query block per CTA:
-// the kernel is bound by the latency of the pooled-K reads from L2, so it wants many
-// CTAs resident (one per query block fills the SMs several times over).
-constexpr int kSelQB = 1;
+// all of them), then one warp per query block selects its top r.
+constexpr int kSelQB = 4;
 
 // Order-preserving map of a float to an unsigned integer (NaN has been replaced by -inf).
 __device__ __forceinline__ uint32_t ordered_bits(float f) {
@@ -433,6 +431,88 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const floa
   score_rows<D>(q_sh, Kp + static_cast<size_t>(bh) * nKB * D, nKB, s_sc);
   __syncthreads();
 
+  if (warp < G) {
+    const int I = I0 + warp;
+    const float* srow = s_sc + warp * nKB;
+    float* sout = scores_out ? scores_out + (static_cast<size_t>(bh) * nQB + I) * nKB : nullptr;
+    if (sout)
+      for (int J = lane; J < nKB; J += 32) sout[J] = srow[J];
+    warp_top_r_scores(srow, nKB, r, lane, idx_out + (static_cast<size_t>(bh) * nQB + I) * r);
+  }
+}
+
+// score_select_kernel with the head's pooled K rows staged in shared memory: they are
+// contiguous ([nKB][D] fp32), so a few bulk copies bring them in at once instead of each
+// thread waiting on its row's L2 loads (the plain kernel is bound by those latencies).
+// Used when nKB * D * 4 bytes fit (kStagedKBytes). Thread J reads its row starting at
+// 16-byte unit J % 32 (rotated), so the 32 lanes of a warp hit distinct banks.
+constexpr int kStagedKBytes = 192 * 1024;
+constexpr int kStageCopyBytes = 32 * 1024;
+
+template <int D>
+__global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(const float* __restrict__ Qp,
+                                                                             const float* __restrict__ Kp, int nQB,
+                                                                             int nKB, int r,
+                                                                             int32_t* __restrict__ idx_out,
+                                                                             float* __restrict__ scores_out,
+                                                                             unsigned long long timeout_ns) {
+  extern __shared__ __align__(128) float st_smem[];
+  float* krows = st_smem;                                 // [nKB][D]
+  float* s_sc = st_smem + static_cast<size_t>(nKB) * D;   // [kSelQB][nKB]
+  __shared__ __align__(16) float q_sh[kSelQB][D];
+  __shared__ uint64_t kbar;
+  const int groups = (nQB + kSelQB - 1) / kSelQB;
+  const int bh = blockIdx.x / groups;
+  const int I0 = (blockIdx.x % groups) * kSelQB;
+  const int G = min(kSelQB, nQB - I0);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t kbytes = static_cast<uint32_t>(nKB) * D * 4;
+  if (threadIdx.x == 0) {
+    mbar_init(&kbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  griddep_wait();
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(Kp + static_cast<size_t>(bh) * nKB * D);
+    mbar_arrive_expect_tx(&kbar, kbytes);
+    for (uint32_t o = 0; o < kbytes; o += kStageCopyBytes)
+      bulk_load(reinterpret_cast<uint8_t*>(krows) + o, src + o, min(kStageCopyBytes, static_cast<int>(kbytes - o)),
+                &kbar);
+  }
+  for (int i = threadIdx.x; i < kSelQB * D; i += kSelectThreads) {
+    const int g = i / D;
+    q_sh[g][i % D] = Qp[(static_cast<size_t>(bh) * nQB + I0 + min(g, G - 1)) * D + i % D];
+  }
+  __syncthreads();
+  // every thread waits for the rows (the copies cannot be abandoned: the wait ignores the
+  // abort flag but stays bounded)
+  const bool landed = mbar_wait_drain(&kbar, 0, timeout_ns, (kKernSelect << 8) | 4);
+  if (__syncthreads_or(!landed)) return;
+  constexpr int kU = D / 4;  // 16-byte units per row
+  for (int J = threadIdx.x; J < nKB; J += kSelectThreads) {
+    const float4* krow = reinterpret_cast<const float4*>(krows + static_cast<size_t>(J) * D);
+    float acc[kSelQB];
+#pragma unroll
+    for (int g = 0; g < kSelQB; ++g) acc[g] = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < kU; ++k) {
+      const int u = (k + J) % kU;
+      const float4 kv = krow[u];
+#pragma unroll
+      for (int g = 0; g < kSelQB; ++g) {
+        const float4 qv = *reinterpret_cast<const float4*>(&q_sh[g][4 * u]);
+        acc[g] = fmaf(qv.x, kv.x, acc[g]);
+        acc[g] = fmaf(qv.y, kv.y, acc[g]);
+        acc[g] = fmaf(qv.z, kv.z, acc[g]);
+        acc[g] = fmaf(qv.w, kv.w, acc[g]);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < kSelQB; ++g) s_sc[g * nKB + J] = acc[g];
+  }
+  __syncthreads();
   if (warp < G) {
     const int I = I0 + warp;
     const float* srow = s_sc + warp * nKB;
