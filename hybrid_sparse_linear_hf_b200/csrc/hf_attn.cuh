@@ -522,13 +522,49 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
       ++i;
     }
 
-    // ---- linear term operands (all MMAs done: the S buffers and both rings are free)
+    // ---- linear term operands. This thread's halves of z and of S's row `row` do not depend
+    // on the MMAs: their loads are issued before the wait for the last MMAs, so that their
+    // L2 latency hides behind it, and the conversions below read registers.
+    constexpr int kQ4 = HD / 4;  // float4 per half row
+    float4 zv[kQ4], sv[kQ4];
+    {
+      const float4* z4 = reinterpret_cast<const float4*>(p.z + static_cast<size_t>(bh) * D + pipe * HD);
+      const float4* s4 =
+          reinterpret_cast<const float4*>(p.S + (static_cast<size_t>(bh) * D + min(row, D - 1)) * D + pipe * HD);
+#pragma unroll
+      for (int k = 0; k < kQ4; ++k) {
+        zv[k] = __ldg(z4 + k);
+        sv[k] = __ldg(s4 + k);
+      }
+    }
+    // (all MMAs done: the S buffers and both rings are free)
     ok = ok && mbar_wait(&final_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 12);
     ok = __all_sync(0xffffffffu, ok);
     float dacc = 0.f;
     if (ok) {
       tc_fence_after();
-      const float* zrow = p.z + static_cast<size_t>(bh) * D;
+      // state rows: thread (k, pipe) converts S[bh][k][pipe*D/2 .. +D/2) into MN-major
+      // bf16 hi/lo tiles over the idle rings
+      if (row < D) {
+        uint8_t* s_hi = kring;
+        uint8_t* s_lo = kring + D * D * 2;
+#pragma unroll
+        for (int u = 0; u < HD / 8; ++u) {
+          const int unit = pipe * (HD / 8) + u;
+          const float4 a = sv[2 * u], b = sv[2 * u + 1];
+          const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+          uint32_t hv[4], lv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t hh = pack_bf16x2(f[2 * e], f[2 * e + 1]);
+            hv[e] = hh;
+            lv[e] = pack_bf16x2(f[2 * e] - bf16_lo_to_f32(hh), f[2 * e + 1] - bf16_hi_to_f32(hh));
+          }
+          const uint32_t off = (unit / 8) * (D * 128) + row * 128 + (((unit % 8) ^ (row & 7)) * 16);
+          *reinterpret_cast<uint4*>(s_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
+          *reinterpret_cast<uint4*>(s_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+        }
+      }
 #pragma unroll
       for (int g = 0; g < HD / 32; ++g) {  // 32 elements -> 16 packed columns of hi and of lo
         uint32_t hi[16], lo[16];
@@ -537,8 +573,7 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
           const int unit = pipe * (HD / 8) + g * 4 + h;  // elements [8*unit, 8*unit + 8)
           const uint32_t off = (unit / 8) * (128 * 128) + row * 128 + (((unit % 8) ^ (row & 7)) * 16);
           const uint4 qv = *reinterpret_cast<const uint4*>(sQ + off);
-          const float4 za = __ldg(reinterpret_cast<const float4*>(zrow + unit * 8));
-          const float4 zb = __ldg(reinterpret_cast<const float4*>(zrow + unit * 8 + 4));
+          const float4 za = zv[(g * 4 + h) * 2], zb = zv[(g * 4 + h) * 2 + 1];
           const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
           const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
 #pragma unroll
@@ -556,30 +591,6 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
         // TMEM column c holds elements (2c, 2c+1) of the row: hi at [0, D/2), lo at [D/2, D)
         tmem_st16(lane_addr + C::kColPhi + pipe * (HD / 2) + g * 16, hi);
         tmem_st16(lane_addr + C::kColPhi + D / 2 + pipe * (HD / 2) + g * 16, lo);
-      }
-      // state rows: thread (k, pipe) converts S[bh][k][pipe*D/2 .. +D/2) into MN-major
-      // bf16 hi/lo tiles over the idle rings
-      if (row < D) {
-        const float* srow = p.S + (static_cast<size_t>(bh) * D + row) * D;
-        uint8_t* s_hi = kring;
-        uint8_t* s_lo = kring + D * D * 2;
-#pragma unroll 4
-        for (int u = 0; u < HD / 8; ++u) {
-          const int unit = pipe * (HD / 8) + u;
-          const float4 a = __ldg(reinterpret_cast<const float4*>(srow + unit * 8));
-          const float4 b = __ldg(reinterpret_cast<const float4*>(srow + unit * 8 + 4));
-          const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-          uint32_t hv[4], lv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t hh = pack_bf16x2(f[2 * e], f[2 * e + 1]);
-            hv[e] = hh;
-            lv[e] = pack_bf16x2(f[2 * e] - bf16_lo_to_f32(hh), f[2 * e + 1] - bf16_hi_to_f32(hh));
-          }
-          const uint32_t off = (unit / 8) * (D * 128) + row * 128 + (((unit % 8) ^ (row & 7)) * 16);
-          *reinterpret_cast<uint4*>(s_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-          *reinterpret_cast<uint4*>(s_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
-        }
       }
       fence_proxy_async_smem();
       tmem_wait_st();

@@ -145,23 +145,12 @@ bool rope_ok(const hf_rope* rope, int d, int Nq, int Nk, int block) {
   return rope->q_frame0 >= 0 && static_cast<long long>(rope->q_frame0) + ceil_div(Nq, rope->tokens_per_frame) <= W;
 }
 
-// Block pooling of Q (and K unless nKB == 0) by the persistent bulk-copy kernel; with a
-// rope (kRope), the means of the turned tokens.
+// Block pooling of Q (and K unless nKB == 0); with a rope (kRope), the means of the
+// turned tokens.
 template <int D, bool kParts, bool kRope = false>
 hf_status launch_pool(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk, int block, int nQB, int nKB,
                       float* Qp, float* Kp, int T, float* Kpart, cudaStream_t st, const hf_rope* rope = nullptr) {
   hf::PoolArgs a;
-  if (kRope) {
-    T = rope->tokens_per_frame;
-    a.q_frame0 = rope->q_frame0;
-    a.n_frames = ceil_div(Nk, T);
-    a.rope_cap = rope->cap;
-    a.rope_dt = rope->d_t;
-    a.rope_log2base = std::log2(rope->base);
-  } else {
-    a.q_frame0 = a.n_frames = a.rope_cap = a.rope_dt = 0;
-    a.rope_log2base = 0.f;
-  }
   a.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
   a.K = reinterpret_cast<const __nv_bfloat16*>(K);
   a.Nq = Nq;
@@ -169,27 +158,22 @@ hf_status launch_pool(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk
   a.block = block;
   a.nQB = nQB;
   a.nKB = nKB;
-  a.BH = BH;
   a.Qp = Qp;
   a.Kp = Kp;
   a.T = T;
   a.Kpart = Kpart;
-  a.stage_bytes = block * D * 2;
-  // up to 192 KB of stages (six 32 KB stages at d = block = 128), at least two
-  constexpr int kStageBudget = 192 * 1024;
-  a.stages = std::min(hf::kPoolMaxStages, std::max(2, kStageBudget / a.stage_bytes));
-  take_injection(1, &a.inject, &a.timeout_ns);
-  const size_t smem = static_cast<size_t>(a.stages) * a.stage_bytes;
-  if (cudaFuncSetAttribute(hf::pool_bulk_kernel<D, kParts, kRope>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem)) != cudaSuccess)
-    return HF_ERR_CUDA;
-  // CTAs per SM that fit beside one another (shared memory, threads), times the SMs
-  const size_t static_smem = 2 * sizeof(float) * hf::kPoolConsumers * 8 + 2 * 1024;
-  const long long per_sm = std::max<long long>(
-      1, std::min<long long>(2048 / hf::kPoolBulkThreads, (227 * 1024) / (smem + static_smem)));
-  const long long items = static_cast<long long>(BH) * (nQB + nKB);
-  const long long grid = std::min(items, per_sm * sm_count());
-  return launch_pdl(hf::pool_bulk_kernel<D, kParts, kRope>, grid, hf::kPoolBulkThreads, smem, st, a);
+  a.q_frame0 = a.n_frames = a.rope_cap = a.rope_dt = 0;
+  a.rope_log2base = 0.f;
+  if (kRope) {
+    a.T = rope->tokens_per_frame;
+    a.q_frame0 = rope->q_frame0;
+    a.n_frames = ceil_div(Nk, rope->tokens_per_frame);
+    a.rope_cap = rope->cap;
+    a.rope_dt = rope->d_t;
+    a.rope_log2base = std::log2(rope->base);
+  }
+  return launch_pdl(hf::pool_blocks_kernel<D, kParts, kRope>, static_cast<long long>(BH) * (nQB + nKB),
+                    hf::kPoolThreads, 0, st, a);
 }
 
 // ---------------------------------------------------------------- select
@@ -210,8 +194,11 @@ hf_status launch_score(const float* Qp, const float* Kp, int BH, int nQB, int nK
     if (cudaFuncSetAttribute(hf::score_select_staged_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return HF_ERR_CUDA;
+    int inject = 0;
+    unsigned long long timeout_ns = kDefaultTimeoutNs;
+    take_injection(1, &inject, &timeout_ns);
     return launch_pdl(hf::score_select_staged_kernel<D>, static_cast<long long>(BH) * ngroups, hf::kSelectThreads,
-                      smem, st, Qp, Kp, nQB, nKB, r, idx, scores, kDefaultTimeoutNs);
+                      smem, st, Qp, Kp, nQB, nKB, r, idx, scores, timeout_ns, inject);
   }
   // the opt-in covers static + dynamic shared memory above the 48 KB default; set on
   // every launch so that no size of nKB depends on it having been set before

@@ -11,16 +11,16 @@
 //
 // All on CUDA cores (the work is a streaming read of Q and K plus a tiny score matrix,
 // so tensor cores would not help):
-//   pool_bulk_kernel     persistent, one CTA per SM: fp32 mean of the valid rows of every
-//                        block of Q and K. HBM-bound: each block's rows (contiguous) come
-//                        in by one bulk copy into a ring of up to 8 stages, 6 in flight.
+//   pool_blocks_kernel   one CTA per (b,h,block) of Q or K: fp32 mean of the valid rows.
+//                        HBM-bound: reads Q and K once with 16-byte loads, 8 in flight
+//                        per thread.
 //   score_select_kernel  one CTA per (b,h, 4 query blocks): s_IJ = Qbar_I . Kbar_J, a
 //                        thread per key block; then one warp per query block finds the
 //                        r-th largest score by a bitwise search (per-lane counts, one warp
 //                        reduction per bit), takes every block above it and the lowest-J
 //                        blocks equal to it, and writes the r blocks in ascending J.
 //                        NaN scores are ranked as -inf, so exactly r blocks are written.
-// Two-stage selection: pool_bulk_kernel<d, true> also writes each key block's sums in
+// Two-stage selection: pool_blocks_kernel<d, true> also writes each key block's sums in
 // its first and next frame, pool_frames_kernel adds them into frame means, and
 // score_select2_kernel keeps frames first, then blocks within them (see there).
 // Pooled-key cache: kpool_push_kernel sums each granule of G new keys into a ring, and
@@ -58,24 +58,18 @@ __device__ __forceinline__ uint4 ld_stream_16(const void* p) {
 }
 
 constexpr uint32_t kKernSelect = 1;
-constexpr int kPoolConsumers = 256;                   // 8 consumer warps
-constexpr int kPoolBulkThreads = kPoolConsumers + 32;  // + the bulk-copy producer warp
-constexpr int kPoolMaxStages = 8;
 
 struct PoolArgs {
   const __nv_bfloat16* Q;
   const __nv_bfloat16* K;
-  int Nq, Nk, block, nQB, nKB, BH;
+  int Nq, Nk, block, nQB, nKB;
   float* Qp;     // [BH][nQB][D]
   float* Kp;     // [BH][nKB][D]
-  int T;         // frame length in tokens (kParts)
+  int T;         // frame length in tokens (kParts, kRope)
   float* Kpart;  // [BH][nKB][2][D] (kParts)
-  int stages, stage_bytes;
-  unsigned long long timeout_ns;
-  int inject;    // test only: the first copy is never issued, so a wait runs out
-  // temporal RoPE (kRope): frames of T tokens; Q's first token lies in window frame
-  // q_frame0, K's in frame 0; the window holds n_frames frames; index cap, rotated
-  // dimensions [0, rope_dt), log2 of the frequency base
+  // temporal RoPE (kRope): Q's first token lies in window frame q_frame0, K's in frame 0;
+  // the window holds n_frames frames; index cap; rotated dimensions [0, rope_dt); log2 of
+  // the frequency base
   int q_frame0, n_frames, rope_cap, rope_dt;
   float rope_log2base;
 };
@@ -92,173 +86,124 @@ __device__ __forceinline__ void rope_cs(int p, int i, int d_t, float log2base, f
   sincosf(static_cast<float>(p) * theta, &s, &c);
 }
 
-// Qp[bh][I][:] = mean of the Q rows of block I; Kp[bh][J][:] likewise for K.
+// Qp[bh][I][:] = mean of the Q rows of block I; Kp[bh][J][:] likewise for K. One CTA per
+// (b, h, block): streaming 16-byte loads, 8 per thread in flight, then a reduction of the
+// row phases through shared memory in a fixed order.
 // kParts (two-stage selection): also Kpart[bh][J][0|1][:] = the sums of the rows of key
 // block J that lie in its first frame (J*block / T) and in the next frame (zero when the
 // block does not reach it); frames are runs of T >= block tokens, so a block touches at
-// most two.
-// kRope: the rows are summed per frame (a block spans at most two, T >= block), each
-// frame's sum is turned by that frame's temporal RoPE index (pairs (2i, 2i+1) of the
-// dimensions below d_t), and the mean is taken of the turned sums: the mean of the
-// turned tokens, as the rotation is linear and one per frame.
-// Persistent: CTA c takes the blocks c, c + gridDim.x, ... of the list [b,h][Q blocks | K
-// blocks]. A block's rows are contiguous in memory, so one bulk copy (up to block x d x 2
-// bytes) brings it into a ring stage; the producer warp keeps up to `stages` copies in
-// flight while the 8 consumer warps sum the stage they hold: thread (row phase rp, unit c)
-// adds 8 columns of the rows rp, rp + kPhases, ... in fp32, and the kPhases partial sums
-// of a column are added in row-phase order through shared memory (deterministic).
+// most two. The block means are computed exactly as without kParts.
+// kRope: the rows of every block are summed per frame (a short second pass over the rows
+// of the next frame, just read and still in L2), each frame's sum is turned by that
+// frame's temporal RoPE index (pairs (2i, 2i+1) of the dimensions below d_t), and the mean
+// is taken of the turned sums: the mean of the turned tokens, as the rotation is linear
+// and one per frame.
 template <int D, bool kParts = false, bool kRope = false>
-__global__ void __launch_bounds__(kPoolBulkThreads, 1) pool_bulk_kernel(PoolArgs a) {
-  constexpr int kUnits = D / 8;                   // 16-byte units per row
-  constexpr int kPhases = kPoolConsumers / kUnits;  // row phases
-  constexpr bool kSplit = kParts || kRope;        // per-frame sums
-  extern __shared__ __align__(128) uint8_t pool_smem[];
-  __shared__ uint64_t full_bar[kPoolMaxStages], empty_bar[kPoolMaxStages];
-  __shared__ float red[kPhases][D];
-  __shared__ float red1[kSplit ? kPhases : 1][kSplit ? D : 1];
-  __shared__ float tot[kRope ? 2 : 1][kRope ? D : 1];
-  __shared__ int abort_sh;
-  volatile int* abort_flag = &abort_sh;
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int NS = a.stages;
-  const long long per_bh = static_cast<long long>(a.nQB) + a.nKB;
-  const long long total = static_cast<long long>(a.BH) * per_bh;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(&full_bar[s], 1);
-      mbar_init(&empty_bar[s], kPoolConsumers / 32);
-    }
-    abort_sh = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
+__global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(PoolArgs a) {
+  constexpr int kVec = 8;                       // bf16 per 16-byte load
+  constexpr int kTpr = D / kVec;                // threads per row
+  constexpr int kRows = kPoolThreads / kTpr;    // rows per pass
+  constexpr int kUnroll = 8;                    // loads in flight per thread
+  constexpr bool kSplit = kParts || kRope;
+  __shared__ float red[kRows * D];
+  __shared__ float red1[kSplit ? kRows * D : 1];
   griddep_wait();
   griddep_launch_dependents();
 
-  // rows [lo, hi) of item `item` and where they live
-  struct Item {
-    const __nv_bfloat16* src;
-    int lo, hi, bh, t;
-    bool key;
-  };
-  auto item_of = [&](long long item) {
-    Item it;
-    it.bh = static_cast<int>(item / per_bh);
-    int t = static_cast<int>(item % per_bh);
-    it.key = t >= a.nQB;
-    if (it.key) t -= a.nQB;
-    it.t = t;
-    const int N = it.key ? a.Nk : a.Nq;
-    it.lo = t * a.block;
-    it.hi = min(it.lo + a.block, N);
-    it.src = (it.key ? a.K : a.Q) + (static_cast<size_t>(it.bh) * N + it.lo) * D;
-    return it;
-  };
-
-  if (warp == kPoolConsumers / 32) {
-    // ---------------- bulk-copy producer ----------------
-    if (lane == 0) {
-      int issued = 0;
-      long long k = 0;
-      for (long long item = blockIdx.x; item < total; item += gridDim.x, ++k) {
-        const int s = static_cast<int>(k % NS), u = static_cast<int>(k / NS);
-        if (u >= 1 && !mbar_wait(&empty_bar[s], (u - 1) & 1, abort_flag, a.timeout_ns, (kKernSelect << 8) | 1))
-          break;
-        if (*abort_flag) break;
-        const Item it = item_of(item);
-        const uint32_t bytes = static_cast<uint32_t>(it.hi - it.lo) * D * 2;
-        issued = static_cast<int>(k) + 1;
-        if (a.inject && k == 0) continue;  // test only: stage 0 never fills
-        mbar_arrive_expect_tx(&full_bar[s], bytes);
-        bulk_load(pool_smem + static_cast<size_t>(s) * a.stage_bytes, it.src, bytes, &full_bar[s]);
-      }
-      // drain: every issued copy must have landed before the CTA may exit
-      for (int kk = max(0, issued - NS); kk < issued; ++kk) {
-        if (a.inject && kk == 0) continue;
-        mbar_wait_drain(&full_bar[kk % NS], (kk / NS) & 1, a.timeout_ns, (kKernSelect << 8) | 2);
-      }
-    }
+  const int per_bh = a.nQB + a.nKB;
+  const int bh = blockIdx.x / per_bh;
+  int t = blockIdx.x % per_bh;
+  const bool is_key_block = t >= a.nQB;
+  const __nv_bfloat16* X;
+  int N;
+  float* out;
+  if (t < a.nQB) {
+    X = a.Q + static_cast<size_t>(bh) * a.Nq * D;
+    N = a.Nq;
+    out = a.Qp + (static_cast<size_t>(bh) * a.nQB + t) * D;
   } else {
-    // ---------------- consumers ----------------
-    const int c = threadIdx.x % kUnits, rp = threadIdx.x / kUnits;
-    long long k = 0;
-    for (long long item = blockIdx.x; item < total; item += gridDim.x, ++k) {
-      const int s = static_cast<int>(k % NS);
-      const bool ok = mbar_wait(&full_bar[s], static_cast<uint32_t>(k / NS) & 1, abort_flag, a.timeout_ns,
-                                (kKernSelect << 8) | 3);
-      // every consumer has waited (or given up) and the previous item's shared-memory sums
-      // have been read; the decision to stop is the same for all of them
-      if (named_bar_any(1, kPoolConsumers, !ok || *abort_flag != 0)) break;
-      const Item it = item_of(item);
-      const int rows = it.hi - it.lo;
-      // first row of the next frame, relative to the block (kParts key blocks and every
-      // kRope block; else rows)
-      const int split = ((kParts && it.key) || kRope) ? min(rows, (it.lo / a.T + 1) * a.T - it.lo) : rows;
-      const uint8_t* stage = pool_smem + static_cast<size_t>(s) * a.stage_bytes;
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      float acc1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-      for (int r = rp; r < rows; r += kPhases) {
-        const uint4 v = *reinterpret_cast<const uint4*>(stage + static_cast<size_t>(r) * (D * 2) + c * 16);
-        if (!kSplit || r < split)
-          acc_bf16x8(acc, v);
-        else
-          acc_bf16x8(acc1, v);
-      }
-      // the stage may be refilled once every consumer warp has read it
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[s]);
+    t -= a.nQB;
+    X = a.K + static_cast<size_t>(bh) * a.Nk * D;
+    N = a.Nk;
+    out = a.Kp + (static_cast<size_t>(bh) * a.nKB + t) * D;
+  }
+  const int lo = t * a.block;
+  const int hi = min(lo + a.block, N);
+  const int c = threadIdx.x % kTpr;
+  const int rr = threadIdx.x / kTpr;
+  // first row of the next frame, if this block reaches it (key blocks with kParts, every
+  // block with kRope)
+  const bool split = (kParts && is_key_block) || kRope;
+  const int bnd = split ? min(hi, (lo / a.T + 1) * a.T) : hi;
+
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int base = lo + rr; base < hi; base += kRows * kUnroll) {
+    uint4 v[kUnroll];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) red[rp][c * 8 + e] = acc[e];
-      if constexpr (kSplit) {
+    for (int u = 0; u < kUnroll; ++u) {
+      const int row = base + u * kRows;
+      v[u] = row < hi ? ld_stream_16(X + static_cast<size_t>(row) * D + c * kVec) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) red1[rp][c * 8 + e] = acc1[e];
-      }
-      named_bar_sync(1, kPoolConsumers);
-      float s0 = 0.f, s1 = 0.f;
-      if (threadIdx.x < D) {
+    for (int u = 0; u < kUnroll; ++u) acc_bf16x8(acc, v[u]);
+  }
+  // the second-frame sum, only in blocks that reach the next frame (CTA-uniform): a short
+  // second pass over those rows, just read and still in L2
+  float acc1[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if constexpr (kSplit) {
+    if (bnd < hi) {
+      for (int row = lo + rr; row < hi; row += kRows)
+        if (row >= bnd) acc_bf16x8(acc1, ld_stream_16(X + static_cast<size_t>(row) * D + c * kVec));
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) red[rr * D + c * kVec + k] = acc[k];
+  if constexpr (kSplit) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) red1[rr * D + c * kVec + k] = acc1[k];
+  }
+  __syncthreads();
+  float s = 0.f, s1 = 0.f;
+  if (threadIdx.x < D) {
 #pragma unroll 8
-        for (int q = 0; q < kPhases; ++q) s0 += red[q][threadIdx.x];
-        if constexpr (kSplit) {
+    for (int q = 0; q < kRows; ++q) s += red[q * D + threadIdx.x];
+    if constexpr (kSplit) {
 #pragma unroll 8
-          for (int q = 0; q < kPhases; ++q) s1 += red1[q][threadIdx.x];
-        }
-      }
-      if constexpr (kRope) {
-        // turn the two frames' sums: pair (2i, 2i+1) needs its partner column
-        if (threadIdx.x < D) {
-          tot[0][threadIdx.x] = s0;
-          tot[1][threadIdx.x] = s1;
-        }
-        named_bar_sync(1, kPoolConsumers);
-        const int t = threadIdx.x;
-        if (t < a.rope_dt) {
-          const int i = t >> 1;
-          const int w0 = (it.key ? 0 : a.q_frame0) + it.lo / a.T;
-          float cs[2], sn[2];
-          rope_cs(rope_index(w0, a.n_frames, a.rope_cap), i, a.rope_dt, a.rope_log2base, cs[0], sn[0]);
-          rope_cs(rope_index(w0 + 1, a.n_frames, a.rope_cap), i, a.rope_dt, a.rope_log2base, cs[1], sn[1]);
-          float r[2];
+      for (int q = 0; q < kRows; ++q) s1 += red1[q * D + threadIdx.x];
+    }
+  }
+  if constexpr (kRope) {
+    // the two frames' sums, s - s1 and s1, turned by their indices; a pair (2i, 2i+1) needs
+    // its partner column, exchanged through shared memory
+    __syncthreads();
+    if (threadIdx.x < D) {
+      red[threadIdx.x] = s - s1;
+      red[D + threadIdx.x] = s1;
+    }
+    __syncthreads();
+    const int tc = threadIdx.x;
+    if (tc < a.rope_dt) {
+      const int i = tc >> 1;
+      const int w0 = (is_key_block ? 0 : a.q_frame0) + lo / a.T;
+      float r2[2];
 #pragma unroll
-          for (int f = 0; f < 2; ++f) {
-            const float x0 = tot[f][2 * i], x1 = tot[f][2 * i + 1];
-            r[f] = (t & 1) ? fmaf(x0, sn[f], x1 * cs[f]) : fmaf(x0, cs[f], -x1 * sn[f]);
-          }
-          s0 = r[0];
-          s1 = r[1];
-        }
+      for (int f = 0; f < 2; ++f) {
+        float cs, sn;
+        rope_cs(rope_index(w0 + f, a.n_frames, a.rope_cap), i, a.rope_dt, a.rope_log2base, cs, sn);
+        const float x0 = red[f * D + 2 * i], x1 = red[f * D + 2 * i + 1];
+        r2[f] = (tc & 1) ? fmaf(x0, sn, x1 * cs) : fmaf(x0, cs, -x1 * sn);
       }
-      if (threadIdx.x < D) {
-        float* out = it.key ? a.Kp + (static_cast<size_t>(it.bh) * a.nKB + it.t) * D
-                            : a.Qp + (static_cast<size_t>(it.bh) * a.nQB + it.t) * D;
-        out[threadIdx.x] = (s0 + s1) / static_cast<float>(rows);
-        if constexpr (kParts) {
-          if (it.key) {
-            float* pt = a.Kpart + ((static_cast<size_t>(it.bh) * a.nKB + it.t) * 2) * D;
-            pt[threadIdx.x] = s0;
-            pt[D + threadIdx.x] = s1;
-          }
-        }
+      s = r2[0] + r2[1];
+      s1 = r2[1];
+    }
+  }
+  if (threadIdx.x < D) {
+    out[threadIdx.x] = s / static_cast<float>(hi - lo);
+    if constexpr (kParts) {
+      if (is_key_block) {
+        float* pt = a.Kpart + ((static_cast<size_t>(bh) * a.nKB + t) * 2) * D;
+        pt[threadIdx.x] = s - s1;
+        pt[D + threadIdx.x] = s1;
       }
     }
   }
@@ -444,8 +389,9 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const floa
 // score_select_kernel with the head's pooled K rows staged in shared memory: they are
 // contiguous ([nKB][D] fp32), so a few bulk copies bring them in at once instead of each
 // thread waiting on its row's L2 loads (the plain kernel is bound by those latencies).
-// Used when nKB * D * 4 bytes fit (kStagedKBytes). Thread J reads its row starting at
-// 16-byte unit J % 32 (rotated), so the 32 lanes of a warp hit distinct banks.
+// Used when nKB * D * 4 bytes fit (kStagedKBytes). A warp takes a row at a time, lane l
+// the 16-byte units l, l + 32, ... (conflict-free), then a butterfly sum over the lanes:
+// every row's dot products add in the same order, so equal rows give equal scores.
 constexpr int kStagedKBytes = 192 * 1024;
 constexpr int kStageCopyBytes = 32 * 1024;
 
@@ -455,7 +401,8 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(con
                                                                              int nKB, int r,
                                                                              int32_t* __restrict__ idx_out,
                                                                              float* __restrict__ scores_out,
-                                                                             unsigned long long timeout_ns) {
+                                                                             unsigned long long timeout_ns,
+                                                                             int inject) {
   extern __shared__ __align__(128) float st_smem[];
   float* krows = st_smem;                                 // [nKB][D]
   float* s_sc = st_smem + static_cast<size_t>(nKB) * D;   // [kSelQB][nKB]
@@ -474,7 +421,7 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(con
   __syncthreads();
   griddep_wait();
   griddep_launch_dependents();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && !inject) {  // test only: with inject the rows never arrive
     const uint8_t* src = reinterpret_cast<const uint8_t*>(Kp + static_cast<size_t>(bh) * nKB * D);
     mbar_arrive_expect_tx(&kbar, kbytes);
     for (uint32_t o = 0; o < kbytes; o += kStageCopyBytes)
@@ -490,27 +437,35 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(con
   // abort flag but stays bounded)
   const bool landed = mbar_wait_drain(&kbar, 0, timeout_ns, (kKernSelect << 8) | 4);
   if (__syncthreads_or(!landed)) return;
-  constexpr int kU = D / 4;  // 16-byte units per row
-  for (int J = threadIdx.x; J < nKB; J += kSelectThreads) {
-    const float4* krow = reinterpret_cast<const float4*>(krows + static_cast<size_t>(J) * D);
+  constexpr int kU = D / 4 / 32;  // 16-byte units per lane: 1 (d = 128) or 0.5 (d = 64)
+  constexpr int kLanesPerRow = kU >= 1 ? 32 : 16;  // d = 64: a half-warp per row, two rows at once
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+  const int sub = lane / kLanesPerRow, l = lane % kLanesPerRow;
+  float4 qv[kSelQB];
+#pragma unroll
+  for (int g = 0; g < kSelQB; ++g) qv[g] = *reinterpret_cast<const float4*>(&q_sh[g][4 * l]);
+#pragma unroll 4
+  for (int J0 = warp * kRowsPerWarp; J0 < nKB; J0 += (kSelectThreads / 32) * kRowsPerWarp) {
+    const int J = J0 + sub;
     float acc[kSelQB];
+    const float4 kv = J < nKB ? *reinterpret_cast<const float4*>(krows + static_cast<size_t>(J) * D + 4 * l)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int g = 0; g < kSelQB; ++g) acc[g] = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < kU; ++k) {
-      const int u = (k + J) % kU;
-      const float4 kv = krow[u];
-#pragma unroll
-      for (int g = 0; g < kSelQB; ++g) {
-        const float4 qv = *reinterpret_cast<const float4*>(&q_sh[g][4 * u]);
-        acc[g] = fmaf(qv.x, kv.x, acc[g]);
-        acc[g] = fmaf(qv.y, kv.y, acc[g]);
-        acc[g] = fmaf(qv.z, kv.z, acc[g]);
-        acc[g] = fmaf(qv.w, kv.w, acc[g]);
-      }
+    for (int g = 0; g < kSelQB; ++g) {
+      float x = qv[g].x * kv.x;
+      x = fmaf(qv[g].y, kv.y, x);
+      x = fmaf(qv[g].z, kv.z, x);
+      acc[g] = fmaf(qv[g].w, kv.w, x);
     }
 #pragma unroll
-    for (int g = 0; g < kSelQB; ++g) s_sc[g * nKB + J] = acc[g];
+    for (int off = kLanesPerRow / 2; off >= 1; off >>= 1) {
+#pragma unroll
+      for (int g = 0; g < kSelQB; ++g) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
+    }
+    if (l == 0 && J < nKB) {
+#pragma unroll
+      for (int g = 0; g < kSelQB; ++g) s_sc[g * nKB + J] = acc[g];
+    }
   }
   __syncthreads();
   if (warp < G) {

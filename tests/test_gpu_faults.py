@@ -67,7 +67,8 @@ def test_attention_timeout_is_reported_and_recoverable(name, H):
 
 
 def test_select_timeout_is_reported_and_recoverable():
-    """The block pooling's consumers give up on a ring stage that never fills."""
+    """The scoring kernel gives up on the pooled key rows that never arrive in shared
+    memory (their bulk copies are not issued)."""
     wl = WORKLOADS["832x480"]
     x = draw_step_inputs(wl, n_evicted=1)
     Q, K = x["Q"][:, :2].contiguous().to(DEV), x["K"][:, :2].contiguous().to(DEV)
@@ -78,7 +79,7 @@ def test_select_timeout_is_reported_and_recoverable():
     hf.hf_select_blocks(Q, K, wl.block, wl.r)
     rc, word = hf.hf_query_status()
     assert rc == hf.HF_ERR_DEVICE_TIMEOUT, (rc, hex(word))
-    assert (word >> 8) & 0xFF == 1, hex(word)  # reported by the selection's pooling kernel
+    assert (word >> 8) & 0xFF == 1, hex(word)  # reported by the selection's scoring kernel
     idx = hf.hf_select_blocks(Q, K, wl.block, wl.r)
     torch.cuda.synchronize()
     assert hf.hf_query_status()[0] == hf.HF_OK
