@@ -18,18 +18,15 @@
 // (the element index contiguous): A = V^T is the V tile as TMA wrote it, B is the
 // converted K tile.
 //   warp 0      TMA producer: the V and K tiles [64 tokens][d] of a tile into one ring
-//               stage laid out [V | K], 64-column chunks of 8 KB (the A chunks 8 KB apart).
-//               The ring is as deep as shared memory allows (5 stages at d = 128): the HBM
-//               latency under load (~2500 cycles) plus a tile's conversion and MMAs must fit
-//               in the ring's turnaround.
+//               stage laid out [V | K, then phi_hi over K | phi_lo], 64-column chunks of
+//               8 KB each, so the A chunks and the 2d/64 B chunks are 8 KB apart.
 //   warp 1      TMEM owner + MMA issuer: per tile 4 MMAs (K = 16 tokens each) into one of
 //               two TMEM accumulators of 2d columns. It waits only for the converters'
-//               "B written" barrier of the tile's B buffer (they arrive after the stage
-//               barrier, so the V tile has landed too), then commits the stage back to the
-//               producer and the B buffer back to the converters.
+//               "B written" barrier of the stage (they arrive after the stage barrier, so
+//               the V tile has landed too) and commits the stage back to the producer.
 //   warps 2..17 converters (four warps per SM sub-partition: the conversion is issue- and
-//               MUFU-bound): phi(k) in fp32, split hi = bf16(phi), lo = bf16(phi - hi),
-//               written into one of kNB B buffers laid out [hi | lo] (chunks 8 KB apart); z
+//               MUFU-bound): phi(k) in fp32, split hi = bf16(phi), lo = bf16(phi - hi);
+//               hi overwrites the K chunk in place and lo goes to the stage's lo chunk; z
 //               is accumulated in fp32 registers. They also drain the accumulator: the
 //               tensor core's fp32 accumulation truncates, so a long chain of MMAs into one
 //               TMEM accumulator drifts (relative error grows with the chain length, ~2e-5
@@ -65,22 +62,21 @@ struct AbsorbCfg {
   static constexpr int kChunks = D / 64;                  // 64-element column chunks of a tile
   static constexpr int kChunkBytes = kAbsTok * 128;       // one chunk: 64 rows x 128 B
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes;      // V | K
+  static constexpr int kStageBytes = 3 * kTileBytes;      // V | K (-> phi_hi) | phi_lo
   static constexpr int kVOff = 0;
   static constexpr int kKOff = kTileBytes;
-  static constexpr int kBBytes = 2 * kTileBytes;          // a B buffer: phi_hi | phi_lo
-  static constexpr int kNB = D == 128 ? 2 : 3;            // B buffers
+  static constexpr int kLoOff = 2 * kTileBytes;
   static constexpr int kN = 2 * D;                        // MMA N: phi_hi and phi_lo columns
   static constexpr uint32_t kAccCols = kN;                // TMEM columns per accumulator
   static constexpr uint32_t kTmemCols = 2 * kAccCols;     // two accumulators (256 or 512)
   static constexpr int kZredBytes = kConvThreads * 8 * 4;  // end-of-kernel z reduction (over the ring)
   static constexpr int kBudget = 232448 - 1024 - 1024;    // shared memory per CTA - alignment - static
-  static constexpr int kStagesFit = (kBudget - kNB * kBBytes) / kStageBytes;
+  static constexpr int kStagesFit = kBudget / kStageBytes;
   static constexpr int kStages = kStagesFit < kAbsMaxStages ? kStagesFit : kAbsMaxStages;
   static_assert(kStages >= 2, "ring too small");
   static constexpr int kRingBytes = kStages * kStageBytes;
   static_assert(kZredBytes <= kRingBytes, "z reduction must fit over the ring");
-  static constexpr int kDynSmem = 1024 + kRingBytes + kNB * kBBytes;
+  static constexpr int kDynSmem = 1024 + kRingBytes;
   static constexpr int kColsPerWarp = D / 4;              // k columns per converter warp in the drain
   static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation is a power of two");
 };
@@ -103,11 +99,9 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
   using C = AbsorbCfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  constexpr int NB = C::kNB;
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* bbuf = ring + C::kRingBytes;  // NB buffers [phi_hi | phi_lo]
 
-  __shared__ uint64_t full_bar[NS], empty_bar[NS], bfull_bar[NB], bempty_bar[NB];
+  __shared__ uint64_t full_bar[NS], empty_bar[NS], bfull_bar[NS];
   __shared__ uint64_t dfull_bar[2], dempty_bar[2], drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -124,10 +118,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-    }
-    for (int b = 0; b < NB; ++b) {
-      mbar_init(&bfull_bar[b], kConvThreads / 32);
-      mbar_init(&bempty_bar[b], 1);
+      mbar_init(&bfull_bar[s], kConvThreads / 32);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&dfull_bar[b], 1);
@@ -187,26 +178,24 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       // B = [phi_hi | phi_lo] (N = 2d, MN-major); chunks 8 KB apart, 8-row groups 1 KB apart
       constexpr uint32_t idesc = idesc_bf16_f32(128, C::kN, true, true);
       const uint64_t adesc0 = sdesc_sw128(smem_u32(ring + C::kVOff), C::kChunkBytes, 1024);
-      const uint64_t bdesc0 = sdesc_sw128(smem_u32(bbuf), C::kChunkBytes, 1024);
+      const uint64_t bdesc0 = sdesc_sw128(smem_u32(ring + C::kKOff), C::kChunkBytes, 1024);
       bool ok = true;
       for (int i = 0; i < ntiles && ok; ++i) {
-        const int s = i % NS, nb = i % NB;
+        const int s = i % NS;
         const int g = i / kAbsGroup, b = g & 1;
         const bool first = (i % kAbsGroup) == 0;
         const bool last = (i % kAbsGroup) == kAbsGroup - 1 || i == ntiles - 1;
-        ok = mbar_wait(&bfull_bar[nb], (i / NB) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 4);
+        ok = mbar_wait(&bfull_bar[s], (i / NS) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 4);
         if (ok && first && g >= 2)
           ok = mbar_wait(&dempty_bar[b], ((g >> 1) - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 9);
         if (!ok) break;
         tc_fence_after();
         const uint64_t so = static_cast<uint64_t>((s * C::kStageBytes) >> 4);
-        const uint64_t bo = static_cast<uint64_t>((nb * C::kBBytes) >> 4);
         const uint32_t d_tmem = tmem_d + b * C::kAccCols;
 #pragma unroll
         for (int ks = 0; ks < kAbsTok / 16; ++ks)  // 16 tokens = 16 rows of 128 B = 2048 B
-          umma_ss(d_tmem, adesc0 + so + ks * 128, bdesc0 + bo + ks * 128, idesc, (!first || ks > 0) ? 1u : 0u);
+          umma_ss(d_tmem, adesc0 + so + ks * 128, bdesc0 + so + ks * 128, idesc, (!first || ks > 0) ? 1u : 0u);
         umma_commit(&empty_bar[s]);
-        umma_commit(&bempty_bar[nb]);
         if (last) umma_commit(&dfull_bar[b]);
       }
       umma_commit(&drain_bar);
@@ -280,15 +269,11 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       lo = pack_bf16x2(r0, r1);
     };
     for (int i = 0; i < ntiles && ok; ++i) {
-      const int s = i % NS, nb = i % NB;
-      bool w = mbar_wait(&full_bar[s], (i / NS) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 6);
-      // B buffer nb is free once the MMAs of tile i - NB are done
-      if (w && i >= NB)
-        w = mbar_wait(&bempty_bar[nb], ((i / NB) - 1) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 7);
-      ok = __all_sync(0xffffffffu, w);
+      const int s = i % NS;
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&full_bar[s], (i / NS) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 6));
       if (!ok) break;
       uint8_t* stage = ring + s * C::kStageBytes;
-      uint8_t* bb = bbuf + nb * C::kBBytes;
       const int valid = min(kAbsTok, p.n_tokens - (tile0 + i) * kAbsTok);
 #pragma unroll
       for (int k = 0; k < kRowsPerThread; ++k) {
@@ -306,13 +291,13 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) hi[e] = lo[e] = 0u;
         }
-        *reinterpret_cast<uint4*>(bb + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(bb + C::kTileBytes + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        *reinterpret_cast<uint4*>(stage + C::kKOff + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(stage + C::kLoOff + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       // every lane's stores are made visible to the tensor core, then one arrival per warp
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bfull_bar[nb]);
+      if (lane == 0) mbar_arrive(&bfull_bar[s]);
       // once group g is fully converted, drain group g - 1 (one group of lag keeps the
       // tensor core busy on the other accumulator)
       const int g = i / kAbsGroup;

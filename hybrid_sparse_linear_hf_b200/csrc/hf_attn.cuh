@@ -397,10 +397,13 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
         const int s = v % NSK;
         ok = mbar_wait(&kfull_bar[s], (v / NSK) & 1, abort_flag, p.timeout_ns, (kKernAttn << 8) | 21);
         if (!ok) break;
+        // rows at index 0 (frames at least cap frames old) are left as they are: the
+        // rotation is the identity there
         const bool valid = rt < BLK && (J < p.nKB - 1 || rt < p.last_len);
-        if (valid) {
+        const int pidx = index_of((J * BLK + rt) / p.rope_T);
+        if (valid && pidx > 0) {
           uint8_t* ktile = kring + s * C::kKVTileBytes;  // chunk 0: BLK rows x 128 B
-          turn_row(ktile, ktile, rt, index_of((J * BLK + rt) / p.rope_T), nunits);
+          turn_row(ktile, ktile, rt, pidx, nunits);
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -558,13 +561,19 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const uint32_t hh = pack_bf16x2(f[2 * e], f[2 * e + 1]);
             hv[e] = hh;
-            lv[e] = pack_bf16x2(f[2 * e] - bf16_lo_to_f32(hh), f[2 * e + 1] - bf16_hi_to_f32(hh));
+            float r0, r1;
+            f32x2_split(ffma2(f32x2(bf16_lo_to_f32(hh), bf16_hi_to_f32(hh)), f32x2(-1.0f, -1.0f),
+                              f32x2(f[2 * e], f[2 * e + 1])), r0, r1);
+            lv[e] = pack_bf16x2(r0, r1);
           }
           const uint32_t off = (unit / 8) * (D * 128) + row * 128 + (((unit % 8) ^ (row & 7)) * 16);
           *reinterpret_cast<uint4*>(s_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
           *reinterpret_cast<uint4*>(s_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
         }
       }
+      // phi(x) = max(x, 0) + 2^(min(x, 0) log2 e) (branch-free elu + 1) on packed fp32 pairs;
+      // phi . z accumulated as a pair, summed at the end
+      uint64_t dacc2 = 0ull;
 #pragma unroll
       for (int g = 0; g < HD / 32; ++g) {  // 32 elements -> 16 packed columns of hi and of lo
         uint32_t hi[16], lo[16];
@@ -575,22 +584,34 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
           const uint4 qv = *reinterpret_cast<const uint4*>(sQ + off);
           const float4 za = zv[(g * 4 + h) * 2], zb = zv[(g * 4 + h) * 2 + 1];
           const uint32_t w[4] = {qv.x, qv.y, qv.z, qv.w};
-          const float zz[8] = {za.x, za.y, za.z, za.w, zb.x, zb.y, zb.z, zb.w};
+          const uint64_t zz[4] = {f32x2(za.x, za.y), f32x2(za.z, za.w), f32x2(zb.x, zb.y), f32x2(zb.z, zb.w)};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float x0 = bf16_lo_to_f32(w[e]), x1 = bf16_hi_to_f32(w[e]);
-            const float p0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
-            const float p1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
-            dacc = fmaf(p0, zz[2 * e], dacc);
-            dacc = fmaf(p1, zz[2 * e + 1], dacc);
+            const float n0 = fminf(x0, 0.f), n1 = fminf(x1, 0.f);
+            float l0, l1;
+            f32x2_split(ffma2(f32x2(n0, n1), f32x2(1.4426950408889634f, 1.4426950408889634f), 0ull), l0, l1);
+            // (x - min(x, 0)) + 2^l
+            const uint64_t p2 = fadd2(ffma2(f32x2(n0, n1), f32x2(-1.0f, -1.0f), f32x2(x0, x1)),
+                                      f32x2(ex2_approx(l0), ex2_approx(l1)));
+            dacc2 = ffma2(p2, zz[e], dacc2);
+            float p0, p1;
+            f32x2_split(p2, p0, p1);
             const uint32_t hh = pack_bf16x2(p0, p1);
             hi[h * 4 + e] = hh;
-            lo[h * 4 + e] = pack_bf16x2(p0 - bf16_lo_to_f32(hh), p1 - bf16_hi_to_f32(hh));
+            float r0, r1;
+            f32x2_split(ffma2(f32x2(bf16_lo_to_f32(hh), bf16_hi_to_f32(hh)), f32x2(-1.0f, -1.0f), p2), r0, r1);
+            lo[h * 4 + e] = pack_bf16x2(r0, r1);
           }
         }
         // TMEM column c holds elements (2c, 2c+1) of the row: hi at [0, D/2), lo at [D/2, D)
         tmem_st16(lane_addr + C::kColPhi + pipe * (HD / 2) + g * 16, hi);
         tmem_st16(lane_addr + C::kColPhi + D / 2 + pipe * (HD / 2) + g * 16, lo);
+      }
+      {
+        float d0, d1;
+        f32x2_split(dacc2, d0, d1);
+        dacc = d0 + d1;
       }
       fence_proxy_async_smem();
       tmem_wait_st();

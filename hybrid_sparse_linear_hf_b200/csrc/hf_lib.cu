@@ -122,18 +122,6 @@ hf_status launch_pdl(void (*kernel)(KArgs...), long long grid, int block, size_t
   return launch_status();
 }
 
-// Streaming multiprocessors of the current device (cached per device).
-int sm_count() {
-  static int cached[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
-  if (dev < 64 && cached[dev] > 0) return cached[dev];
-  int n = 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
-  if (dev < 64) cached[dev] = n;
-  return n;
-}
-
 // Checks of an hf_rope for a step with Nq queries, a window of Nk keys and blocks of
 // `block` tokens: the chunk must lie inside the window's frames.
 bool rope_ok(const hf_rope* rope, int d, int Nq, int Nk, int block) {
