@@ -19,10 +19,7 @@
 // converted K tile.
 //   warp 0      TMA producer: the V and K tiles [64 tokens][d] of a tile into one ring
 //               stage laid out [V | K, then phi_hi over K | phi_lo], 64-column chunks of
-//               8 KB each, so the A chunks and the 2d/64 B chunks are 8 KB apart. Each
-//               load also prefetches into L2 the tile one ring length ahead: the four
-//               stages alone cannot cover the HBM latency under load (~3000 cycles) plus a
-//               tile's conversion and MMAs, while a load served from L2 can be.
+//               8 KB each, so the A chunks and the 2d/64 B chunks are 8 KB apart.
 //   warp 1      TMEM owner + MMA issuer: per tile 4 MMAs (K = 16 tokens each) into one of
 //               two TMEM accumulators of 2d columns. It waits only for the converters'
 //               "B written" barrier of the stage (they arrive after the stage barrier, so
@@ -157,16 +154,6 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
           break;
         if (*abort_flag) break;
         if (p.inject && i == 0) continue;  // test only: tile 0 never arrives
-        // the tile one ring length ahead goes into L2 now, so that its load (issued when
-        // this stage comes round again) is served from L2 instead of waiting on HBM
-        if (i + NS < ntiles) {
-          const int prow = (tile0 + i + NS) * kAbsTok;
-#pragma unroll
-          for (int c = 0; c < C::kChunks; ++c) {
-            tma_prefetch_l2_3d(&mapK, c * 64, prow, bh);
-            tma_prefetch_l2_3d(&mapV, c * 64, prow, bh);
-          }
-        }
         uint8_t* st = ring + s * C::kStageBytes;
         mbar_arrive_expect_tx(&full_bar[s], 2 * C::kTileBytes);
         const int row = (tile0 + i) * kAbsTok;
