@@ -358,8 +358,9 @@ __global__ void __launch_bounds__(256) reduce_state_kernel(float* __restrict__ S
     float4* s4 = reinterpret_cast<float4*>(S + static_cast<size_t>(bh) * D * D) + e4;
     float4 acc = *s4;
     const float4* p4 = reinterpret_cast<const float4*>(part_S + static_cast<size_t>(bh) * nsplit * D * D) + e4;
-    // all loads of a batch in flight, then the adds in slice order
-    constexpr int kBatch = 8;
+    // all loads of a batch in flight (one L2 round trip for up to 16 slices), then the
+    // adds in slice order
+    constexpr int kBatch = 16;
     for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
       float4 v[kBatch];
 #pragma unroll
