@@ -133,11 +133,10 @@ bool rope_ok(const hf_rope* rope, int d, int Nq, int Nk, int block) {
   return rope->q_frame0 >= 0 && static_cast<long long>(rope->q_frame0) + ceil_div(Nq, rope->tokens_per_frame) <= W;
 }
 
-// Block pooling of Q (and K unless nKB == 0); with a rope (kRope), the means of the
-// turned tokens.
-template <int D, bool kParts, bool kRope = false>
-hf_status launch_pool(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk, int block, int nQB, int nKB,
-                      float* Qp, float* Kp, int T, float* Kpart, cudaStream_t st, const hf_rope* rope = nullptr) {
+// Arguments of the block pooling of Q (and K unless nKB == 0); with a rope, the means of
+// the turned tokens.
+hf::PoolArgs pool_args(const hf_bf16* Q, const hf_bf16* K, int Nq, int Nk, int block, int nQB, int nKB, float* Qp,
+                       float* Kp, int T, float* Kpart, const hf_rope* rope) {
   hf::PoolArgs a;
   a.Q = reinterpret_cast<const __nv_bfloat16*>(Q);
   a.K = reinterpret_cast<const __nv_bfloat16*>(K);
@@ -152,7 +151,8 @@ hf_status launch_pool(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk
   a.Kpart = Kpart;
   a.q_frame0 = a.n_frames = a.rope_cap = a.rope_dt = 0;
   a.rope_log2base = 0.f;
-  if (kRope) {
+  a.k_transposed = 0;
+  if (rope) {
     a.T = rope->tokens_per_frame;
     a.q_frame0 = rope->q_frame0;
     a.n_frames = ceil_div(Nk, rope->tokens_per_frame);
@@ -160,6 +160,17 @@ hf_status launch_pool(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk
     a.rope_dt = rope->d_t;
     a.rope_log2base = std::log2(rope->base);
   }
+  return a;
+}
+
+// Block pooling (the means of Q's and K's blocks into the workspace; the key means
+// transposed with `k_transposed`).
+template <int D, bool kParts, bool kRope = false>
+hf_status launch_pool(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int Nk, int block, int nQB, int nKB,
+                      float* Qp, float* Kp, int T, float* Kpart, cudaStream_t st, const hf_rope* rope = nullptr,
+                      bool k_transposed = false) {
+  hf::PoolArgs a = pool_args(Q, K, Nq, Nk, block, nQB, nKB, Qp, Kp, T, Kpart, kRope ? rope : nullptr);
+  a.k_transposed = k_transposed ? 1 : 0;
   return launch_pdl(hf::pool_blocks_kernel<D, kParts, kRope>, static_cast<long long>(BH) * (nQB + nKB),
                     hf::kPoolThreads, 0, st, a);
 }
@@ -171,13 +182,25 @@ size_t select_ws_bytes(int B, int H, int Nq, int Nk, int d, int block) {
          align256(static_cast<size_t>(bh) * ceil_div(Nk, block) * d * 4);
 }
 
-// scores and top-r from the pooled rows in the workspace
+// The selection's grids fit the launch limit (a pooling CTA per block).
+bool select_grid_ok(long long BH, int Nq, int nKB, int block) {
+  return BH * (ceil_div(Nq, block) + nKB) <= 0x7fffffffLL;
+}
+
+// Whether the scores come from the staged kernel (the pooling then writes the key means
+// transposed).
+template <int D>
+bool staged_scores(int nKB) {
+  return static_cast<long long>(nKB) * D * 4 <= hf::kStagedKBytes;
+}
+
+// Scores and top-r from the pooled means in the workspace: the staged kernel on
+// transposed key means (`transposed`), else the plain kernel on row-major means.
 template <int D>
 hf_status launch_score(const float* Qp, const float* Kp, int BH, int nQB, int nKB, int r, int32_t* idx,
-                       float* scores, cudaStream_t st) {
-  const long long ngroups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
-  if (static_cast<long long>(nKB) * D * 4 <= hf::kStagedKBytes) {
-    // the head's pooled K rows staged in shared memory by bulk copies
+                       float* scores, cudaStream_t st, bool transposed) {
+  const long long groups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
+  if (transposed) {
     const size_t smem = static_cast<size_t>(nKB) * D * 4 + static_cast<size_t>(nKB) * hf::kSelQB * sizeof(float);
     if (cudaFuncSetAttribute(hf::score_select_staged_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
@@ -185,8 +208,8 @@ hf_status launch_score(const float* Qp, const float* Kp, int BH, int nQB, int nK
     int inject = 0;
     unsigned long long timeout_ns = kDefaultTimeoutNs;
     take_injection(1, &inject, &timeout_ns);
-    return launch_pdl(hf::score_select_staged_kernel<D>, static_cast<long long>(BH) * ngroups, hf::kSelectThreads,
-                      smem, st, Qp, Kp, nQB, nKB, r, idx, scores, timeout_ns, inject);
+    return launch_pdl(hf::score_select_staged_kernel<D>, BH * groups, hf::kSelectThreads, smem, st, Qp, Kp, nQB, nKB,
+                      r, idx, scores, timeout_ns, inject);
   }
   // the opt-in covers static + dynamic shared memory above the 48 KB default; set on
   // every launch so that no size of nKB depends on it having been set before
@@ -194,9 +217,8 @@ hf_status launch_score(const float* Qp, const float* Kp, int BH, int nQB, int nK
   if (cudaFuncSetAttribute(hf::score_select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return HF_ERR_CUDA;
-  const long long groups = (nQB + hf::kSelQB - 1) / hf::kSelQB;
-  return launch_pdl(hf::score_select_kernel<D>, static_cast<long long>(BH) * groups, hf::kSelectThreads, smem, st, Qp,
-                    Kp, nQB, nKB, r, idx, scores);
+  return launch_pdl(hf::score_select_kernel<D>, BH * groups, hf::kSelectThreads, smem, st, Qp, Kp, nQB, nKB, r, idx,
+                    scores);
 }
 
 template <int D>
@@ -205,11 +227,13 @@ hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int 
   const int nQB = ceil_div(Nq, block), nKB = ceil_div(Nk, block);
   float* Qp = static_cast<float*>(ws);
   float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(BH) * nQB * D * 4));
+  const bool staged = staged_scores<D>(nKB);
   const hf_status rc = rope ? launch_pool<D, false, true>(Q, K, BH, Nq, Nk, block, nQB, nKB, Qp, Kp, 0, nullptr, st,
-                                                            rope)
-                            : launch_pool<D, false>(Q, K, BH, Nq, Nk, block, nQB, nKB, Qp, Kp, 0, nullptr, st);
+                                                            rope, staged)
+                            : launch_pool<D, false>(Q, K, BH, Nq, Nk, block, nQB, nKB, Qp, Kp, 0, nullptr, st,
+                                                    nullptr, staged);
   if (rc != HF_OK) return HF_ERR_CUDA;
-  return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st);
+  return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st, staged);
 }
 
 // selection over the pooled-key cache: Q pooled as above (no key blocks), key blocks from
@@ -227,7 +251,7 @@ hf_status launch_select_cached(const hf_bf16* Q, const hf_kpool* kp, int BH, int
   if (launch_pdl(hf::kpool_blocks_kernel<D>, ctas, hf::kPoolThreads, 0, st, static_cast<const float*>(kp->sums),
                  kp->capacity, kp->head, kp->n_gran, kp->granule, block, nKB, BH, Kp) != HF_OK)
     return HF_ERR_CUDA;
-  return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st);
+  return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st, /*transposed=*/false);
 }
 
 // ---------------------------------------------------------------- two-stage select
@@ -568,7 +592,7 @@ HF_API hf_status hf_select_blocks(const hf_bf16* Q, const hf_bf16* K, int B, int
   if (!ws || ws_bytes < select_ws_bytes(B, H, Nq, Nk, d, block)) return HF_ERR_WORKSPACE;
   if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
   const long long BH = static_cast<long long>(B) * H;
-  if (BH * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  if (!select_grid_ok(BH, Nq, nKB, block)) return HF_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_select<128>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s)
                   : launch_select<64>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s);
@@ -590,7 +614,7 @@ HF_API hf_status hf_select_blocks_rope(const hf_bf16* Q, const hf_bf16* K, int B
   if (!ws || ws_bytes < select_ws_bytes(B, H, Nq, Nk, d, block)) return HF_ERR_WORKSPACE;
   if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
   const long long BH = static_cast<long long>(B) * H;
-  if (BH * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  if (!select_grid_ok(BH, Nq, nKB, block)) return HF_ERR_UNSUPPORTED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128
              ? launch_select<128>(Q, K, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s, rope)
@@ -819,7 +843,7 @@ HF_API hf_status hf_select_blocks_noalloc(const hf_bf16* Q, const hf_bf16* K, in
   if (!Q || !K || !idx_out) return HF_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(idx_out) || (scores_out && !aligned16(scores_out)))
     return HF_ERR_ALIGNMENT;
-  if (static_cast<long long>(B) * H * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  if (!select_grid_ok(static_cast<long long>(B) * H, Nq, nKB, block)) return HF_ERR_UNSUPPORTED;
   const size_t need = select_ws_bytes(B, H, Nq, Nk, d, block);
   if (need > HF_SELECT_NOALLOC_SCRATCH_BYTES) return HF_ERR_WORKSPACE;
   void* scratch = nullptr;

@@ -14,6 +14,9 @@
 //   pool_blocks_kernel   one CTA per (b,h,block) of Q or K: fp32 mean of the valid rows.
 //                        HBM-bound: reads Q and K once with 16-byte loads, 8 in flight
 //                        per thread.
+//   score_select_staged_kernel  the same with a head's pooled K means (written
+//                        transposed by the pooling) staged in shared memory by bulk
+//                        copies, when they fit (see there).
 //   score_select_kernel  one CTA per (b,h, 4 query blocks): s_IJ = Qbar_I . Kbar_J, a
 //                        thread per key block; then one warp per query block finds the
 //                        r-th largest score by a bitwise search (per-lane counts, one warp
@@ -72,6 +75,8 @@ struct PoolArgs {
   // the frequency base
   int q_frame0, n_frames, rope_cap, rope_dt;
   float rope_log2base;
+  // 1: the key means go to Kp transposed, [BH][D][nKB] (for score_select_staged_kernel)
+  int k_transposed;
 };
 
 // Temporal RoPE index of window frame w: the newest frame (n_frames - 1) at cap, every
@@ -98,31 +103,33 @@ __device__ __forceinline__ void rope_cs(int p, int i, int d_t, float log2base, f
 // frame's temporal RoPE index (pairs (2i, 2i+1) of the dimensions below d_t), and the mean
 // is taken of the turned sums: the mean of the turned tokens, as the rotation is linear
 // and one per frame.
-template <int D, bool kParts = false, bool kRope = false>
-__global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(PoolArgs a) {
-  constexpr int kVec = 8;                       // bf16 per 16-byte load
-  constexpr int kTpr = D / kVec;                // threads per row
-  constexpr int kRows = kPoolThreads / kTpr;    // rows per pass
+template <int D>
+struct PoolShape {
+  static constexpr int kVec = 8;                     // bf16 per 16-byte load
+  static constexpr int kTpr = D / kVec;              // threads per row
+  static constexpr int kRows = kPoolThreads / kTpr;  // rows per pass
+  static constexpr int kRedFloats = kRows * D;       // one row-phase reduction buffer
+};
+
+// The mean of block t of Q (is_key_block false) or K of head bh, computed by the whole
+// CTA (kPoolThreads threads) with the reduction buffers red and red1 (kRedFloats each;
+// red1 used with kParts or kRope), written by threads 0..D-1.
+template <int D, bool kParts, bool kRope>
+__device__ __forceinline__ void pool_block(const PoolArgs& a, int bh, int t, bool is_key_block, float* red,
+                                           float* red1) {
+  constexpr int kVec = PoolShape<D>::kVec;
+  constexpr int kTpr = PoolShape<D>::kTpr;
+  constexpr int kRows = PoolShape<D>::kRows;
   constexpr int kUnroll = 8;                    // loads in flight per thread
   constexpr bool kSplit = kParts || kRope;
-  __shared__ float red[kRows * D];
-  __shared__ float red1[kSplit ? kRows * D : 1];
-  griddep_wait();
-  griddep_launch_dependents();
-
-  const int per_bh = a.nQB + a.nKB;
-  const int bh = blockIdx.x / per_bh;
-  int t = blockIdx.x % per_bh;
-  const bool is_key_block = t >= a.nQB;
   const __nv_bfloat16* X;
   int N;
   float* out;
-  if (t < a.nQB) {
+  if (!is_key_block) {
     X = a.Q + static_cast<size_t>(bh) * a.Nq * D;
     N = a.Nq;
     out = a.Qp + (static_cast<size_t>(bh) * a.nQB + t) * D;
   } else {
-    t -= a.nQB;
     X = a.K + static_cast<size_t>(bh) * a.Nk * D;
     N = a.Nk;
     out = a.Kp + (static_cast<size_t>(bh) * a.nKB + t) * D;
@@ -198,7 +205,11 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(PoolArgs a) {
     }
   }
   if (threadIdx.x < D) {
-    out[threadIdx.x] = s / static_cast<float>(hi - lo);
+    const float mean = s / static_cast<float>(hi - lo);
+    if (is_key_block && a.k_transposed)
+      a.Kp[(static_cast<size_t>(bh) * D + threadIdx.x) * a.nKB + t] = mean;
+    else
+      out[threadIdx.x] = mean;
     if constexpr (kParts) {
       if (is_key_block) {
         float* pt = a.Kpart + ((static_cast<size_t>(bh) * a.nKB + t) * 2) * D;
@@ -207,6 +218,22 @@ __global__ void __launch_bounds__(kPoolThreads) pool_blocks_kernel(PoolArgs a) {
       }
     }
   }
+}
+
+// Eight CTAs per SM (2048 threads): the loads in flight fit in 32 registers a thread.
+template <int D, bool kParts = false, bool kRope = false>
+__global__ void __launch_bounds__(kPoolThreads, kRope ? 6 : 8) pool_blocks_kernel(PoolArgs a) {
+  __shared__ float red[PoolShape<D>::kRedFloats];
+  __shared__ float red1[(kParts || kRope) ? PoolShape<D>::kRedFloats : 1];
+  griddep_wait();
+  griddep_launch_dependents();
+  const int per_bh = a.nQB + a.nKB;
+  const int bh = blockIdx.x / per_bh;
+  const int t = blockIdx.x % per_bh;
+  if (t < a.nQB)
+    pool_block<D, kParts, kRope>(a, bh, t, false, red, red1);
+  else
+    pool_block<D, kParts, kRope>(a, bh, t - a.nQB, true, red, red1);
 }
 
 // Kf[bh][w][:] = mean of the key rows of frame w (rows [w*T, min((w+1)*T, Nk))), summed
@@ -386,26 +413,28 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_kernel(const floa
   }
 }
 
-// score_select_kernel with the head's pooled K rows staged in shared memory: they are
-// contiguous ([nKB][D] fp32), so a few bulk copies bring them in at once instead of each
-// thread waiting on its row's L2 loads (the plain kernel is bound by those latencies).
-// Used when nKB * D * 4 bytes fit (kStagedKBytes). A warp takes a row at a time, lane l
-// the 16-byte units l, l + 32, ... (conflict-free), then a butterfly sum over the lanes:
-// every row's dot products add in the same order, so equal rows give equal scores.
+// ------------------------------------------------------------ staged scoring
+// score_select_staged_kernel: score_select_kernel with the head's pooled key means staged
+// in shared memory, used when they fit (kStagedKBytes). The pooling kernel writes them
+// transposed for it ([BH][D][nKB] fp32, contiguous per head), so that a few 32 KB bulk
+// copies bring a head's means in at once, and thread J then reads column J: consecutive
+// lanes read consecutive words (no bank conflicts) and every key block's dot products add
+// over k in the same order, so equal key blocks give equal scores (the tie rule needs
+// exact equality).
 constexpr int kStagedKBytes = 192 * 1024;
 constexpr int kStageCopyBytes = 32 * 1024;
 
 template <int D>
 __global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(const float* __restrict__ Qp,
-                                                                             const float* __restrict__ Kp, int nQB,
+                                                                             const float* __restrict__ KpT, int nQB,
                                                                              int nKB, int r,
                                                                              int32_t* __restrict__ idx_out,
                                                                              float* __restrict__ scores_out,
                                                                              unsigned long long timeout_ns,
                                                                              int inject) {
   extern __shared__ __align__(128) float st_smem[];
-  float* krows = st_smem;                                 // [nKB][D]
-  float* s_sc = st_smem + static_cast<size_t>(nKB) * D;   // [kSelQB][nKB]
+  float* kcols = st_smem;                                // [D][nKB]
+  float* s_sc = st_smem + static_cast<size_t>(nKB) * D;  // [kSelQB][nKB]
   __shared__ __align__(16) float q_sh[kSelQB][D];
   __shared__ uint64_t kbar;
   const int groups = (nQB + kSelQB - 1) / kSelQB;
@@ -413,7 +442,7 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(con
   const int I0 = (blockIdx.x % groups) * kSelQB;
   const int G = min(kSelQB, nQB - I0);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const uint32_t kbytes = static_cast<uint32_t>(nKB) * D * 4;
+  const uint32_t kbytes = static_cast<uint32_t>(nKB) * D * 4;  // a multiple of 16
   if (threadIdx.x == 0) {
     mbar_init(&kbar, 1);
     fence_mbar_init();
@@ -421,11 +450,11 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(con
   __syncthreads();
   griddep_wait();
   griddep_launch_dependents();
-  if (threadIdx.x == 0 && !inject) {  // test only: with inject the rows never arrive
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(Kp + static_cast<size_t>(bh) * nKB * D);
+  if (threadIdx.x == 0 && !inject) {  // test only: with inject the means never arrive
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(KpT + static_cast<size_t>(bh) * nKB * D);
     mbar_arrive_expect_tx(&kbar, kbytes);
     for (uint32_t o = 0; o < kbytes; o += kStageCopyBytes)
-      bulk_load(reinterpret_cast<uint8_t*>(krows) + o, src + o, min(kStageCopyBytes, static_cast<int>(kbytes - o)),
+      bulk_load(reinterpret_cast<uint8_t*>(kcols) + o, src + o, min(kStageCopyBytes, static_cast<int>(kbytes - o)),
                 &kbar);
   }
   for (int i = threadIdx.x; i < kSelQB * D; i += kSelectThreads) {
@@ -433,39 +462,30 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(con
     q_sh[g][i % D] = Qp[(static_cast<size_t>(bh) * nQB + I0 + min(g, G - 1)) * D + i % D];
   }
   __syncthreads();
-  // every thread waits for the rows (the copies cannot be abandoned: the wait ignores the
-  // abort flag but stays bounded)
+  // every thread waits for the means (the wait ignores the abort flag: issued copies must
+  // land before the CTA exits)
   const bool landed = mbar_wait_drain(&kbar, 0, timeout_ns, (kKernSelect << 8) | 4);
   if (__syncthreads_or(!landed)) return;
-  constexpr int kU = D / 4 / 32;  // 16-byte units per lane: 1 (d = 128) or 0.5 (d = 64)
-  constexpr int kLanesPerRow = kU >= 1 ? 32 : 16;  // d = 64: a half-warp per row, two rows at once
-  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
-  const int sub = lane / kLanesPerRow, l = lane % kLanesPerRow;
-  float4 qv[kSelQB];
-#pragma unroll
-  for (int g = 0; g < kSelQB; ++g) qv[g] = *reinterpret_cast<const float4*>(&q_sh[g][4 * l]);
-#pragma unroll 4
-  for (int J0 = warp * kRowsPerWarp; J0 < nKB; J0 += (kSelectThreads / 32) * kRowsPerWarp) {
-    const int J = J0 + sub;
+  for (int J = threadIdx.x; J < nKB; J += kSelectThreads) {
     float acc[kSelQB];
-    const float4 kv = J < nKB ? *reinterpret_cast<const float4*>(krows + static_cast<size_t>(J) * D + 4 * l)
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int g = 0; g < kSelQB; ++g) {
-      float x = qv[g].x * kv.x;
-      x = fmaf(qv[g].y, kv.y, x);
-      x = fmaf(qv[g].z, kv.z, x);
-      acc[g] = fmaf(qv[g].w, kv.w, x);
+    for (int g = 0; g < kSelQB; ++g) acc[g] = 0.f;
+#pragma unroll 4
+    for (int k0 = 0; k0 < D; k0 += 4) {
+      float kv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) kv[u] = kcols[static_cast<size_t>(k0 + u) * nKB + J];
+#pragma unroll
+      for (int g = 0; g < kSelQB; ++g) {
+        const float4 qv = *reinterpret_cast<const float4*>(&q_sh[g][k0]);
+        acc[g] = fmaf(qv.x, kv[0], acc[g]);
+        acc[g] = fmaf(qv.y, kv[1], acc[g]);
+        acc[g] = fmaf(qv.z, kv[2], acc[g]);
+        acc[g] = fmaf(qv.w, kv[3], acc[g]);
+      }
     }
 #pragma unroll
-    for (int off = kLanesPerRow / 2; off >= 1; off >>= 1) {
-#pragma unroll
-      for (int g = 0; g < kSelQB; ++g) acc[g] += __shfl_xor_sync(0xffffffffu, acc[g], off);
-    }
-    if (l == 0 && J < nKB) {
-#pragma unroll
-      for (int g = 0; g < kSelQB; ++g) s_sc[g * nKB + J] = acc[g];
-    }
+    for (int g = 0; g < kSelQB; ++g) s_sc[g * nKB + J] = acc[g];
   }
   __syncthreads();
   if (warp < G) {

@@ -80,6 +80,7 @@ def test_select_timeout_is_reported_and_recoverable():
     rc, word = hf.hf_query_status()
     assert rc == hf.HF_ERR_DEVICE_TIMEOUT, (rc, hex(word))
     assert (word >> 8) & 0xFF == 1, hex(word)  # reported by the selection's scoring kernel
+    assert word & 0xFF == 4, hex(word)  # at the wait for the staged key rows
     idx = hf.hf_select_blocks(Q, K, wl.block, wl.r)
     torch.cuda.synchronize()
     assert hf.hf_query_status()[0] == hf.HF_OK
