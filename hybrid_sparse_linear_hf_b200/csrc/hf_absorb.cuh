@@ -252,14 +252,16 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       return true;
     };
     // phi(x) = x + 1 (x > 0) or exp(x) (x <= 0) for the two bf16 halves of w, in fp32,
-    // written branch-free as max(x, 0) + 2^(min(x, 0) log2 e) (the exponential is 1 for
-    // x > 0); hi = bf16(phi), lo = bf16(phi - hi); z accumulates phi.
+    // written branch-free as (x - m) + 2^(m log2 e) with m = min(x, 0) (the exponential
+    // is 1 for x > 0; x - m, exact, is one packed FMA instead of two max operations on
+    // the busier ALU pipe); hi = bf16(phi), lo = bf16(phi - hi); z accumulates phi.
     auto convert_pair = [&](uint32_t w, uint64_t& z2, uint32_t& hi, uint32_t& lo) {
       const float x0 = bf16_lo_to_f32(w), x1 = bf16_hi_to_f32(w);
+      const uint64_t m2 = f32x2(fminf(x0, 0.f), fminf(x1, 0.f));
       float l0, l1;
-      f32x2_split(ffma2(f32x2(fminf(x0, 0.f), fminf(x1, 0.f)),
-                        f32x2(1.4426950408889634f, 1.4426950408889634f), 0ull), l0, l1);
-      const uint64_t pp = fadd2(f32x2(fmaxf(x0, 0.f), fmaxf(x1, 0.f)), f32x2(ex2_approx(l0), ex2_approx(l1)));
+      f32x2_split(ffma2(m2, f32x2(1.4426950408889634f, 1.4426950408889634f), 0ull), l0, l1);
+      const uint64_t xm = ffma2(m2, f32x2(-1.0f, -1.0f), f32x2(x0, x1));
+      const uint64_t pp = fadd2(xm, f32x2(ex2_approx(l0), ex2_approx(l1)));
       float p0, p1;
       f32x2_split(pp, p0, p1);
       z2 = fadd2(z2, pp);
