@@ -70,6 +70,22 @@ def test_select_matches_oracle(B, H, Nq, Nk, d, block, r):
     _check_status()
 
 
+@pytest.mark.parametrize("d,nKB", [(128, 384), (128, 385), (64, 768), (64, 769)])
+def test_select_staged_boundary(d, nKB):
+    """Either side of the largest key-block count whose means (nKB x d fp32) are staged in
+    shared memory (192 KB): the staged scoring kernel on transposed means, and the plain one
+    on row-major means, against the oracle; the last key block is partial."""
+    block, r = 128, 40
+    Nk = (nKB - 1) * block + 57
+    Q = _gen(11, 1, 2, 3 * block + 5, d, w=0.5)
+    K = _gen(12, 1, 2, Nk, d, w=0.5)
+    idx, scores = _run_select(Q, K, block, r)
+    oidx, osc = oracle.select_blocks(f64(Q), f64(K), block, r)
+    assert np.abs(scores - osc).max() <= SCORE_ABS
+    assert_masks_match(idx, oidx, osc, r)
+    _check_status()
+
+
 def test_select_ties_lower_index():
     """Duplicated key blocks produce exactly equal pooled scores: the lower index wins."""
     d, block = 64, 32
