@@ -10,7 +10,7 @@ input generator.
 from ._binding import (  # noqa: F401
     HF_ERR_ALIGNMENT, HF_ERR_CUDA, HF_ERR_DEVICE_BAD_INDEX, HF_ERR_DEVICE_TIMEOUT, HF_ERR_INVALID_ARG,
     HF_ERR_UNSUPPORTED, HF_ERR_WORKSPACE, HF_OK, HF_SELECT_NOALLOC_SCRATCH_BYTES, HF_WS_ABSORB, HF_WS_ATTN,
-    HF_WS_SELECT, HF_WS_SELECT_TWO_STAGE, LIB_PATH, HfError, HfKpool, HfState, hf_absorb_evicted, hf_debug_exp2,
+    HF_WS_SELECT, HF_WS_SELECT_TWO_STAGE, LIB_PATH, HfError, HfKpool, HfState, hf_absorb_evicted,
     hf_debug_inject_timeout, hf_hybrid_attn_fwd, hf_hybrid_attn_fwd_absorb, hf_hybrid_attn_fwd_rope,
     hf_keep_schedule, hf_rope, hf_select_blocks_rope, HfRopeC, hf_launch_count, hf_kpool_init, hf_kpool_push,
     hf_query_status, hf_select_blocks, hf_select_blocks_cached, hf_select_blocks_noalloc,

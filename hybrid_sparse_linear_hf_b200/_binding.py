@@ -103,8 +103,6 @@ _SIGNATURES = {
     "hf_version": (ctypes.c_char_p, []),
     "hf_launch_count": (ctypes.c_ulonglong, []),
     "hf_debug_inject_timeout": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_ulonglong]),
-    "hf_debug_exp2": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
-                                     ctypes.c_void_p]),
 }
 
 
@@ -479,15 +477,6 @@ def hf_query_status(stream=None) -> tuple[int, int]:
     detail = ctypes.c_uint32(0)
     rc = lib().hf_query_status(_stream(stream), ctypes.byref(detail))
     return int(rc), int(detail.value)
-
-
-def hf_debug_exp2(x: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
-    """Test only: (FMA-pipe exp2, MUFU exp2) of the softmax for x <= 8 (fp32, device)."""
-    yp = torch.empty_like(x)
-    ym = torch.empty_like(x)
-    _check(lib().hf_debug_exp2(_dev(x, torch.float32, "x"), yp.data_ptr(), ym.data_ptr(), x.numel(),
-                               _stream(stream)), "hf_debug_exp2")
-    return yp, ym
 
 
 def hf_debug_inject_timeout(kernel_id: int, count: int, timeout_ns: int) -> None:

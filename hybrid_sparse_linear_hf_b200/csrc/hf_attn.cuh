@@ -37,7 +37,7 @@
 // Softmax: online in the log2 domain with a lazily raised running max (O is rescaled only
 // when a block maximum exceeds the running max by more than 8, i.e. a factor 256; exact
 // since numerator and denominator share the max); the O rescale is warp-uniform because
-// TMEM access is warp-collective; 3 exp2 pairs in 8 run on the FMA pipe, the rest on MUFU.
+// TMEM access is warp-collective; exp2 runs on MUFU (ex2.approx).
 // Temporal RoPE variant (kRope, hf_hybrid_attn_fwd_rope; Hybrid Forcing, German technical
 // summary section 2 C): a fourth warpgroup (warps 12..15, one thread per row) builds a
 // table of (cos, sin) for every index 0..cap and pair, turns the Q tile's first 64
@@ -67,7 +67,6 @@ static_assert(2 * 128 * kRegsSupportRope + 256 * kRegsRows <= kAttnThreadsRope *
               "setmaxnreg split exceeds the launch");
 constexpr int kSmemLimit = 232448;  // max shared memory per CTA on sm_100
 constexpr int kAttnStaticSmem = 1024;  // upper bound of the kernel's static shared memory
-constexpr int kPolyOf8 = 3;         // pairs (of every 8) that take exp2 on the FMA pipe
 constexpr int kMaxSlots = 6;
 
 template <int D, int BLK, bool kRope = false>
@@ -470,10 +469,11 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
         l_run *= alpha;
         m_run = mx;
       }
-      // p = 2^(s * scale * log2 e - m) as packed fp32 pairs, 32 columns at a time; each
-      // chunk of P goes to TMEM over the first columns of S_p at once (S is in registers).
-      // kPolyOf8 pairs of every 8 run exp2 on the FMA pipe, the others on MUFU, so neither
-      // unit alone sets the pace.
+      // p = 2^(s * scale * log2 e - m): scale and shift as packed fp32 pairs, exp2 on MUFU,
+      // 32 columns at a time; each chunk of P goes to TMEM over the first columns of S_p at
+      // once (S is in registers). The softmax warps share their SM sub-partitions with the
+      // MMA-issuing thread, so fewer instructions per element matter more than spreading
+      // exp2 over the FMA pipe (a polynomial exp2 costs ~6x the issue slots of MUFU's).
       {
         const uint64_t sl2 = f32x2(p.scale_log2, p.scale_log2);
         const uint64_t nm2 = f32x2(-m_run, -m_run);
@@ -483,16 +483,9 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int c = c0; c < c0 + 32; c += 2) {
-            const uint64_t x2 = ffma2(f32x2(srow[c], srow[c + 1]), sl2, nm2);
-            float p0, p1;
-            if (((c / 2) & 7) >= 8 - kPolyOf8) {
-              exp2_poly_x2(x2, p0, p1);
-            } else {
-              float x0, x1;
-              f32x2_split(x2, x0, x1);
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
+            float x0, x1;
+            f32x2_split(ffma2(f32x2(srow[c], srow[c + 1]), sl2, nm2), x0, x1);
+            const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
             lacc[(c / 2) & 3] = fadd2(lacc[(c / 2) & 3], f32x2(p0, p1));
             pk[(c - c0) / 2] = pack_bf16x2(p0, p1);
           }

@@ -382,21 +382,6 @@ hf_status launch_attn(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int 
                     kRope ? hf::kAttnThreadsRope : hf::kAttnThreads, C::kDynSmem, stream, mq, mk, mv, mo, p);
 }
 
-__global__ void debug_exp2_kernel(const float* __restrict__ x, float* __restrict__ yp, float* __restrict__ ym,
-                                  int n) {
-  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-  if (i >= n) return;
-  const float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.0f;
-  float p0, p1;
-  hf::exp2_poly_x2(hf::f32x2(a, b), p0, p1);
-  yp[i] = p0;
-  ym[i] = hf::ex2_approx(a);
-  if (i + 1 < n) {
-    yp[i + 1] = p1;
-    ym[i + 1] = hf::ex2_approx(b);
-  }
-}
-
 }  // namespace
 
 // ---------------------------------------------------------------- select without a caller workspace
@@ -809,15 +794,6 @@ HF_API hf_status hf_query_status(void* stream, uint32_t* detail_out) {
   if (cudaMemcpyToSymbol(hf::g_hf_error_word, &zero, sizeof(zero)) != cudaSuccess) return HF_ERR_CUDA;
   if (detail_out) *detail_out = word;
   return (word >> 16) == 0x7200u ? HF_ERR_DEVICE_BAD_INDEX : HF_ERR_DEVICE_TIMEOUT;
-}
-
-HF_API hf_status hf_debug_exp2(const float* x, float* y_poly, float* y_mufu, int n, void* stream) {
-  if (n < 0) return HF_ERR_INVALID_ARG;
-  if (n == 0) return HF_OK;
-  if (!x || !y_poly || !y_mufu) return HF_ERR_INVALID_ARG;
-  const int pairs = (n + 1) / 2;
-  debug_exp2_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_mufu, n);
-  return launch_status();
 }
 
 HF_API hf_status hf_debug_inject_timeout(int kernel_id, int count, unsigned long long timeout_ns) {

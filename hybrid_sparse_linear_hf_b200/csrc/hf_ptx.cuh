@@ -373,31 +373,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of arguments x <= 8 on the FMA/ALU pipes instead of MUFU.
-// Cody-Waite range reduction: j = round(x) via the 1.5*2^23 rounding constant, f = x - j
-// in [-1/2, 1/2]; 2^f by a degree-3 minimax polynomial (relative error 7.5e-5, fitted by
-// csrc/exp2_poly_fit.py); 2^j is added to the exponent bits. Arguments below -125 are
-// clamped (the result is then ~1e-38 instead of 0, negligible next to the row sum).
-__device__ __forceinline__ void exp2_poly_x2(uint64_t x2, float& p0, float& p1) {
-  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-  constexpr int kRoundBits = 0x4B400000;
-  float x0, x1;
-  f32x2_split(x2, x0, x1);
-  const uint64_t xc = f32x2(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t t = fadd2(xc, f32x2(kRound, kRound));
-  const uint64_t j = fadd2(t, f32x2(-kRound, -kRound));
-  const uint64_t f = ffma2(j, f32x2(-1.0f, -1.0f), xc);
-  uint64_t q = ffma2(f, f32x2(0.0551716685295105f, 0.0551716685295105f),
-                     f32x2(0.2426111251115799f, 0.2426111251115799f));
-  q = ffma2(q, f, f32x2(0.6932609677314758f, 0.6932609677314758f));
-  q = ffma2(q, f, f32x2(0.9999280571937561f, 0.9999280571937561f));
-  float q0, q1, t0, t1;
-  f32x2_split(q, q0, q1);
-  f32x2_split(t, t0, t1);
-  p0 = __int_as_float(__float_as_int(q0) + ((__float_as_int(t0) - kRoundBits) << 23));
-  p1 = __int_as_float(__float_as_int(q1) + ((__float_as_int(t1) - kRoundBits) << 23));
-}
-
 // ----------------------------------------------------------------------------
 // descriptors
 // ----------------------------------------------------------------------------

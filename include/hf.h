@@ -371,13 +371,6 @@ HF_API unsigned long long hf_launch_count(void);
  * those launches is also `timeout_ns`. Host-side setting of this library instance. */
 HF_API hf_status hf_debug_inject_timeout(int kernel_id, int count, unsigned long long timeout_ns);
 
-/* TEST ONLY. Evaluates, for each x[i] <= 8, the two exp2 paths of the attention softmax:
- * y_poly[i] = the FMA-pipe path (Cody-Waite reduction + degree-3 minimax polynomial,
- * relative error <= 1e-4 for x >= -125, a result below 1e-37 for smaller x) and
- * y_mufu[i] = the hardware ex2.approx path. x, y_poly, y_mufu: device fp32 [n].
- * Errors: HF_ERR_INVALID_ARG (n < 0, NULL with n > 0), HF_ERR_CUDA. */
-HF_API hf_status hf_debug_exp2(const float* x, float* y_poly, float* y_mufu, int n, void* stream);
-
 #ifdef __cplusplus
 }
 #endif
