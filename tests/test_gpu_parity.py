@@ -431,19 +431,22 @@ def test_1280x720_state_build_sampled_heads():
 
 
 @pytest.mark.parametrize("tail", [128, 50])
-def test_attention_online_rescale_mixed_rows(tail):
-    """Even query rows meet much larger scores in later blocks (their running max must be
-    raised twice, rescaling O) while odd rows do not: every warp mixes both cases. With a
-    tail of 50 the block that raises the max the most is the partial last one, whose
-    padding columns must stay masked when a raised max has its exponentials taken again."""
+@pytest.mark.parametrize("k2,k3", [(40.0, 70.0), (26.0, 30.0)])
+def test_attention_online_rescale_mixed_rows(tail, k2, k3):
+    """Even query rows meet much larger scores in later blocks while odd rows do not:
+    every warp mixes both cases. With (40, 70) the even rows' logits jump by ~15 and ~27
+    (log2 units) over the first blocks' (their running max must be raised twice, O
+    rescaled); with (26, 30) by ~10 and ~11.5, large p values the running max may keep.
+    With a tail of 50 the block that raises the max the most is the partial last one,
+    whose padding columns must stay masked when its exponentials are taken again."""
     d, block, Nq, Nk = 128, 128, 256, 3 * 128 + tail
     g = torch.Generator().manual_seed(77)
     Q = torch.randn(1, 2, Nq, d, generator=g) * 0.3
     Q[:, :, 0::2, 0] = 3.0
     K = torch.randn(1, 2, Nk, d, generator=g) * 0.3
     V = torch.randn(1, 2, Nk, d, generator=g)
-    K[:, :, 2 * block:3 * block, 0] = 40.0   # block 2: scores ~120 for even rows
-    K[:, :, 3 * block:4 * block, 0] = 70.0   # block 3: scores ~210 for even rows
+    K[:, :, 2 * block:3 * block, 0] = k2   # block 2: scores ~3 k2 for even rows
+    K[:, :, 3 * block:4 * block, 0] = k3   # block 3: scores ~3 k3 for even rows
     Q, K, V = Q.bfloat16(), K.bfloat16(), V.bfloat16()
     S = torch.empty(1, 2, d, d, device=DEV)
     z = torch.empty(1, 2, d, device=DEV)
