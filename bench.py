@@ -576,6 +576,9 @@ def run_gpu(args, wl) -> None:
     t_push = timer.run(lambda: hf.hf_kpool_push(kp, K_in, n_evict=wl.Nq), n=n_leg, warm=3)
     t_selc = timer.run(lambda: hf.hf_select_blocks_cached(Q, kp, wl.block, wl.r, idx_out=idx_c, ws=ws_sel),
                        n=n_leg, warm=3)
+    # the same step as one call: the push's sums computed in the Q pooling launch
+    t_selcp = timer.run(lambda: hf.hf_select_blocks_cached_push(Q, kp, K_in, wl.block, wl.r, n_evict=wl.Nq,
+                                                                idx_out=idx_c, ws=ws_sel), n=n_leg, warm=3)
     del kp_sums, K_in
     check_status(hf, "the pooled-key cache leg")
     # ---- sparsity sweep: the attention alone at other keep ratios (same inputs and state)
@@ -665,9 +668,12 @@ def run_gpu(args, wl) -> None:
                                            "hbm_frac": select_bytes(wl) / statistics.mean(t_sel2) / 1e9
                                            / peaks["hbm_gbs"]},
             "hf_select_blocks_cached": {"us": statistics.mean(t_selc) * 1e6,
-                                        "push_us": statistics.mean(t_push) * 1e6, "granule": KPOOL_GRANULE,
+                                        "push_us": statistics.mean(t_push) * 1e6,
+                                        "push_and_select_one_call_us": statistics.mean(t_selcp) * 1e6,
+                                        "granule": KPOOL_GRANULE,
                                         "note": "per step: hf_kpool_push of the 4680 new keys (and eviction "
-                                                "of the oldest 4680), then the selection from the granule sums"},
+                                                "of the oldest 4680), then the selection from the granule sums; "
+                                                "hf_select_blocks_cached_push does both in one call"},
             "hf_absorb_evicted_step": {"us": abs_mean * 1e6, "tokens": wl.Ne_step,
                                        "bytes": absorb_bytes(wl, wl.Ne_step),
                                        "gbs": absorb_bytes(wl, wl.Ne_step) / abs_mean / 1e9},

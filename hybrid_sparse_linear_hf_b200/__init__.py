@@ -13,6 +13,6 @@ from ._binding import (  # noqa: F401
     HF_WS_SELECT, HF_WS_SELECT_TWO_STAGE, LIB_PATH, HfError, HfKpool, HfState, hf_absorb_evicted,
     hf_debug_inject_timeout, hf_hybrid_attn_fwd, hf_hybrid_attn_fwd_absorb, hf_hybrid_attn_fwd_rope,
     hf_keep_schedule, hf_rope, hf_select_blocks_rope, HfRopeC, hf_launch_count, hf_kpool_init, hf_kpool_push,
-    hf_query_status, hf_select_blocks, hf_select_blocks_cached, hf_select_blocks_noalloc,
+    hf_query_status, hf_select_blocks, hf_select_blocks_cached, hf_select_blocks_cached_push, hf_select_blocks_noalloc,
     hf_select_blocks_two_stage, hf_state_init, hf_status_string, hf_version, hf_workspace_size, lib,
 )

@@ -93,6 +93,9 @@ _SIGNATURES = {
     "hf_kpool_init": (ctypes.c_int, [ctypes.POINTER(HfKpoolC)] + [ctypes.c_int] * 5 + [ctypes.c_void_p]),
     "hf_kpool_push": (ctypes.c_int, [ctypes.POINTER(HfKpoolC), ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
                                      ctypes.c_void_p]),
+    "hf_select_blocks_cached_push": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(HfKpoolC), ctypes.c_void_p]
+                                     + [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                             ctypes.c_size_t, ctypes.c_void_p]),
     "hf_select_blocks_cached": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(HfKpoolC)] + [ctypes.c_int] * 3 +
                                 [ctypes.c_void_p] * 3 + [ctypes.c_size_t, ctypes.c_void_p]),
     "hf_keep_schedule": (ctypes.c_int, [ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_double,
@@ -337,6 +340,36 @@ def hf_select_blocks_cached(Q: torch.Tensor, kp: HfKpool, block: int, r: int, id
                                          if scores_out is not None else None,
                                          ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
            "hf_select_blocks_cached")
+    return idx_out
+
+
+def hf_select_blocks_cached_push(Q: torch.Tensor, kp: HfKpool, K_new, block: int, r: int, n_evict: int = 0,
+                                 idx_out=None, scores_out=None, ws=None, stream=None) -> torch.Tensor:
+    """hf_kpool_push(kp, K_new, n_evict) then hf_select_blocks_cached(Q, kp, ...), in one call."""
+    if not isinstance(Q, torch.Tensor) or Q.dim() != 4:
+        raise ValueError("Q must be a 4-D tensor [B,H,Nq,d]")
+    B, H, Nq, d = Q.shape
+    if (B, H, d) != (kp.c.B, kp.c.H, kp.c.d):
+        raise ValueError(f"Q's (B, H, d) = {(B, H, d)} must match the cache's {(kp.c.B, kp.c.H, kp.c.d)}")
+    n = 0 if K_new is None else int(K_new.shape[2])
+    if K_new is not None and (K_new.dim() != 4 or tuple(K_new.shape[:2]) != (B, H) or K_new.shape[3] != d):
+        raise ValueError("K_new must be [B,H,n,d] matching the cache")
+    G = int(kp.c.granule)
+    Nk = (int(kp.c.n_gran) - int(n_evict) // G + n // G) * G  # the window after the push
+    nQB, nKB = -(-Nq // block), -(-max(Nk, 1) // block)
+    _shape(idx_out, (B, H, nQB, r), "idx_out")
+    _shape(scores_out, (B, H, nQB, nKB), "scores_out")
+    if idx_out is None:
+        idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
+    nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, max(Nk, 1), d, block, 1)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    _check(lib().hf_select_blocks_cached_push(_dev(Q, torch.bfloat16, "Q"), ctypes.byref(kp.c),
+                                              _dev(K_new, torch.bfloat16, "K_new") if n > 0 else None, n,
+                                              int(n_evict), Nq, block, r, _dev(idx_out, torch.int32, "idx_out"),
+                                              _dev(scores_out, torch.float32, "scores_out")
+                                              if scores_out is not None else None,
+                                              ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
+           "hf_select_blocks_cached_push")
     return idx_out
 
 

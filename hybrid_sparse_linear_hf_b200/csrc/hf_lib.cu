@@ -238,20 +238,36 @@ hf_status launch_select(const hf_bf16* Q, const hf_bf16* K, int BH, int Nq, int 
 
 // selection over the pooled-key cache: Q pooled as above (no key blocks), key blocks from
 // the granule sums
+// (with `push`: the push's granule sums are computed by the CTAs after the Q pooling's,
+// in the same launch; kp is then the window after the push)
 template <int D>
 hf_status launch_select_cached(const hf_bf16* Q, const hf_kpool* kp, int BH, int Nq, int Nk, int block, int r,
-                               int32_t* idx, float* scores, void* ws, cudaStream_t st) {
+                               int32_t* idx, float* scores, void* ws, cudaStream_t st,
+                               const hf::PushArgs* push = nullptr, long long push_ctas = 0) {
   const int nQB = ceil_div(Nq, block), nKB = ceil_div(Nk, block);
   float* Qp = static_cast<float*>(ws);
   float* Kp = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(BH) * nQB * D * 4));
-  if (launch_pool<D, false>(Q, nullptr, BH, Nq, 0, block, nQB, 0, Qp, Kp, 0, nullptr, st) != HF_OK)
+  if (push) {
+    const hf::PoolArgs a = pool_args(Q, nullptr, Nq, 0, block, nQB, 0, Qp, Kp, 0, nullptr, nullptr);
+    const long long q_ctas = static_cast<long long>(BH) * nQB;
+    if (launch_pdl(hf::pool_q_push_kernel<D>, q_ctas + push_ctas, hf::kPoolThreads, 0, st, a, *push,
+                   static_cast<int>(q_ctas)) != HF_OK)
+      return HF_ERR_CUDA;
+  } else if (launch_pool<D, false>(Q, nullptr, BH, Nq, 0, block, nQB, 0, Qp, Kp, 0, nullptr, st) != HF_OK) {
     return HF_ERR_CUDA;
+  }
   constexpr int kWarpsPerCta = hf::kPoolThreads / 32;
-  const long long ctas = (static_cast<long long>(BH) * nKB + kWarpsPerCta - 1) / kWarpsPerCta;
-  if (launch_pdl(hf::kpool_blocks_kernel<D>, ctas, hf::kPoolThreads, 0, st, static_cast<const float*>(kp->sums),
-                 kp->capacity, kp->head, kp->n_gran, kp->granule, block, nKB, BH, Kp) != HF_OK)
-    return HF_ERR_CUDA;
-  return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st, /*transposed=*/false);
+  const bool staged = staged_scores<D>(nKB);
+  const float* sums = static_cast<const float*>(kp->sums);
+  const hf_status rc =
+      staged ? launch_pdl(hf::kpool_blocks_kernel<D, true>,
+                          static_cast<long long>(BH) * ((nKB + kWarpsPerCta - 1) / kWarpsPerCta), hf::kPoolThreads, 0,
+                          st, sums, kp->capacity, kp->head, kp->n_gran, kp->granule, block, nKB, BH, Kp)
+             : launch_pdl(hf::kpool_blocks_kernel<D, false>,
+                          (static_cast<long long>(BH) * nKB + kWarpsPerCta - 1) / kWarpsPerCta, hf::kPoolThreads, 0,
+                          st, sums, kp->capacity, kp->head, kp->n_gran, kp->granule, block, nKB, BH, Kp);
+  if (rc != HF_OK) return HF_ERR_CUDA;
+  return launch_score<D>(Qp, Kp, BH, nQB, nKB, r, idx, scores, st, staged);
 }
 
 // ---------------------------------------------------------------- two-stage select
@@ -624,7 +640,14 @@ HF_API hf_status hf_kpool_init(hf_kpool* kp, int B, int H, int d, int granule, i
   return HF_OK;
 }
 
-HF_API hf_status hf_kpool_push(hf_kpool* kp, const hf_bf16* K_new, int n_tokens, int n_evict, void* stream) {
+// The window after a push (validated; kp unchanged) and the push's kernel arguments.
+struct PushPlan {
+  int head, n_gran;     // the window after the push
+  hf::PushArgs args;    // n_new == 0: no device work
+  long long ctas;       // push CTAs
+};
+
+static hf_status plan_push(const hf_kpool* kp, const hf_bf16* K_new, int n_tokens, int n_evict, PushPlan* pl) {
   if (!kp || !kp->sums || kp->B < 1 || kp->H < 1 || kp->capacity < 1 || kp->granule < 1) return HF_ERR_INVALID_ARG;
   if (!supported_d(kp->d)) return HF_ERR_UNSUPPORTED;
   const int G = kp->granule, cap = kp->capacity;
@@ -635,29 +658,37 @@ HF_API hf_status hf_kpool_push(hf_kpool* kp, const hf_bf16* K_new, int n_tokens,
   if (n_new > 0 && !K_new) return HF_ERR_INVALID_ARG;
   if (n_new > 0 && !aligned16(K_new)) return HF_ERR_ALIGNMENT;
   const int head = (kp->head + ev) % cap, kept = kp->n_gran - ev;
-  if (n_new > 0) {
-    const long long BH = static_cast<long long>(kp->B) * kp->H;
-    constexpr int kGran128 = hf::kPoolThreads / (128 / 8), kGran64 = hf::kPoolThreads / (64 / 8);
-    const long long groups = (n_new + (kp->d == 128 ? kGran128 : kGran64) - 1) / (kp->d == 128 ? kGran128 : kGran64);
-    if (BH * groups > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
-    const int base = (head + kept) % cap;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const __nv_bfloat16* K = reinterpret_cast<const __nv_bfloat16*>(K_new);
-    const hf_status rc =
-        kp->d == 128 ? launch_pdl(hf::kpool_push_kernel<128>, BH * groups, hf::kPoolThreads, 0, s, K, n_tokens, G,
-                                  n_new, base, cap, kp->sums)
-                     : launch_pdl(hf::kpool_push_kernel<64>, BH * groups, hf::kPoolThreads, 0, s, K, n_tokens, G,
-                                  n_new, base, cap, kp->sums);
-    if (rc != HF_OK) return HF_ERR_CUDA;
-  }
-  kp->head = head;
-  kp->n_gran = kept + n_new;
+  constexpr int kGran128 = hf::kPoolThreads / (128 / 8), kGran64 = hf::kPoolThreads / (64 / 8);
+  const int per_cta = kp->d == 128 ? kGran128 : kGran64;
+  const long long BH = static_cast<long long>(kp->B) * kp->H;
+  pl->ctas = n_new > 0 ? BH * ((n_new + per_cta - 1) / per_cta) : 0;
+  if (pl->ctas > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  pl->head = head;
+  pl->n_gran = kept + n_new;
+  pl->args = hf::PushArgs{reinterpret_cast<const __nv_bfloat16*>(K_new), n_tokens, G, n_new, (head + kept) % cap,
+                          cap, kp->sums};
   return HF_OK;
 }
 
-HF_API hf_status hf_select_blocks_cached(const hf_bf16* Q, const hf_kpool* kp, int Nq, int block, int r,
-                                         int32_t* idx_out, float* scores_out, void* ws, size_t ws_bytes,
-                                         void* stream) {
+HF_API hf_status hf_kpool_push(hf_kpool* kp, const hf_bf16* K_new, int n_tokens, int n_evict, void* stream) {
+  PushPlan pl;
+  const hf_status rc = plan_push(kp, K_new, n_tokens, n_evict, &pl);
+  if (rc != HF_OK) return rc;
+  if (pl.ctas > 0) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const hf_status lr = kp->d == 128 ? launch_pdl(hf::kpool_push_kernel<128>, pl.ctas, hf::kPoolThreads, 0, s, pl.args)
+                                      : launch_pdl(hf::kpool_push_kernel<64>, pl.ctas, hf::kPoolThreads, 0, s, pl.args);
+    if (lr != HF_OK) return HF_ERR_CUDA;
+  }
+  kp->head = pl.head;
+  kp->n_gran = pl.n_gran;
+  return HF_OK;
+}
+
+// Checks of a cached selection over the window of kp; *Nk_out: its key tokens.
+static hf_status check_select_cached(const hf_bf16* Q, const hf_kpool* kp, int Nq, int block, int r,
+                                     const int32_t* idx_out, const float* scores_out, const void* ws,
+                                     size_t ws_bytes, int* Nk_out) {
   if (!kp || !kp->sums || kp->B < 1 || kp->H < 1 || kp->granule < 1 || Nq < 0) return HF_ERR_INVALID_ARG;
   if (kp->n_gran < 1 || kp->n_gran > kp->capacity || kp->head < 0 || kp->head >= kp->capacity)
     return HF_ERR_INVALID_ARG;
@@ -669,6 +700,7 @@ HF_API hf_status hf_select_blocks_cached(const hf_bf16* Q, const hf_kpool* kp, i
   const int nKB = ceil_div(Nk, block);
   if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
   if (nKB > hf::kMaxKeyBlocks) return HF_ERR_UNSUPPORTED;
+  *Nk_out = Nk;
   if (Nq == 0) return HF_OK;
   if (!Q || !idx_out) return HF_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(idx_out) || (scores_out && !aligned16(scores_out))) return HF_ERR_ALIGNMENT;
@@ -676,10 +708,47 @@ HF_API hf_status hf_select_blocks_cached(const hf_bf16* Q, const hf_kpool* kp, i
   if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
   const long long BH = static_cast<long long>(B) * H;
   if (BH * (ceil_div(Nq, block) + nKB) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  return HF_OK;
+}
+
+HF_API hf_status hf_select_blocks_cached(const hf_bf16* Q, const hf_kpool* kp, int Nq, int block, int r,
+                                         int32_t* idx_out, float* scores_out, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  int Nk = 0;
+  const hf_status rc = check_select_cached(Q, kp, Nq, block, r, idx_out, scores_out, ws, ws_bytes, &Nk);
+  if (rc != HF_OK || Nq == 0) return rc;
+  const int BH = kp->B * kp->H;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 128
-             ? launch_select_cached<128>(Q, kp, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s)
-             : launch_select_cached<64>(Q, kp, static_cast<int>(BH), Nq, Nk, block, r, idx_out, scores_out, ws, s);
+  return kp->d == 128 ? launch_select_cached<128>(Q, kp, BH, Nq, Nk, block, r, idx_out, scores_out, ws, s)
+                      : launch_select_cached<64>(Q, kp, BH, Nq, Nk, block, r, idx_out, scores_out, ws, s);
+}
+
+HF_API hf_status hf_select_blocks_cached_push(const hf_bf16* Q, hf_kpool* kp, const hf_bf16* K_new, int n_tokens,
+                                              int n_evict, int Nq, int block, int r, int32_t* idx_out,
+                                              float* scores_out, void* ws, size_t ws_bytes, void* stream) {
+  PushPlan pl;
+  hf_status rc = plan_push(kp, K_new, n_tokens, n_evict, &pl);
+  if (rc != HF_OK) return rc;
+  hf_kpool after = *kp;
+  after.head = pl.head;
+  after.n_gran = pl.n_gran;
+  int Nk = 0;
+  rc = check_select_cached(Q, &after, Nq, block, r, idx_out, scores_out, ws, ws_bytes, &Nk);
+  if (rc != HF_OK) return rc;
+  const int BH = kp->B * kp->H;
+  if (static_cast<long long>(BH) * ceil_div(Nq, block) + pl.ctas > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (Nq == 0) {
+    // nothing to select: the push alone
+    return hf_kpool_push(kp, K_new, n_tokens, n_evict, stream);
+  }
+  const hf::PushArgs* push = pl.ctas > 0 ? &pl.args : nullptr;
+  rc = kp->d == 128
+           ? launch_select_cached<128>(Q, &after, BH, Nq, Nk, block, r, idx_out, scores_out, ws, s, push, pl.ctas)
+           : launch_select_cached<64>(Q, &after, BH, Nq, Nk, block, r, idx_out, scores_out, ws, s, push, pl.ctas);
+  if (rc != HF_OK) return rc;
+  *kp = after;
+  return HF_OK;
 }
 
 HF_API hf_status hf_select_blocks_two_stage(const hf_bf16* Q, const hf_bf16* K, int B, int H, int Nq, int Nk,

@@ -504,90 +504,147 @@ __global__ void __launch_bounds__(kSelectThreads) score_select_staged_kernel(con
 // selection pools its key blocks from the sums (kpool_blocks_kernel) instead of reading
 // K. G divides the block size, so a key block is a whole run of granules.
 
-// sums[bh][(base + g) % cap][:] = sum of the rows [g*G, g*G + G) of K[bh], g < n_new.
-// A thread sums 8 columns of one granule (16-byte loads, 8 in flight); a warp reads whole
-// rows (two granules at d = 128, four at d = 64).
+// A push of n_new granules of G tokens of K ([BH][n_tokens][D]) into ring slots
+// (base + g) % cap of sums ([BH][cap][D]).
+struct PushArgs {
+  const __nv_bfloat16* K;
+  int n_tokens, G, n_new, base, cap;
+  float* sums;
+};
+
+// sums[bh][(base + g) % cap][:] = sum of the rows [g*G, g*G + G) of K[bh], g < n_new, for
+// the granules of push CTA `cta` (BH x ceil(n_new / granules per CTA) of them). A thread
+// sums 8 columns of one granule (16-byte loads, 8 in flight); a warp reads whole rows (two
+// granules at d = 128, four at d = 64).
 template <int D>
-__global__ void __launch_bounds__(kPoolThreads) kpool_push_kernel(const __nv_bfloat16* __restrict__ K,
-                                                                  int n_tokens, int G, int n_new, int base,
-                                                                  int cap, float* __restrict__ sums) {
+__device__ __forceinline__ void push_granules(const PushArgs& q, int cta) {
   constexpr int kVec = 8;
   constexpr int kTpr = D / kVec;                 // threads per granule
   constexpr int kGran = kPoolThreads / kTpr;     // granules per CTA
   constexpr int kUnroll = 8;
-  griddep_wait();
-  griddep_launch_dependents();
-  const int groups = (n_new + kGran - 1) / kGran;
-  const int bh = blockIdx.x / groups;
-  const int g = (blockIdx.x % groups) * kGran + threadIdx.x / kTpr;
+  const int groups = (q.n_new + kGran - 1) / kGran;
+  const int bh = cta / groups;
+  const int g = (cta % groups) * kGran + threadIdx.x / kTpr;
   const int c = threadIdx.x % kTpr;
-  if (g >= n_new) return;
-  const __nv_bfloat16* X = K + (static_cast<size_t>(bh) * n_tokens + static_cast<size_t>(g) * G) * D + c * kVec;
+  if (g >= q.n_new) return;
+  const __nv_bfloat16* X = q.K + (static_cast<size_t>(bh) * q.n_tokens + static_cast<size_t>(g) * q.G) * D + c * kVec;
   float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   int row = 0;
-  for (; row + kUnroll <= G; row += kUnroll) {
+  for (; row + kUnroll <= q.G; row += kUnroll) {
     uint4 v[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) v[u] = ld_stream_16(X + static_cast<size_t>(row + u) * D);
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) acc_bf16x8(acc, v[u]);
   }
-  for (; row < G; ++row) acc_bf16x8(acc, ld_stream_16(X + static_cast<size_t>(row) * D));
-  float4* out = reinterpret_cast<float4*>(sums + (static_cast<size_t>(bh) * cap + (base + g) % cap) * D + c * kVec);
+  for (; row < q.G; ++row) acc_bf16x8(acc, ld_stream_16(X + static_cast<size_t>(row) * D));
+  float4* out =
+      reinterpret_cast<float4*>(q.sums + (static_cast<size_t>(bh) * q.cap + (q.base + g) % q.cap) * D + c * kVec);
   out[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
   out[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads) kpool_push_kernel(PushArgs q) {
+  griddep_wait();
+  griddep_launch_dependents();
+  push_granules<D>(q, blockIdx.x);
+}
+
+// The query blocks' means (CTAs [0, BH nQB), as pool_blocks_kernel without key blocks) and
+// a push (the other CTAs) in one launch: a chunk step's new keys enter the cache while its
+// queries are pooled.
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads, 8) pool_q_push_kernel(PoolArgs a, PushArgs q, int q_ctas) {
+  __shared__ float red[PoolShape<D>::kRedFloats];
+  griddep_wait();
+  griddep_launch_dependents();
+  if (static_cast<int>(blockIdx.x) < q_ctas)
+    pool_block<D, false, false>(a, blockIdx.x / a.nQB, blockIdx.x % a.nQB, false, red, red);
+  else
+    push_granules<D>(q, blockIdx.x - q_ctas);
 }
 
 // Kp[bh][J][:] = mean of key block J of the window = (sum of its granule sums, in order) /
 // its valid length; the window is the n_gran granules from ring slot head on. One warp per
 // key block, D/32 columns a lane (512 contiguous bytes per load at d = 128), 8 in flight.
-template <int D>
+// kT: the means go out transposed, Kp[bh][k][J] (for score_select_staged_kernel): a CTA
+// takes 8 consecutive key blocks of one (b, h), stages their means in shared memory and
+// writes each k's 8 values as one 32-byte run.
+template <int D, bool kT>
 __global__ void __launch_bounds__(kPoolThreads) kpool_blocks_kernel(const float* __restrict__ sums, int cap,
                                                                     int head, int n_gran, int G, int block,
                                                                     int nKB, int BH, float* __restrict__ Kp) {
   constexpr int kC = D / 32;  // columns per lane: 4 or 2
   constexpr int kUnroll = 8;
+  constexpr int kWarps = kPoolThreads / 32;
+  __shared__ float tile[kT ? kWarps : 1][D];
   griddep_wait();
   griddep_launch_dependents();
-  const long long wid = static_cast<long long>(blockIdx.x) * (kPoolThreads / 32) + threadIdx.x / 32;
-  if (wid >= static_cast<long long>(BH) * nKB) return;
-  const int lane = threadIdx.x % 32;
-  const int bh = static_cast<int>(wid / nKB), J = static_cast<int>(wid % nKB);
-  const int per_block = block / G;
-  const int g_lo = J * per_block, g_hi = min(g_lo + per_block, n_gran);
-  const float* S = sums + static_cast<size_t>(bh) * cap * D + lane * kC;
+  const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
+  int bh, J;
+  if constexpr (kT) {
+    const int groups = (nKB + kWarps - 1) / kWarps;
+    bh = blockIdx.x / groups;
+    J = (blockIdx.x % groups) * kWarps + w;
+  } else {
+    const long long wid = static_cast<long long>(blockIdx.x) * kWarps + w;
+    if (wid >= static_cast<long long>(BH) * nKB) return;
+    bh = static_cast<int>(wid / nKB);
+    J = static_cast<int>(wid % nKB);
+  }
   float acc[kC];
 #pragma unroll
   for (int k = 0; k < kC; ++k) acc[k] = 0.f;
-  for (int g0 = g_lo; g0 < g_hi; g0 += kUnroll) {
-    float v[kUnroll][kC];
+  const int per_block = block / G;
+  const int g_lo = J * per_block, g_hi = min(g_lo + per_block, n_gran);
+  if (J < nKB) {
+    const float* S = sums + static_cast<size_t>(bh) * cap * D + lane * kC;
+    for (int g0 = g_lo; g0 < g_hi; g0 += kUnroll) {
+      float v[kUnroll][kC];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int g = g0 + u;
-      if (g < g_hi) {
-        const float* src = S + static_cast<size_t>((head + g) % cap) * D;
-        if constexpr (kC == 4) {
-          const float4 f = __ldg(reinterpret_cast<const float4*>(src));
-          v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
+      for (int u = 0; u < kUnroll; ++u) {
+        const int g = g0 + u;
+        if (g < g_hi) {
+          const float* src = S + static_cast<size_t>((head + g) % cap) * D;
+          if constexpr (kC == 4) {
+            const float4 f = __ldg(reinterpret_cast<const float4*>(src));
+            v[u][0] = f.x; v[u][1] = f.y; v[u][2] = f.z; v[u][3] = f.w;
+          } else {
+            const float2 f = __ldg(reinterpret_cast<const float2*>(src));
+            v[u][0] = f.x; v[u][1] = f.y;
+          }
         } else {
-          const float2 f = __ldg(reinterpret_cast<const float2*>(src));
-          v[u][0] = f.x; v[u][1] = f.y;
+#pragma unroll
+          for (int k = 0; k < kC; ++k) v[u][k] = 0.f;
         }
-      } else {
-#pragma unroll
-        for (int k = 0; k < kC; ++k) v[u][k] = 0.f;
       }
-    }
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < kUnroll; ++u) {
 #pragma unroll
-      for (int k = 0; k < kC; ++k) acc[k] += v[u][k];
+        for (int k = 0; k < kC; ++k) acc[k] += v[u][k];
+      }
     }
   }
   const float L = static_cast<float>((g_hi - g_lo) * G);
-  float* out = Kp + (static_cast<size_t>(bh) * nKB + J) * D + lane * kC;
+  if constexpr (kT) {
+    if (J < nKB) {
 #pragma unroll
-  for (int k = 0; k < kC; ++k) out[k] = acc[k] / L;
+      for (int k = 0; k < kC; ++k) tile[w][lane * kC + k] = acc[k] / L;
+    }
+    __syncthreads();
+    // thread t writes key block J0 + t % 8 of dimension t / 8 (+ 32 per step)
+    const int j = threadIdx.x % kWarps, J0 = J - w;
+    if (J0 + j < nKB) {
+#pragma unroll
+      for (int k = threadIdx.x / kWarps; k < D; k += kPoolThreads / kWarps)
+        Kp[(static_cast<size_t>(bh) * D + k) * nKB + J0 + j] = tile[j][k];
+    }
+  } else {
+    float* out = Kp + (static_cast<size_t>(bh) * nKB + J) * D + lane * kC;
+#pragma unroll
+    for (int k = 0; k < kC; ++k) out[k] = acc[k] / L;
+  }
 }
 
 // ------------------------------------------------------------ two-stage selection

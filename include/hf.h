@@ -243,6 +243,15 @@ HF_API hf_status hf_select_blocks_cached(const hf_bf16* Q, const hf_kpool* kp, i
                                          int32_t* idx_out, float* scores_out, void* ws, size_t ws_bytes,
                                          void* stream);
 
+/* hf_kpool_push(kp, K_new, n_tokens, n_evict) then hf_select_blocks_cached(Q, kp, ...) as
+ * one call, the chunk step of the cache: the new keys' granule sums are computed in the
+ * launch that pools Q (one launch fewer than the two calls). Same results, ordering rules
+ * and errors as the two calls; on any error kp is unchanged and nothing is launched
+ * (HF_ERR_CUDA: a launch failed, kp unchanged). Nq == 0: the push alone. */
+HF_API hf_status hf_select_blocks_cached_push(const hf_bf16* Q, hf_kpool* kp, const hf_bf16* K_new, int n_tokens,
+                                              int n_evict, int Nq, int block, int r, int32_t* idx_out,
+                                              float* scores_out, void* ws, size_t ws_bytes, void* stream);
+
 /* Upper bound, in bytes, of the select workspace that hf_select_blocks_noalloc can
  * serve: a call is accepted when hf_workspace_size(HF_WS_SELECT, ...) for its shapes
  * is at most this (e.g. 12 heads x 4680 query x 32760 key tokens at d = 128, block

@@ -217,6 +217,33 @@ def test_select_cached_validation():
     assert sel(kp) == B.HF_ERR_INVALID_ARG            # a corrupted head
 
 
+def test_select_cached_push_validation():
+    """The fused push + cached selection checks both halves before anything runs: an error
+    from either leaves the cache unchanged."""
+    L = hf.lib()
+    _, kp = _kp()
+    kp.n_gran, kp.head = 32, 60   # 256 key tokens: 8 blocks of 32, the window wrapping the ring
+
+    def call(**kw):
+        a = dict(Q=A, K=A, n=64, ev=64, Nq=64, block=32, r=2, idx=A, ws=A, ws_bytes=1 << 20)
+        a.update(kw)
+        return L.hf_select_blocks_cached_push(a["Q"], ctypes.byref(kp), a["K"], a["n"], a["ev"], a["Nq"],
+                                              a["block"], a["r"], a["idx"], None, a["ws"], a["ws_bytes"], None)
+    assert call(n=12) == B.HF_ERR_INVALID_ARG              # the push: not whole granules
+    assert call(n=41 * 8) == B.HF_ERR_INVALID_ARG          # the push: over capacity (32 - 8 + 41 > 64)
+    assert call(K=A + 2) == B.HF_ERR_ALIGNMENT              # the push: unaligned keys
+    assert call(r=9) == B.HF_ERR_INVALID_ARG                # the select: r above the window's 8 blocks
+    assert call(ev=0, r=11) == B.HF_ERR_INVALID_ARG         # ... and above 10 blocks after a push of 64
+    assert call(block=48) == B.HF_ERR_UNSUPPORTED
+    assert call(Q=A + 2) == B.HF_ERR_ALIGNMENT
+    assert call(ws_bytes=100) == B.HF_ERR_WORKSPACE
+    assert call(n=0, ev=256) == B.HF_ERR_INVALID_ARG        # the window left empty
+    assert (kp.n_gran, kp.head) == (32, 60)
+    # evicting only, with no queries, is the push's host bookkeeping alone
+    assert call(K=None, n=0, ev=64, Nq=0) == B.HF_OK
+    assert (kp.n_gran, kp.head) == (24, (60 + 8) % 64)
+
+
 def test_kpool_binding_checks_shapes_before_any_call():
     """The Python binding rejects mismatched tensors on the host (no device needed)."""
     import torch

@@ -92,3 +92,33 @@ def test_cached_select_832x480_window():
     hf.hf_kpool_push(kp, new.contiguous().to(DEV), n_evict=wl.Nq)
     moved = torch.cat([K[:, :, wl.Nq:], new], dim=2)
     _check(Q, moved, kp, wl.block, wl.r)
+
+
+def test_cached_push_equals_push_then_select():
+    """hf_select_blocks_cached_push (the push's sums computed in the Q pooling launch) gives
+    the same ring, blocks and scores, bit for bit, as hf_kpool_push then
+    hf_select_blocks_cached, step after step of a moving window that wraps its ring."""
+    B, H, d, G, block, r = 2, 3, 128, 8, 64, 3
+    W, step = 640, 200
+    keys = _gen(21, B, H, W + 6 * step, d).to(DEV)
+    sums_a = torch.zeros(B, H, W // G + 5, d, dtype=torch.float32, device=DEV)
+    sums_b = torch.zeros_like(sums_a)
+    kp_a, kp_b = hf.hf_kpool_init(sums_a, G), hf.hf_kpool_init(sums_b, G)
+    hf.hf_kpool_push(kp_a, keys[:, :, :W].contiguous())
+    hf.hf_kpool_push(kp_b, keys[:, :, :W].contiguous())
+    for s in range(6):
+        Q = _gen(200 + s, B, H, 150, d).to(DEV)
+        new = keys[:, :, W + s * step:W + (s + 1) * step].contiguous()
+        nKB = -(-W // block)
+        sc_a = torch.empty(B, H, -(-150 // block), nKB, dtype=torch.float32, device=DEV)
+        sc_b = torch.empty_like(sc_a)
+        hf.hf_kpool_push(kp_a, new, n_evict=step)
+        idx_a = hf.hf_select_blocks_cached(Q, kp_a, block, r, scores_out=sc_a)
+        idx_b = hf.hf_select_blocks_cached_push(Q, kp_b, new, block, r, n_evict=step, scores_out=sc_b)
+        torch.cuda.synchronize()
+        assert hf.hf_query_status()[0] == hf.HF_OK
+        assert (kp_a.c.head, kp_a.c.n_gran) == (kp_b.c.head, kp_b.c.n_gran)
+        assert torch.equal(idx_a, idx_b) and torch.equal(sc_a, sc_b)
+        assert torch.equal(sums_a, sums_b)
+    # and against the oracle over the last window
+    _check(Q.cpu(), keys[:, :, 6 * step:6 * step + W].cpu(), kp_b, block, r)
