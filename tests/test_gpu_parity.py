@@ -102,6 +102,32 @@ def test_select_ties_lower_index():
                     assert J - 4 in row
 
 
+@pytest.mark.parametrize("nKB,r", [(256, 1), (256, 64), (256, 255), (256, 256), (200, 37), (300, 64), (300, 299)])
+def test_select_scores_differing_in_low_bits(nKB, r):
+    """Pooled scores 1 + j 2^-20 (exact in fp32: query rows (1, 1, 0, ...), key block J's rows
+    (1, j_J 2^-20, 0, ...)), so the order is decided by the low bytes of the keys, with
+    every value of j repeated: the kept blocks are the r largest j, the lower J first among
+    equal ones, exactly."""
+    d, block = 128, 32
+    g = torch.Generator().manual_seed(nKB + r)
+    j = torch.randint(0, 64, (nKB,), generator=g) * 4 + torch.randint(0, 2, (nKB,), generator=g)
+    K = torch.zeros(1, 2, nKB * block, d)
+    K[..., 0] = 1.0
+    K[0, 0, :, 1] = (j.double() * 2.0 ** -20).repeat_interleave(block).float()
+    K[0, 1, :, 1] = (j.flip(0).double() * 2.0 ** -20).repeat_interleave(block).float()
+    Q = torch.zeros(1, 2, 2 * block, d)
+    Q[..., :2] = 1.0
+    Q, K = Q.bfloat16(), K.bfloat16()
+    assert torch.equal(K[0, 0, ::block, 1].double(), j.double() * 2.0 ** -20)  # exact in bf16
+    idx, scores = _run_select(Q, K, block, r)
+    for h, jj in ((0, j), (1, j.flip(0))):
+        assert np.array_equal(scores[0, h, 0], (1.0 + jj.double() * 2.0 ** -20).float().numpy())
+        order = sorted(range(nKB), key=lambda J: (-int(jj[J]), J))
+        want = np.sort(np.array(order[:r], dtype=np.int32))
+        for I in range(2):
+            assert np.array_equal(idx[0, h, I], want), (h, I)
+
+
 # --------------------------------------------------------------------------- absorb
 @pytest.mark.parametrize("B,H,n,d", [(1, 1, 192, 64), (1, 2, 1000, 128), (2, 3, 77, 128), (1, 12, 4680, 128),
                                      (1, 1, 1, 64), (1, 40, 130, 64),
