@@ -34,7 +34,8 @@ class HfStateC(ctypes.Structure):
     """Mirror of ``struct hf_state``."""
 
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("d", ctypes.c_int),
-                ("S", ctypes.c_void_p), ("z", ctypes.c_void_p), ("n_absorbed", ctypes.c_longlong)]
+                ("S", ctypes.c_void_p), ("z", ctypes.c_void_p), ("S_split", ctypes.c_void_p),
+                ("n_absorbed", ctypes.c_longlong)]
 
 
 class HfKpoolC(ctypes.Structure):
@@ -68,7 +69,7 @@ _lib = None
 _SIGNATURES = {
     "hf_workspace_size": (ctypes.c_size_t, [ctypes.c_int] * 8),
     "hf_state_init": (ctypes.c_int, [ctypes.POINTER(HfStateC), ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+                                     ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
     "hf_absorb_evicted": (ctypes.c_int, [ctypes.POINTER(HfStateC), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
                                          ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "hf_select_blocks": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 7 +
@@ -185,11 +186,13 @@ def _qkv_dims(Q: torch.Tensor, K: torch.Tensor, name_k: str = "K"):
 
 
 class HfState:
-    """Python handle of ``hf_state``: keeps S [B,H,d,d] and z [B,H,d] (fp32, device) alive."""
+    """Python handle of ``hf_state``: keeps S [B,H,d,d], z [B,H,d] (fp32, device) and the
+    split copy of S that the library maintains (``S_split``, bytes) alive."""
 
-    def __init__(self, S: torch.Tensor, z: torch.Tensor):
+    def __init__(self, S: torch.Tensor, z: torch.Tensor, S_split: torch.Tensor):
         self.S = S
         self.z = z
+        self.S_split = S_split
         self.c = HfStateC()
 
     @property
@@ -229,14 +232,20 @@ def _workspace(nbytes: int, device, ws):
     return ws, ws.numel() * ws.element_size()
 
 
-def hf_state_init(S: torch.Tensor, z: torch.Tensor, stream=None) -> HfState:
-    """Bind S [B,H,d,d] and z [B,H,d] (fp32) as a state and zero them."""
+def hf_state_init(S: torch.Tensor, z: torch.Tensor, S_split=None, stream=None) -> HfState:
+    """Bind S [B,H,d,d] and z [B,H,d] (fp32) as a state and zero them. S_split: the
+    library's split copy of S (uint8 [B*H*4*d*d] on S's device; allocated when None)."""
     if S.dim() != 4 or z.dim() != 3:
         raise ValueError("S must be [B,H,d,d] and z [B,H,d]")
     B, H, d, _ = S.shape
-    st = HfState(S, z)
+    if S_split is None:
+        S_split = torch.empty(B * H * 4 * d * d, dtype=torch.uint8, device=S.device)
+    if S_split.dtype != torch.uint8 or S_split.numel() < B * H * 4 * d * d:
+        raise ValueError(f"S_split must be uint8 with at least {B * H * 4 * d * d} bytes")
+    st = HfState(S, z, S_split)
     _check(lib().hf_state_init(ctypes.byref(st.c), B, H, d, _dev(S, torch.float32, "S"),
-                               _dev(z, torch.float32, "z"), _stream(stream)), "hf_state_init")
+                               _dev(z, torch.float32, "z"), _dev(S_split, torch.uint8, "S_split"),
+                               _stream(stream)), "hf_state_init")
     return st
 
 

@@ -345,9 +345,13 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
   if (!p.wait_first) griddep_wait();
 }
 
-// S[bh] += sum_s part_S[bh][s], z[bh] += sum_s part_z[bh][s], slices in order.
+// S[bh] += sum_s part_S[bh][s], z[bh] += sum_s part_z[bh][s], slices in order; S_split[bh]
+// (4 d^2 bytes a head) gets the new S as hi = bf16(S), lo = bf16(S - hi) in the tiles the
+// hybrid attention's readout MMAs read: hi, then lo, each d/64 chunks of 64 columns n, a
+// chunk d rows k of 128 bytes, 16-byte group g of row k at position g ^ (k % 8).
 template <int D>
 __global__ void __launch_bounds__(256) reduce_state_kernel(float* __restrict__ S, float* __restrict__ z,
+                                                           uint8_t* __restrict__ S_split,
                                                            const float* __restrict__ part_S,
                                                            const float* __restrict__ part_z, int nsplit) {
   constexpr int kVec4PerHead = D * D / 4;
@@ -379,6 +383,15 @@ __global__ void __launch_bounds__(256) reduce_state_kernel(float* __restrict__ S
       }
     }
     *s4 = acc;
+    // elements (k, n0 .. n0 + 3): half of a 16-byte group of the split tiles
+    const int k = (4 * e4) / D, n0 = (4 * e4) % D;
+    const uint32_t off = (n0 / 64) * (D * 128) + k * 128 + ((((n0 % 64) / 8) ^ (k & 7)) * 16) + (n0 % 8) * 2;
+    const uint32_t h01 = pack_bf16x2(acc.x, acc.y), h23 = pack_bf16x2(acc.z, acc.w);
+    const uint32_t l01 = pack_bf16x2(acc.x - bf16_lo_to_f32(h01), acc.y - bf16_hi_to_f32(h01));
+    const uint32_t l23 = pack_bf16x2(acc.z - bf16_lo_to_f32(h23), acc.w - bf16_hi_to_f32(h23));
+    uint8_t* sp = S_split + static_cast<size_t>(bh) * 4 * D * D + off;
+    *reinterpret_cast<uint2*>(sp) = make_uint2(h01, h23);
+    *reinterpret_cast<uint2*>(sp + 2 * D * D) = make_uint2(l01, l23);
   }
   if (blockIdx.x % kCtasPerHead == 0 && threadIdx.x < D) {
     float acc = z[static_cast<size_t>(bh) * D + threadIdx.x];

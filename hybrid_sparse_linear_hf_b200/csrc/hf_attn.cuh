@@ -68,6 +68,7 @@ static_assert(2 * 128 * kRegsSupportRope + 256 * kRegsRows <= kAttnThreadsRope *
 constexpr int kSmemLimit = 232448;  // max shared memory per CTA on sm_100
 constexpr int kAttnStaticSmem = 1024;  // upper bound of the kernel's static shared memory
 constexpr int kMaxSlots = 6;
+constexpr int kSplitCopyBytes = 32 * 1024;  // bytes per bulk copy of the state's split tiles
 
 template <int D, int BLK, bool kRope = false>
 struct AttnCfg {
@@ -96,7 +97,7 @@ struct AttnCfg {
 
 struct AttnParams {
   const int32_t* idx;  // [BH][nQB][r]
-  const float* S;      // [BH][D][D]
+  const uint8_t* S_split;  // [BH][hi | lo tile]: the state S split into two bf16 terms
   const float* z;      // [BH][D]
   int nQB, nKB, r;
   int last_len;        // valid tokens of key block nKB - 1
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
   uint8_t* vring = kring + NSK * C::kKVTileBytes;  // NSV V slots (S_hi/S_lo + exchange over both rings at the end)
 
   __shared__ uint64_t q_bar, kfull_bar[NSK], kempty_bar[NSK], vfull_bar[NSV], vempty_bar[NSV];
-  __shared__ uint64_t sfull_bar[2], pfull_bar[2], final_bar, pro_bar, lin_bar, drain_bar;
+  __shared__ uint64_t sfull_bar[2], pfull_bar[2], final_bar, pro_bar, lin_bar, drain_bar, split_bar;
   __shared__ uint64_t qrot_bar, krot_bar[NSK];  // kRope: the Q tile / K slot has been turned
   __shared__ uint32_t tmem_base_sh;
   __shared__ int abort_sh;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
       mbar_init(&pfull_bar[b], 5);  // the pipeline's 4 warps + warp 3
     }
     mbar_init(&final_bar, 1);
+    mbar_init(&split_bar, 1);
     mbar_init(&pro_bar, 8);  // the 8 softmax warps
     mbar_init(&lin_bar, 1);
     mbar_init(&drain_bar, 1);
@@ -291,8 +293,19 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
       }
       if (ok) {
         umma_commit(&final_bar);
+        // once every MMA is done the K ring is idle: the state's hi and lo tiles, kept beside
+        // the state in the readout MMAs' layout, go into it by bulk copies
+        bool copying = false;
+        if ((ok = mbar_wait(&final_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 9))) {
+          const uint8_t* src = p.S_split + static_cast<size_t>(bh) * C::kReadoutBytes;
+          mbar_arrive_expect_tx(&split_bar, C::kReadoutBytes);
+          for (int o = 0; o < C::kReadoutBytes; o += kSplitCopyBytes)
+            bulk_load(kring + o, src + o, min(kSplitCopyBytes, C::kReadoutBytes - o), &split_bar);
+          copying = true;
+        }
         // linear term: D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi
-        if ((ok = mbar_wait(&pro_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 5))) {
+        if (ok && (ok = mbar_wait(&pro_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 5)) &&
+            (ok = mbar_wait(&split_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 16))) {
           tc_fence_after();
           const uint64_t sdesc_hi = sdesc_sw128(smem_u32(kring), D * 128, 1024);
           const uint64_t sdesc_lo = sdesc_hi + ((D * D * 2) >> 4);
@@ -307,6 +320,7 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
           }
           umma_commit(&lin_bar);
         }
+        if (copying) mbar_wait_drain(&split_bar, 0, p.timeout_ns, (kKernAttn << 8) | 16);
       }
       umma_commit(&drain_bar);
       mbar_wait_drain(&drain_bar, 0, p.timeout_ns, (kKernAttn << 8) | 8);
@@ -518,20 +532,15 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
       ++i;
     }
 
-    // ---- linear term operands. This thread's halves of z and of S's row `row` do not depend
-    // on the MMAs: their loads are issued before the wait for the last MMAs, so that their
-    // L2 latency hides behind it, and the conversions below read registers.
+    // ---- linear term operands. This thread's half of z does not depend on the MMAs: its
+    // loads are issued before the wait for the last MMAs, so that their latency hides behind
+    // it. (The state's hi and lo tiles arrive in the K ring by the MMA thread's bulk copies.)
     constexpr int kQ4 = HD / 4;  // float4 per half row
-    float4 zv[kQ4], sv[kQ4];
+    float4 zv[kQ4];
     {
       const float4* z4 = reinterpret_cast<const float4*>(p.z + static_cast<size_t>(bh) * D + pipe * HD);
-      const float4* s4 =
-          reinterpret_cast<const float4*>(p.S + (static_cast<size_t>(bh) * D + min(row, D - 1)) * D + pipe * HD);
 #pragma unroll
-      for (int k = 0; k < kQ4; ++k) {
-        zv[k] = __ldg(z4 + k);
-        sv[k] = __ldg(s4 + k);
-      }
+      for (int k = 0; k < kQ4; ++k) zv[k] = __ldg(z4 + k);
     }
     // (all MMAs done: the S buffers and both rings are free)
     ok = ok && mbar_wait(&final_bar, 0, abort_flag, p.timeout_ns, (kKernAttn << 8) | 12);
@@ -539,31 +548,6 @@ __global__ void __launch_bounds__(kRope ? kAttnThreadsRope : kAttnThreads, 1)
     float dacc = 0.f;
     if (ok) {
       tc_fence_after();
-      // state rows: thread (k, pipe) converts S[bh][k][pipe*D/2 .. +D/2) into MN-major
-      // bf16 hi/lo tiles over the idle rings
-      if (row < D) {
-        uint8_t* s_hi = kring;
-        uint8_t* s_lo = kring + D * D * 2;
-#pragma unroll
-        for (int u = 0; u < HD / 8; ++u) {
-          const int unit = pipe * (HD / 8) + u;
-          const float4 a = sv[2 * u], b = sv[2 * u + 1];
-          const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-          uint32_t hv[4], lv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t hh = pack_bf16x2(f[2 * e], f[2 * e + 1]);
-            hv[e] = hh;
-            float r0, r1;
-            f32x2_split(ffma2(f32x2(bf16_lo_to_f32(hh), bf16_hi_to_f32(hh)), f32x2(-1.0f, -1.0f),
-                              f32x2(f[2 * e], f[2 * e + 1])), r0, r1);
-            lv[e] = pack_bf16x2(r0, r1);
-          }
-          const uint32_t off = (unit / 8) * (D * 128) + row * 128 + (((unit % 8) ^ (row & 7)) * 16);
-          *reinterpret_cast<uint4*>(s_hi + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-          *reinterpret_cast<uint4*>(s_lo + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
-        }
-      }
       // phi(x) = max(x, 0) + 2^(min(x, 0) log2 e) (branch-free elu + 1) on packed fp32 pairs;
       // phi . z accumulated as a pair, summed at the end
       uint64_t dacc2 = 0ull;

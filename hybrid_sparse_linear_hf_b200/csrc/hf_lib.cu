@@ -357,7 +357,8 @@ hf_status launch_absorb(hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, 
     return HF_ERR_CUDA;
   constexpr int kCtasPerHead = (D * D / 4 + 255) / 256;
   return launch_pdl(hf::reduce_state_kernel<D>, BH * kCtasPerHead, 256, 0, stream, st->S, st->z,
-                    static_cast<const float*>(p.part_S), static_cast<const float*>(p.part_z), pl.nsplit);
+                    static_cast<uint8_t*>(st->S_split), static_cast<const float*>(p.part_S),
+                    static_cast<const float*>(p.part_z), pl.nsplit);
 }
 
 // ---------------------------------------------------------------- attention
@@ -373,7 +374,7 @@ hf_status launch_attn(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, int 
     return HF_ERR_CUDA;
   hf::AttnParams p;
   p.idx = idx;
-  p.S = st->S;
+  p.S_split = static_cast<const uint8_t*>(st->S_split);
   p.z = st->z;
   p.nQB = nQB;
   p.nKB = nKB;
@@ -461,12 +462,12 @@ hf_status check_attn_args(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, 
   if (!supported_d(d) || !supported_block(block)) return HF_ERR_UNSUPPORTED;
   const int nKB = ceil_div(Nk, block);
   if (r < 1 || r > nKB) return HF_ERR_INVALID_ARG;
-  if (st->B != B || st->H != H || st->d != d || !st->S || !st->z) return HF_ERR_INVALID_ARG;
+  if (st->B != B || st->H != H || st->d != d || !st->S || !st->z || !st->S_split) return HF_ERR_INVALID_ARG;
   if (!(scale == scale) || std::isinf(scale)) return HF_ERR_INVALID_ARG;
   if (Nq == 0) return HF_OK;
   if (!Q || !K || !V || !idx || !O) return HF_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(idx) || !aligned16(st->S) ||
-      !aligned16(st->z))
+      !aligned16(st->z) || !aligned16(st->S_split))
     return HF_ERR_ALIGNMENT;
   if (static_cast<long long>(B) * H * ceil_div(Nq, block) > 0x7fffffffLL) return HF_ERR_UNSUPPORTED;
   return HF_OK;
@@ -475,11 +476,12 @@ hf_status check_attn_args(const hf_bf16* Q, const hf_bf16* K, const hf_bf16* V, 
 // Argument checks of hf_absorb_evicted for n_tokens >= 1 (nothing is launched).
 hf_status check_absorb_args(const hf_state* st, const hf_bf16* K_ev, const hf_bf16* V_ev, int n_tokens,
                             const void* ws, size_t ws_bytes) {
-  if (!st || !st->S || !st->z || st->B < 1 || st->H < 1 || n_tokens < 0) return HF_ERR_INVALID_ARG;
+  if (!st || !st->S || !st->z || !st->S_split || st->B < 1 || st->H < 1 || n_tokens < 0) return HF_ERR_INVALID_ARG;
   if (!supported_d(st->d)) return HF_ERR_UNSUPPORTED;
   if (n_tokens == 0) return HF_OK;
   if (!K_ev || !V_ev) return HF_ERR_INVALID_ARG;
-  if (!aligned16(K_ev) || !aligned16(V_ev) || !aligned16(st->S) || !aligned16(st->z)) return HF_ERR_ALIGNMENT;
+  if (!aligned16(K_ev) || !aligned16(V_ev) || !aligned16(st->S) || !aligned16(st->z) || !aligned16(st->S_split))
+    return HF_ERR_ALIGNMENT;
   const size_t need = absorb_ws_bytes(st->B, st->H, n_tokens, st->d);
   if (!ws || ws_bytes < need) return HF_ERR_WORKSPACE;
   if (!aligned16(ws)) return HF_ERR_ALIGNMENT;
@@ -550,19 +552,22 @@ HF_API size_t hf_workspace_size(int which, int B, int H, int Nq, int Nk, int d, 
   return static_cast<size_t>(-1);
 }
 
-HF_API hf_status hf_state_init(hf_state* st, int B, int H, int d, float* S_dev, float* z_dev, void* stream) {
-  if (!st || !S_dev || !z_dev || B < 1 || H < 1) return HF_ERR_INVALID_ARG;
+HF_API hf_status hf_state_init(hf_state* st, int B, int H, int d, float* S_dev, float* z_dev, void* S_split_dev,
+                               void* stream) {
+  if (!st || !S_dev || !z_dev || !S_split_dev || B < 1 || H < 1) return HF_ERR_INVALID_ARG;
   if (!supported_d(d)) return HF_ERR_UNSUPPORTED;
-  if (!aligned16(S_dev) || !aligned16(z_dev)) return HF_ERR_ALIGNMENT;
+  if (!aligned16(S_dev) || !aligned16(z_dev) || !aligned16(S_split_dev)) return HF_ERR_ALIGNMENT;
   const size_t bh = static_cast<size_t>(B) * H;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(S_dev, 0, bh * d * d * sizeof(float), s) != cudaSuccess) return HF_ERR_CUDA;
   if (cudaMemsetAsync(z_dev, 0, bh * d * sizeof(float), s) != cudaSuccess) return HF_ERR_CUDA;
+  if (cudaMemsetAsync(S_split_dev, 0, HF_STATE_SPLIT_BYTES(B, H, d), s) != cudaSuccess) return HF_ERR_CUDA;
   st->B = B;
   st->H = H;
   st->d = d;
   st->S = S_dev;
   st->z = z_dev;
+  st->S_split = S_split_dev;
   st->n_absorbed = 0;
   return HF_OK;
 }

@@ -80,15 +80,26 @@ typedef enum hf_status {
 /* Compact key-value state of the linear temporal attention, one per (b, h):
  *   S[b][h][k][n] = sum over absorbed tokens t of phi(k_t)[k] * v_t[n]   (fp32, d x d)
  *   z[b][h][k]    = sum over absorbed tokens t of phi(k_t)[k]           (fp32, d)
- * S and z are caller-owned device buffers of B*H*d*d and B*H*d floats. n_absorbed is a
- * host-side count of tokens absorbed per head (bookkeeping only; the kernels do not
- * read it). The state's size does not depend on how many tokens it has absorbed. */
+ * S and z are caller-owned device buffers of B*H*d*d and B*H*d floats. S_split is a
+ * caller-owned device buffer of HF_STATE_SPLIT_BYTES(B, H, d) bytes (16-byte aligned)
+ * that the library keeps equal to S split into two bf16 terms, hi = bf16(S) and
+ * lo = bf16(S - hi) (round to nearest even), in the layout the hybrid attention's
+ * readout MMAs read: per (b, h) the hi tile, then the lo tile, each d/64 chunks of 64
+ * columns n, a chunk d rows k of 128 bytes, the 16-byte group g of row k stored at
+ * position g ^ (k % 8). It changes with S (hf_state_init, hf_absorb_evicted and the fused
+ * calls); a caller that writes S itself leaves it stale. n_absorbed is a host-side count
+ * of tokens absorbed per head (bookkeeping only; the kernels do not read it). The state's
+ * size does not depend on how many tokens it has absorbed. */
 typedef struct hf_state {
   int B, H, d;
   float* S;
   float* z;
+  void* S_split;
   long long n_absorbed;
 } hf_state;
+
+/* Bytes of a state's S_split buffer: two bf16 d x d tiles per (b, h). */
+#define HF_STATE_SPLIT_BYTES(B, H, d) ((size_t)(B) * (size_t)(H) * 4u * (size_t)(d) * (size_t)(d))
 
 /* Workspace kinds for hf_workspace_size. */
 enum { HF_WS_SELECT = 1, HF_WS_ATTN = 2, HF_WS_ABSORB = 3, HF_WS_SELECT_TWO_STAGE = 4 };
@@ -98,10 +109,11 @@ enum { HF_WS_SELECT = 1, HF_WS_ATTN = 2, HF_WS_ABSORB = 3, HF_WS_SELECT_TWO_STAG
  * Returns (size_t)-1 for arguments the call would reject. Host-only, no CUDA call. */
 HF_API size_t hf_workspace_size(int which, int B, int H, int Nq, int Nk, int d, int block, int r);
 
-/* Bind S_dev / z_dev to *st and zero them (stream-ordered memset): the empty state.
- * Errors: HF_ERR_INVALID_ARG (st/S_dev/z_dev NULL, B/H < 1), HF_ERR_UNSUPPORTED (d),
- * HF_ERR_ALIGNMENT, HF_ERR_CUDA. */
-HF_API hf_status hf_state_init(hf_state* st, int B, int H, int d, float* S_dev, float* z_dev, void* stream);
+/* Bind S_dev / z_dev / S_split_dev to *st and zero them (stream-ordered memsets): the
+ * empty state. Errors: HF_ERR_INVALID_ARG (st/S_dev/z_dev/S_split_dev NULL, B/H < 1),
+ * HF_ERR_UNSUPPORTED (d), HF_ERR_ALIGNMENT, HF_ERR_CUDA. */
+HF_API hf_status hf_state_init(hf_state* st, int B, int H, int d, float* S_dev, float* z_dev, void* S_split_dev,
+                               void* stream);
 
 /* Absorb n_tokens evicted tokens per (b, h) into the state:
  *   S += phi(K_ev)^T V_ev, z += sum_t phi(K_ev[t])   (K_ev, V_ev: [B][H][n_tokens][d])

@@ -78,7 +78,7 @@ def test_select_validation():
 
 def _state(Bn=1, H=1, d=64):
     st = B.HfStateC()
-    st.B, st.H, st.d, st.S, st.z, st.n_absorbed = Bn, H, d, A, A, 0
+    st.B, st.H, st.d, st.S, st.z, st.S_split, st.n_absorbed = Bn, H, d, A, A, A, 0
     return st
 
 
@@ -110,10 +110,16 @@ def test_attention_validation():
 def test_state_and_absorb_validation():
     lib = hf.lib()
     st = B.HfStateC()
-    assert lib.hf_state_init(None, 1, 1, 64, A, A, None) == B.HF_ERR_INVALID_ARG
-    assert lib.hf_state_init(ctypes.byref(st), 1, 1, 32, A, A, None) == B.HF_ERR_UNSUPPORTED
-    assert lib.hf_state_init(ctypes.byref(st), 1, 1, 64, A + 4, A, None) == B.HF_ERR_ALIGNMENT
-    assert lib.hf_state_init(ctypes.byref(st), 0, 1, 64, A, A, None) == B.HF_ERR_INVALID_ARG
+    assert lib.hf_state_init(None, 1, 1, 64, A, A, A, None) == B.HF_ERR_INVALID_ARG
+    assert lib.hf_state_init(ctypes.byref(st), 1, 1, 32, A, A, A, None) == B.HF_ERR_UNSUPPORTED
+    assert lib.hf_state_init(ctypes.byref(st), 1, 1, 64, A + 4, A, A, None) == B.HF_ERR_ALIGNMENT
+    assert lib.hf_state_init(ctypes.byref(st), 1, 1, 64, A, A, A + 8, None) == B.HF_ERR_ALIGNMENT
+    assert lib.hf_state_init(ctypes.byref(st), 1, 1, 64, A, A, None, None) == B.HF_ERR_INVALID_ARG
+    assert lib.hf_state_init(ctypes.byref(st), 0, 1, 64, A, A, A, None) == B.HF_ERR_INVALID_ARG
+    s = _state()
+    s.S_split = None
+    assert lib.hf_absorb_evicted(ctypes.byref(s), A, A, 100, A, 1 << 30, None) == B.HF_ERR_INVALID_ARG
+    assert _fwd(st=s) == B.HF_ERR_INVALID_ARG
     s = _state()
     assert lib.hf_absorb_evicted(ctypes.byref(s), A, A, -1, A, 1 << 30, None) == B.HF_ERR_INVALID_ARG
     assert lib.hf_absorb_evicted(ctypes.byref(s), A, A, 0, None, 0, None) == B.HF_OK
@@ -290,7 +296,7 @@ def test_binding_checks_every_tensor_shape_before_any_call():
     with pytest.raises(ValueError, match="scores_out"):
         hf.hf_select_blocks_noalloc(Q, K, 32, 2, i32(1, 2, 4, 2), scores_out=torch.empty(1, 2, 4, 11))
     # attention: V, idx, O and the state against Q and K
-    st = hf.HfState(torch.empty(0), torch.empty(0))
+    st = hf.HfState(torch.empty(0), torch.empty(0), torch.empty(0, dtype=torch.uint8))
     st.c.B, st.c.H, st.c.d = 1, 2, 64
     V = torch.empty_like(K)
     idx = i32(1, 2, 4, 2)

@@ -128,6 +128,49 @@ def test_select_scores_differing_in_low_bits(nKB, r):
             assert np.array_equal(idx[0, h, I], want), (h, I)
 
 
+def _split_bytes(S):
+    """The state's split copy from S [B,H,d,d] fp32: per (b, h) the hi tile bf16(S), then the
+    lo tile bf16(S - hi), each d/64 chunks of 64 columns n, a chunk d rows k of 128 bytes,
+    16-byte group g of row k at position g ^ (k % 8)."""
+    B, H, d, _ = S.shape
+    hi = S.to(torch.bfloat16)
+    lo = (S - hi.float()).to(torch.bfloat16)
+    k = torch.arange(d).view(d, 1)
+    pos = torch.arange(8).view(1, 8)
+    g_at = pos ^ (k % 8)  # group stored at position pos of row k
+    tiles = []
+    for t in (hi, lo):
+        x = t.reshape(B * H, d, d // 64, 8, 8)                                   # [bh][k][c][g][e]
+        x = x[:, torch.arange(d).view(d, 1, 1), torch.arange(d // 64).view(1, -1, 1),
+              g_at.view(d, 1, 8)]                                              # [bh][k][c][pos][e]
+        tiles.append(x.permute(0, 2, 1, 3, 4).reshape(B * H, d * d))           # [bh][c][k][pos][e]
+    return torch.stack(tiles, dim=1).reshape(-1).view(torch.uint8)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_state_split_follows_S(d):
+    """The split copy kept beside the state equals bf16 hi / lo of S in the readout layout,
+    byte for byte: zero after hf_state_init, then after absorptions (separate and fused)."""
+    B, H = 1, 3
+    S = torch.empty(B, H, d, d, device=DEV)
+    z = torch.empty(B, H, d, device=DEV)
+    st = hf.hf_state_init(S, z)
+    torch.cuda.synchronize()
+    assert not st.S_split.any()
+    for seed, n in ((1, 300), (2, 64), (3, 1000)):
+        hf.hf_absorb_evicted(st, _gen(seed, B, H, n, d, w=0.5).to(DEV), _gen(seed + 10, B, H, n, d).to(DEV))
+        torch.cuda.synchronize()
+        assert torch.equal(st.S_split.cpu(), _split_bytes(st.S.cpu())), (seed, n)
+    Q = _gen(7, B, H, 128, d).to(DEV)
+    K = _gen(8, B, H, 512, d).to(DEV)
+    V = _gen(9, B, H, 512, d).to(DEV)
+    idx = hf.hf_select_blocks(Q, K, 128, 2)
+    hf.hf_hybrid_attn_fwd_absorb(Q, K, V, 128, 2, idx, st, K[:, :, :256].contiguous(), V[:, :, :256].contiguous())
+    torch.cuda.synchronize()
+    _check_status()
+    assert torch.equal(st.S_split.cpu(), _split_bytes(st.S.cpu()))
+
+
 # --------------------------------------------------------------------------- absorb
 @pytest.mark.parametrize("B,H,n,d", [(1, 1, 192, 64), (1, 2, 1000, 128), (2, 3, 77, 128), (1, 12, 4680, 128),
                                      (1, 1, 1, 64), (1, 40, 130, 64),
