@@ -46,7 +46,8 @@
 // [0, d_t), pairs (2i, 2i+1), the index of the row's frame); the MMA issuer and warp 3
 // wait for "turned" in place of "landed". The rings lose one V slot to make room.
 // Linear term, after the last block: phi(q) in fp32 split into bf16 hi + lo (TMEM, over
-// S_B), the state S split into bf16 hi + lo (shared memory, over the idle rings),
+// S_B); the state's S as bf16 hi + lo comes from the split copy kept beside the state
+// (bulk copies into the idle K ring, issued by the MMA thread once the last MMAs are done);
 // D_lin = phi_hi S_hi + phi_hi S_lo + phi_lo S_hi on the tensor cores (TMEM, over S_A),
 // denominator phi(q).z + 1e-6 in fp32; the epilogue writes
 // (w_A O_A + w_B O_B) / (w_A l_A + w_B l_B) + D_lin / den, w_p = 2^(m_p - max(m_A, m_B)).
