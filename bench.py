@@ -810,8 +810,19 @@ def streaming_e2e_leg(hf, wl, dev, stream, x, st, ws_sel, ws_abs, args, dist) ->
     t = max_over_ranks(e0.elapsed_time(e1) * 1e-3 / n_e2e, dist, dev)
     world = dist.get_world_size() if dist else 1
     nbytes = 2 * B * H * Nq * d
+    # the link alone: the same three host-to-device copies per step, nothing else
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(up)
+    for j in range(n_e2e):
+        with torch.cuda.stream(up):
+            for i in range(3):
+                dev_in[j % 2][i].copy_(host_in[i], non_blocking=True)
+    c1.record(up)
+    torch.cuda.synchronize(dev)
+    t_copy = c0.elapsed_time(c1) * 1e-3 / n_e2e
     return {"value": job_throughput(world, B, Nq, t), "unit": UNIT, "h2d_bytes_per_step": 3 * nbytes,
             "d2h_bytes_per_step": nbytes, "steps": n_e2e, "ms_per_step": t * 1e3,
+            "h2d_gbs": 3 * nbytes / t / 1e9, "h2d_copies_alone_gbs": 3 * nbytes / t_copy / 1e9,
             "note": "streaming: per step the chunk's Q, K, V (4680 tokens) in from pinned host memory on an upload "
                     "stream overlapping the previous step, window shift on the device, select, attention + "
                     "absorption of the chunk leaving the window (one call), O out to pinned host memory"}

@@ -224,11 +224,16 @@ def hf_workspace_size(which: int, B: int, H: int, Nq: int, Nk: int, d: int, bloc
     return int(n)
 
 
-def _workspace(nbytes: int, device, ws):
+def _workspace(nbytes: int, device, ws, stream=None):
+    """The caller's workspace, or a new one; a new one used on another torch stream than the
+    current one is recorded on it, so that the allocator does not hand its memory out again
+    before that stream's work is done."""
     if nbytes == 0:
         return None, 0
     if ws is None:
         ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        if isinstance(stream, torch.cuda.Stream) and stream != torch.cuda.current_stream(ws.device):
+            ws.record_stream(stream)
     return ws, ws.numel() * ws.element_size()
 
 
@@ -256,7 +261,7 @@ def hf_absorb_evicted(state: HfState, K_ev: torch.Tensor, V_ev: torch.Tensor, ws
         raise ValueError("K_ev and V_ev must both be [B,H,n,d] matching the state")
     n = K_ev.shape[2]
     nbytes = hf_workspace_size(HF_WS_ABSORB, B, H, 0, n, d, 0, 0)
-    ws, ws_bytes = _workspace(nbytes, K_ev.device, ws)
+    ws, ws_bytes = _workspace(nbytes, K_ev.device, ws, stream)
     _check(lib().hf_absorb_evicted(ctypes.byref(state.c), _dev(K_ev, torch.bfloat16, "K_ev"),
                                    _dev(V_ev, torch.bfloat16, "V_ev"), n,
                                    ws.data_ptr() if ws is not None else None, ws_bytes, _stream(stream)),
@@ -273,7 +278,7 @@ def hf_select_blocks(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, idx_o
     if idx_out is None:
         idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
     nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, Nk, d, block, r)
-    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws, stream)
     _check(lib().hf_select_blocks(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), B, H, Nq, Nk, d,
                                   block, r, _dev(idx_out, torch.int32, "idx_out"),
                                   _dev(scores_out, torch.float32, "scores_out") if scores_out is not None else None,
@@ -294,7 +299,7 @@ def hf_select_blocks_rope(Q: torch.Tensor, K: torch.Tensor, block: int, r: int, 
     if idx_out is None:
         idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
     nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, Nk, d, block, r)
-    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws, stream)
     _check(lib().hf_select_blocks_rope(_dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), B, H, Nq, Nk, d,
                                        block, r, ctypes.byref(rope), _dev(idx_out, torch.int32, "idx_out"),
                                        _dev(scores_out, torch.float32, "scores_out")
@@ -342,7 +347,7 @@ def hf_select_blocks_cached(Q: torch.Tensor, kp: HfKpool, block: int, r: int, id
     if idx_out is None:
         idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
     nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, max(Nk, 1), d, block, 1)
-    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws, stream)
     _check(lib().hf_select_blocks_cached(_dev(Q, torch.bfloat16, "Q"), ctypes.byref(kp.c), Nq, block, r,
                                          _dev(idx_out, torch.int32, "idx_out"),
                                          _dev(scores_out, torch.float32, "scores_out")
@@ -371,7 +376,7 @@ def hf_select_blocks_cached_push(Q: torch.Tensor, kp: HfKpool, K_new, block: int
     if idx_out is None:
         idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
     nbytes = hf_workspace_size(HF_WS_SELECT, B, H, Nq, max(Nk, 1), d, block, 1)
-    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws, stream)
     _check(lib().hf_select_blocks_cached_push(_dev(Q, torch.bfloat16, "Q"), ctypes.byref(kp.c),
                                               _dev(K_new, torch.bfloat16, "K_new") if n > 0 else None, n,
                                               int(n_evict), Nq, block, r, _dev(idx_out, torch.int32, "idx_out"),
@@ -395,7 +400,7 @@ def hf_select_blocks_two_stage(Q: torch.Tensor, K: torch.Tensor, block: int, r: 
     if idx_out is None:
         idx_out = torch.empty(B, H, nQB, r, dtype=torch.int32, device=Q.device)
     nbytes = hf_workspace_size(HF_WS_SELECT_TWO_STAGE, B, H, Nq, Nk, d, block, r)
-    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws, stream)
     _check(lib().hf_select_blocks_two_stage(
         _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), B, H, Nq, Nk, d, block, r, tokens_per_frame,
         n_frames, _dev(idx_out, torch.int32, "idx_out"),
@@ -505,7 +510,7 @@ def hf_hybrid_attn_fwd_absorb(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
     if O is None:
         O = torch.empty_like(Q)
     nbytes = hf_workspace_size(HF_WS_ABSORB, B, H, 0, n, d, 0, 0)
-    ws, ws_bytes = _workspace(nbytes, Q.device, ws)
+    ws, ws_bytes = _workspace(nbytes, Q.device, ws, stream)
     _check(lib().hf_hybrid_attn_fwd_absorb(
         _dev(Q, torch.bfloat16, "Q"), _dev(K, torch.bfloat16, "K"), _dev(V, torch.bfloat16, "V"), B, H, Nq, Nk, d,
         block, r, _dev(idx, torch.int32, "idx"), ctypes.byref(state.c), float(scale), _dev(O, torch.bfloat16, "O"),

@@ -559,6 +559,48 @@ def test_bench_step_sequence_on_device_drawn_inputs():
     assert n == wl.B * wl.H * wl.nQB
 
 
+def test_absorb_beside_next_selection_equals_sequential_steps():
+    """A step's absorption on a second stream beside the next step's selection (which does
+    not read the state), the next attention waiting for it, gives step after step
+    bit-identically the outputs and the state of the sequential select -> attention ->
+    absorb: the calls are safe on any stream, their workspaces included."""
+    wl = WORKLOADS["832x480"]
+    x = draw_step_inputs(wl, seed=321, n_evicted=wl.Ne_step, device=DEV)
+    Q, K, V, K_ev, V_ev = x["Q"], x["K"], x["V"], x["K_ev"], x["V_ev"]
+    states, outs = [], []
+    for _ in range(2):
+        S = torch.empty(wl.B, wl.H, wl.d, wl.d, device=DEV)
+        z = torch.empty(wl.B, wl.H, wl.d, device=DEV)
+        states.append(hf.hf_state_init(S, z))
+        outs.append([])
+    stream, side = torch.cuda.current_stream(), torch.cuda.Stream()
+    absorbed = torch.cuda.Event()
+    idx = torch.empty(wl.B, wl.H, wl.nQB, wl.r, dtype=torch.int32, device=DEV)
+    idx2 = torch.empty_like(idx)
+    for k in range(4):
+        # sequential
+        hf.hf_select_blocks(Q, K, wl.block, wl.r, idx_out=idx)
+        outs[0].append(hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wl.r, idx, states[0]))
+        hf.hf_absorb_evicted(states[0], K_ev, V_ev)
+        # overlapped: step k absorbs step k-1's frames beside its selection
+        side.wait_stream(stream)
+        if k > 0:
+            hf.hf_absorb_evicted(states[1], K_ev, V_ev, stream=side)
+        absorbed.record(side)
+        hf.hf_select_blocks(Q, K, wl.block, wl.r, idx_out=idx2)
+        stream.wait_event(absorbed)
+        outs[1].append(hf.hf_hybrid_attn_fwd(Q, K, V, wl.block, wl.r, idx2, states[1]))
+    side.wait_stream(stream)
+    hf.hf_absorb_evicted(states[1], K_ev, V_ev, stream=side)
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    _check_status()
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+    assert torch.equal(states[0].S, states[1].S) and torch.equal(states[0].z, states[1].z)
+    assert torch.equal(states[0].S_split, states[1].S_split)
+
+
 # --------------------------------------------------------------------------- fused step
 @pytest.mark.parametrize("B,H,Nq,Nk,d,block,r,n_state,n_ev", [
     (1, 1, 64, 256, 64, 32, 2, 192, 192),       # the tiny workload's shape
