@@ -30,7 +30,7 @@
 //               is accumulated in fp32 registers. They also drain the accumulator: the
 //               tensor core's fp32 accumulation truncates, so a long chain of MMAs into one
 //               TMEM accumulator drifts (relative error grows with the chain length, ~2e-5
-//               after 500 MMAs). The MMAs of every group of kAbsGroup tiles (256 tokens)
+//               after 500 MMAs). The MMAs of every group of kAbsGroup tiles (512 tokens)
 //               therefore go to one of two TMEM accumulators, which the converters add into
 //               fp32 registers with round-to-nearest while the other one fills; the four
 //               warps that share a TMEM lane quarter (rows n) take a quarter of the k
@@ -55,7 +55,7 @@ constexpr int kAbsTok = 64;        // tokens per tile
 constexpr int kAbsMaxStages = 8;   // ring depth cap
 constexpr int kConvThreads = 512;  // converter warps 2..17
 constexpr int kAbsThreads = 64 + kConvThreads;
-constexpr int kAbsGroup = 4;       // tiles per TMEM accumulation chain
+constexpr int kAbsGroup = 8;       // tiles per TMEM accumulation chain
 
 template <int D>
 struct AbsorbCfg {
