@@ -94,12 +94,12 @@ def test_cached_select_832x480_window():
     _check(Q, moved, kp, wl.block, wl.r)
 
 
-def test_cached_push_equals_push_then_select():
+@pytest.mark.parametrize("d,G,block,W,step", [(128, 8, 64, 640, 200), (64, 4, 32, 512, 100)])
+def test_cached_push_equals_push_then_select(d, G, block, W, step):
     """hf_select_blocks_cached_push (the push's sums computed in the Q pooling launch) gives
     the same ring, blocks and scores, bit for bit, as hf_kpool_push then
     hf_select_blocks_cached, step after step of a moving window that wraps its ring."""
-    B, H, d, G, block, r = 2, 3, 128, 8, 64, 3
-    W, step = 640, 200
+    B, H, r = 2, 3, 3
     keys = _gen(21, B, H, W + 6 * step, d).to(DEV)
     sums_a = torch.zeros(B, H, W // G + 5, d, dtype=torch.float32, device=DEV)
     sums_b = torch.zeros_like(sums_a)
