@@ -56,6 +56,7 @@ constexpr int kAbsMaxStages = 8;   // ring depth cap
 constexpr int kConvThreads = 512;  // converter warps 2..17
 constexpr int kAbsThreads = 64 + kConvThreads;
 constexpr int kAbsGroup = 8;       // tiles per TMEM accumulation chain
+constexpr int kConvGroups = 2;     // converter groups; group g converts the tiles i with i % 2 == g
 
 template <int D>
 struct AbsorbCfg {
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
-      mbar_init(&bfull_bar[s], kConvThreads / 32);
+      mbar_init(&bfull_bar[s], kConvThreads / 32 / kConvGroups);  // the converting group's warps
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&dfull_bar[b], 1);
@@ -205,10 +206,18 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
     // ---------------- converters + epilogue (512 threads) ----------------
     const int t = threadIdx.x - 64;
     constexpr int kUnits = D / 8;    // 16-byte units per row
-    constexpr int kPhases = kConvThreads / kUnits;
-    constexpr int kRowsPerThread = kAbsTok / kPhases;
+    constexpr int kPhases = kConvThreads / kUnits;  // (over both groups, for the z reduction)
+    constexpr int kGroupThreads = kConvThreads / kConvGroups;
+    constexpr int kGPhases = kGroupThreads / kUnits;
+    constexpr int kRowsPerThread = kAbsTok / kGPhases;
+    static_assert(kGPhases % 8 == 0, "a thread's rows share their swizzle phase");
+    // each ring stage serves one group only, so a group waits on a stage's phases in order
+    static_assert(NS % kConvGroups == 0, "ring stages per converter group");
+    // The two groups convert alternate tiles, so that one group's arithmetic overlaps the
+    // other's waits and the tile stream; all converter warps drain the accumulators.
+    const int cgroup = t / kGroupThreads;
     const int ucol = t % kUnits;     // logical unit column: elements [8*ucol, 8*ucol + 8)
-    const int phase = t / kUnits;    // rows phase, phase + kPhases, ...
+    const int phase = (t % kGroupThreads) / kUnits;  // rows phase, phase + kGPhases, ...
     const int chunk = ucol / 8;
     const uint32_t swz = static_cast<uint32_t>(((ucol % 8) ^ (phase & 7)) * 16);
     uint64_t zacc[4] = {0ull, 0ull, 0ull, 0ull};  // fp32 pairs: elements (2e, 2e+1) of the unit
@@ -270,7 +279,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       f32x2_split(ffma2(f32x2(bf16_lo_to_f32(hi), bf16_hi_to_f32(hi)), f32x2(-1.0f, -1.0f), pp), r0, r1);
       lo = pack_bf16x2(r0, r1);
     };
-    for (int i = 0; i < ntiles && ok; ++i) {
+    for (int i = cgroup; i < ntiles && ok; i += kConvGroups) {
       const int s = i % NS;
       ok = __all_sync(0xffffffffu,
                       mbar_wait(&full_bar[s], (i / NS) & 1, abort_flag, p.timeout_ns, (kKernAbsorb << 8) | 6));
@@ -279,7 +288,7 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       const int valid = min(kAbsTok, p.n_tokens - (tile0 + i) * kAbsTok);
 #pragma unroll
       for (int k = 0; k < kRowsPerThread; ++k) {
-        const int row = phase + k * kPhases;
+        const int row = phase + k * kGPhases;
         const uint32_t off = chunk * C::kChunkBytes + row * 128 + swz;
         const uint4 kv = *reinterpret_cast<const uint4*>(stage + C::kKOff + off);
         uint32_t hi[4], lo[4];
@@ -300,10 +309,10 @@ __global__ void __launch_bounds__(kAbsThreads, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bfull_bar[s]);
-      // once group g is fully converted, drain group g - 1 (one group of lag keeps the
-      // tensor core busy on the other accumulator)
+      // once this thread's share of group g is converted, drain group g - 1 (one group of lag
+      // keeps the tensor core busy on the other accumulator)
       const int g = i / kAbsGroup;
-      const bool group_done = (i % kAbsGroup) == kAbsGroup - 1 || i == ntiles - 1;
+      const bool group_done = (i + kConvGroups) / kAbsGroup != g || i + kConvGroups >= ntiles;
       if (group_done && g >= 1) {
         ok = flush_group(g - 1);
         flushed = g;
